@@ -1,0 +1,15 @@
+"""CPU oracle (test infrastructure only; see :mod:`oracle.glmq_oracle`)."""
+from .glmq_oracle import (  # noqa: F401
+    divisor,
+    row_absmax,
+    row_scale,
+    quantize_rows,
+    pack_int4,
+    pack,
+    quantize_linear,
+    unpack,
+    dequantize,
+    linear_forward,
+    linear_forward_rows,
+    relative_max_error,
+)

@@ -1,0 +1,22 @@
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+
+def pytest_configure(config):
+    config.addinivalue_line("markers", "gpu: needs a CUDA GPU (sm_100a) and the built library")
+    config.addinivalue_line("markers", "slow: long CPU-only check, enabled with GLMQ_SLOW=1")
+
+
+def pytest_collection_modifyitems(config, items):
+    if os.environ.get("GLMQ_SLOW") == "1":
+        return
+    skip = pytest.mark.skip(reason="slow check; set GLMQ_SLOW=1")
+    for item in items:
+        if "slow" in item.keywords:
+            item.add_marker(skip)

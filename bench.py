@@ -1,0 +1,550 @@
+#!/usr/bin/env python
+"""Benchmark of the GLM-130B weight-only INT4 decode GEMM (and friends) on B200.
+
+Default workload ("decode"): GLM-130B layer shapes QKV 12288->36864, attn-out
+12288->12288, FFN-up 12288->65536 (GeGLU gate+value), FFN-down 32768->12288;
+W ~ N(0, 0.02) fp16 quantized once to INT4 (one-shot, timed separately), X ~ N(0, 1)
+fp16. One step = the decode GEMM for M in {1, 4, 16} on all four projections
+(12 launches of glmq_gemm, weights resident in HBM). Metric: packed-weight GB/s
+(decimal GB) over the step, plus the roofline of the decode kernel.
+
+Other workloads: "sweep" (70 layers x 4 projections INT4-resident, one-shot
+quantization layer by layer, then M=1 decode through all 280 projections in a
+CUDA graph, tokens/s).
+
+Timing: W >= 3 warm-up steps; K timed steps bracketed by a barrier and
+torch.cuda.synchronize(); CUDA events on the launching stream; the max over
+ranks. The step's working set (906 MB of packed weights) is larger than the
+126 MB L2, so no separate flush is needed between steps.
+
+`--impl reference` times the CPU oracle (the only reference this method has)
+on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "W4A16 GEMM weight GB/s (decode) and TFLOP/s (prefill) vs B200 roofline"
+HIDDEN = 12288
+DECODE_MS = (1, 4, 16)
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+# ----------------------------------------------------------------------------- helpers
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": FALLBACK_HBM_GBS, "bf16_tflops": FALLBACK_BF16_TFLOPS,
+                "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def source_digest() -> str:
+    csrc = os.path.join(ROOT, "int8_quantized_glmq_b200", "csrc")
+    h = hashlib.sha256()
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(f.encode())
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profile_traffic_ratio(kernel_tag: str):
+    """DRAM traffic / algorithmic bytes recorded by an ncu capture of this exact source, or None."""
+    path = os.path.join(ROOT, "profiles", f"{kernel_tag}.md")
+    if not os.path.exists(path):
+        return None
+    ratio, digest = None, None
+    with open(path) as f:
+        for line in f:
+            if line.startswith("source_digest:"):
+                digest = line.split(":", 1)[1].strip()
+            if line.startswith("traffic_over_algorithmic:"):
+                ratio = float(line.split(":", 1)[1].strip())
+    if digest != source_digest():
+        return None
+    return ratio
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples during the timed region."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        import tempfile
+        try:
+            fd, self.path = tempfile.mkstemp(prefix="glmq_clocks_", suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.15)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def dist_setup():
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------- workloads
+def make_weights(torch, seed_base: int):
+    """fp16 GLM-130B projection weights ~ N(0, 0.02), generated on the device (seeded)."""
+    from inputs import GLM_PROJECTIONS, PROJECTION_ORDER
+    out = {}
+    for i, name in enumerate(PROJECTION_ORDER):
+        N, K = GLM_PROJECTIONS[name]
+        g = torch.Generator(device="cuda").manual_seed(seed_base + i)
+        w = torch.empty((N, K), dtype=torch.float16, device="cuda")
+        w.normal_(0.0, 0.02, generator=g)
+        out[name] = w
+    return out
+
+
+def time_launches(torch, fn, iters: int, warmup: int = 2):
+    """Average device time of fn() per call, CUDA events on the current stream."""
+    for _ in range(warmup):
+        fn()
+    s = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(s)
+    for _ in range(iters):
+        fn()
+    e1.record(s)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / 1e3 / iters
+
+
+def run_decode(args, world, rank, local):
+    import torch
+    import int8_quantized_glmq_b200 as glmq
+    from inputs import GLM_PROJECTIONS, PROJECTION_ORDER
+
+    peaks = measured_peaks()
+    torch.manual_seed(0)
+    W16 = make_weights(torch, 1000)
+    bits = 4
+    # one-shot quantization (timed separately: not part of the decode step)
+    quant = {}
+    qstats = {}
+    for name in PROJECTION_ORDER:
+        N, K = GLM_PROJECTIONS[name]
+        packed = torch.empty((N, K // 2), dtype=torch.uint8, device="cuda")
+        scale = torch.empty((N,), dtype=torch.float16, device="cuda")
+        quant[name] = (packed, scale)
+        t = time_launches(torch, lambda: glmq.quantize(W16[name], bits, out=(packed, scale)), 5)
+        qbytes = N * K * 2 + N * K // 2 + N * 2
+        qstats[name] = {"us": t * 1e6, "gbs": qbytes / t / 1e9}
+    extras = {}
+    if not args.no_extras:
+        extras = run_extras(torch, glmq, W16, quant, peaks)
+    del W16
+    torch.cuda.empty_cache()
+
+    # activations for the decode step
+    xs = {}
+    for M in DECODE_MS:
+        for name in PROJECTION_ORDER:
+            N, K = GLM_PROJECTIONS[name]
+            g = torch.Generator(device="cuda").manual_seed(2000 + M)
+            xs[(M, name)] = torch.randn((M, K), generator=g, device="cuda", dtype=torch.float32).half()
+    ys = {(M, name): torch.empty((M, GLM_PROJECTIONS[name][0]), dtype=torch.float16, device="cuda")
+          for M in DECODE_MS for name in PROJECTION_ORDER}
+    launches = [(M, name) for M in DECODE_MS for name in PROJECTION_ORDER]
+    weight_bytes = sum(quant[n][0].numel() for (_, n) in launches)
+    alg_bytes = sum(quant[n][0].numel() + quant[n][1].numel() * 2 + xs[(M, n)].numel() * 2 + ys[(M, n)].numel() * 2
+                    for (M, n) in launches)
+
+    def step():
+        for (M, n) in launches:
+            glmq.gemm(xs[(M, n)], quant[n][0], quant[n][1], bits, out=ys[(M, n)])
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    # per-launch timing of the dominant kernel (decode), measured inside the timed region
+    stream = torch.cuda.current_stream()
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in launches]
+          for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier(world)
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for it in range(args.steps):
+        for j, (M, n) in enumerate(launches):
+            ev[it][j][0].record(stream)
+            glmq.gemm(xs[(M, n)], quant[n][0], quant[n][1], bits, out=ys[(M, n)])
+            ev[it][j][1].record(stream)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    elapsed = t0.elapsed_time(t1) / 1e3
+    per_launch_s = [sum(ev[it][j][0].elapsed_time(ev[it][j][1]) for it in range(args.steps)) / 1e3 / args.steps
+                    for j in range(len(launches))]
+    elapsed_max = max_over_ranks(elapsed, world)
+    value = world * weight_bytes * args.steps / elapsed_max / 1e9
+
+    # e2e through the public API: pinned host X in, pinned host Y out, every step
+    hx = {k: v.cpu().pin_memory() for k, v in xs.items()}
+    hy = {k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in ys.items()}
+    h2d = sum(v.numel() * 2 for v in hx.values())
+    d2h = sum(v.numel() * 2 for v in hy.values())
+
+    def e2e_step():
+        for (M, n) in launches:
+            xd = hx[(M, n)].to("cuda", non_blocking=True)
+            y = glmq.gemm(xd, quant[n][0], quant[n][1], bits)
+            hy[(M, n)].copy_(y, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    barrier(world)
+    torch.cuda.synchronize()
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    a1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_elapsed = max_over_ranks(a0.elapsed_time(a1) / 1e3, world)
+    e2e_value = world * weight_bytes * args.steps / e2e_elapsed / 1e9
+
+    kern_time = sum(per_launch_s)
+    achieved = alg_bytes / kern_time / 1e9
+    ratio = profile_traffic_ratio("decode_int4_glm_shapes")
+    roofline = {"kernel": "decode_kernel (INT4, M in {1,4,16})", "bound": "hbm", "achieved": round(achieved, 1),
+                "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+                "peak_source": peaks["source"],
+                "traffic": (round(ratio * alg_bytes / len(launches)) if ratio else None),
+                "algorithmic_bytes_per_launch": round(alg_bytes / len(launches))}
+    per_launch = {f"{n}/M={M}": {"us": round(per_launch_s[j] * 1e6, 2),
+                                 "gbs": round((quant[n][0].numel() + quant[n][1].numel() * 2 + xs[(M, n)].numel() * 2
+                                               + ys[(M, n)].numel() * 2) / per_launch_s[j] / 1e9, 1)}
+                  for j, (M, n) in enumerate(launches)}
+    extras["decode_per_launch"] = per_launch
+    extras["quantize_int4"] = {k: {"us": round(v["us"], 1), "gbs": round(v["gbs"], 1)} for k, v in qstats.items()}
+    return {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(elapsed_max / args.steps * 1e3, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "fp16", "weight_dtype": "int4", "data": "synthetic",
+        "config": {"workload": "decode GEMV on GLM-130B layer shapes (QKV 12288->36864, attn-out 12288->12288, "
+                               "FFN-up 12288->65536, FFN-down 32768->12288), M in {1,4,16}, INT4 weights",
+                   "global_batch": list(DECODE_MS), "parallelism": f"replicas x{world}" if world > 1 else "1 GPU",
+                   "weights": "N(0,0.02) fp16 on device, quantized once to INT4 (not in the step)",
+                   "activations": "N(0,1) fp16",
+                   "l2": "step working set 906 MB of packed weights > 126 MB L2 (no flush needed)"},
+        "roofline": roofline,
+        "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": len(launches) * args.steps,
+        "clocks": clk,
+        "extras": extras,
+    }
+
+
+def run_extras(torch, glmq, W16, quant, peaks):
+    """Short, separately timed numbers: quantize roofline, prefill TFLOP/s, INT8."""
+    from inputs import GLM_PROJECTIONS, PROJECTION_ORDER
+    out = {"prefill_int4_m2048": {}, "int8": {}}
+    for name in PROJECTION_ORDER:
+        N, K = GLM_PROJECTIONS[name]
+        packed, scale = quant[name]
+        g = torch.Generator(device="cuda").manual_seed(3000)
+        X = torch.randn((2048, K), generator=g, device="cuda", dtype=torch.float32).half()
+        Y = torch.empty((2048, N), dtype=torch.float16, device="cuda")
+        t = time_launches(torch, lambda: glmq.gemm(X, packed, scale, 4, out=Y), 5)
+        tf = 2.0 * 2048 * N * K / t / 1e12
+        out["prefill_int4_m2048"][name] = {"us": round(t * 1e6, 1), "tflops": round(tf, 1),
+                                           "frac_burst": round(tf / peaks["bf16_tflops"], 4)}
+        del X, Y
+    for name in PROJECTION_ORDER:
+        N, K = GLM_PROJECTIONS[name]
+        p8 = torch.empty((N, K), dtype=torch.uint8, device="cuda")
+        s8 = torch.empty((N,), dtype=torch.float16, device="cuda")
+        tq = time_launches(torch, lambda: glmq.quantize(W16[name], 8, out=(p8, s8)), 3)
+        res = {"quantize_us": round(tq * 1e6, 1), "quantize_gbs": round((N * K * 3 + N * 2) / tq / 1e9, 1)}
+        for M in (1, 64, 2048):
+            g = torch.Generator(device="cuda").manual_seed(4000 + M)
+            X = torch.randn((M, K), generator=g, device="cuda", dtype=torch.float32).half()
+            Y = torch.empty((M, N), dtype=torch.float16, device="cuda")
+            t = time_launches(torch, lambda: glmq.gemm(X, p8, s8, 8, out=Y), 5)
+            res[f"M={M}"] = {"us": round(t * 1e6, 1), "weight_gbs": round(N * K / t / 1e9, 1),
+                             "tflops": round(2.0 * M * N * K / t / 1e12, 1)}
+        out["int8"][name] = res
+        del p8, s8
+    return out
+
+
+# ----------------------------------------------------------------------------- reference arm
+def run_reference(args, world, rank):
+    """The CPU oracle, as it stands, on a bounded sample of the decode workload."""
+    import numpy as np
+    import oracle
+    from inputs import GLM_PROJECTIONS, PROJECTION_ORDER, decode_activations, projection_weight
+
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        cores = os.cpu_count() or 1
+    rows = 256  # sampled output features per projection per step
+    samples = {}
+    for i, name in enumerate(PROJECTION_ORDER):
+        N, K = GLM_PROJECTIONS[name]
+        W = projection_weight(name, seed=1000 + i, rows=slice(0, rows))
+        samples[name] = oracle.quantize_linear(W, 4)
+    xs = {(M, n): decode_activations(M, GLM_PROJECTIONS[n][1], 2000 + M) for M in DECODE_MS for n in PROJECTION_ORDER}
+
+    def step():
+        for M in DECODE_MS:
+            for n in PROJECTION_ORDER:
+                p, s = samples[n]
+                oracle.linear_forward(xs[(M, n)], p, s, 4)
+
+    for _ in range(args.warmup):
+        step()
+    t = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    el = time.perf_counter() - t
+    wbytes = sum(samples[n][0].nbytes for n in PROJECTION_ORDER) * len(DECODE_MS)
+    value = wbytes * args.steps / el / 1e9
+    sample = (f"{rows} output rows of each projection (of 12288..65536), M in {{1,4,16}}, INT4, "
+              "oracle float64 dequantizing linear")
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(el / args.steps * 1e3, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "decode GEMV on GLM-130B layer shapes, M in {1,4,16}, INT4 weights (sampled rows)"},
+            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def cpu_baseline(budget_s: float = 12.0):
+    """Oracle timing on the host cores for the cpu_baseline key (rank 0, N=1)."""
+    import numpy as np
+    import oracle
+    from inputs import GLM_PROJECTIONS, decode_activations, projection_weight
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        cores = os.cpu_count() or 1
+    N, K = GLM_PROJECTIONS["qkv"]
+    rows = 2048
+    W = projection_weight("qkv", seed=1000, rows=slice(0, rows))
+    packed, s = oracle.quantize_linear(W, 4)
+    X = decode_activations(1, K, 2001)
+    t0 = time.perf_counter()
+    n = 0
+    while time.perf_counter() - t0 < budget_s:
+        oracle.linear_forward(X, packed, s, 4)
+        n += 1
+    el = time.perf_counter() - t0
+    return {"value": round(packed.nbytes * n / el / 1e9, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": f"QKV decode M=1, {rows} of 36864 output rows x K=12288, INT4, repeated {n}x for {el:.1f} s"}
+
+
+# ----------------------------------------------------------------------------- sweep
+def run_sweep(args, world, rank, local):
+    """70 layers x 4 projections resident as INT4; M=1 decode through all 280 in one CUDA graph."""
+    import torch
+    import int8_quantized_glmq_b200 as glmq
+    from inputs import GLM_PROJECTIONS, PROJECTION_ORDER
+
+    layers = args.layers
+    bits = 4
+    quant = []
+    qtime = 0.0
+    qbytes = 0
+    wbuf = {n: torch.empty(GLM_PROJECTIONS[n], dtype=torch.float16, device="cuda") for n in PROJECTION_ORDER}
+    s = torch.cuda.current_stream()
+    for layer in range(layers):
+        row = []
+        for p, n in enumerate(PROJECTION_ORDER):
+            N, K = GLM_PROJECTIONS[n]
+            g = torch.Generator(device="cuda").manual_seed(10000 + 4 * layer + p)
+            wbuf[n].normal_(0.0, 0.02, generator=g)
+            packed = torch.empty((N, K // 2), dtype=torch.uint8, device="cuda")
+            scale = torch.empty((N,), dtype=torch.float16, device="cuda")
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(s)
+            glmq.quantize(wbuf[n], bits, out=(packed, scale))
+            e1.record(s)
+            torch.cuda.synchronize()
+            qtime += e0.elapsed_time(e1) / 1e3
+            qbytes += N * K * 2 + N * K // 2 + N * 2
+            row.append((packed, scale))
+        quant.append(row)
+    del wbuf
+    torch.cuda.empty_cache()
+    xs = {n: torch.randn((1, GLM_PROJECTIONS[n][1]), device="cuda").half() for n in PROJECTION_ORDER}
+    ys = {n: torch.empty((1, GLM_PROJECTIONS[n][0]), dtype=torch.float16, device="cuda") for n in PROJECTION_ORDER}
+    cs = torch.cuda.Stream()
+    cs.wait_stream(s)
+    with torch.cuda.stream(cs):
+        for _ in range(2):
+            for layer in range(layers):
+                for p, n in enumerate(PROJECTION_ORDER):
+                    glmq.gemm(xs[n], quant[layer][p][0], quant[layer][p][1], bits, out=ys[n])
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=cs):
+        for layer in range(layers):
+            for p, n in enumerate(PROJECTION_ORDER):
+                glmq.gemm(xs[n], quant[layer][p][0], quant[layer][p][1], bits, out=ys[n])
+    for _ in range(args.warmup):
+        graph.replay()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier(world)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s)
+    for _ in range(args.steps):
+        graph.replay()
+    e1.record(s)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    el = max_over_ranks(e0.elapsed_time(e1) / 1e3, world)
+    wbytes = sum(q[0].numel() for row in quant for q in row)
+    tok_s = world * args.steps / el
+    peaks = measured_peaks()
+    gbs = wbytes * args.steps / (el) / 1e9
+    del graph
+    return {"metric": "GLM-130B 70-layer INT4 decode sweep (M=1, 280 projections), tokens/s", "value": round(tok_s, 2),
+            "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(el / args.steps * 1e3, 4), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "fp16", "weight_dtype": "int4", "data": "synthetic",
+            "config": {"workload": f"{layers}-layer GLM-130B projection sweep, M=1, CUDA graph of {4 * layers} launches",
+                       "packed_weight_bytes": wbytes, "l2": "63 GB working set >> L2"},
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": None},
+            "quantize_all_layers": {"ms": round(qtime * 1e3, 2), "gbs": round(qbytes / qtime / 1e9, 1)},
+            "gpu_launches": 4 * layers * args.steps, "clocks": clk}
+
+
+# ----------------------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="decode", choices=["decode", "sweep"])
+    ap.add_argument("--layers", type=int, default=70)
+    ap.add_argument("--no-extras", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        if rank != 0:
+            return
+        print(json.dumps(run_reference(args, world, rank)), flush=True)
+        return
+
+    world, rank, local = dist_setup()
+    if args.workload == "sweep":
+        res = run_sweep(args, world, rank, local)
+    else:
+        res = run_decode(args, world, rank, local)
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            res["cpu_baseline"] = cpu_baseline()
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

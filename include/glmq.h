@@ -1,0 +1,139 @@
+/*
+ * glmq: weight-only INT4 / INT8 quantization and the dequantizing linear layer
+ * (W4A16 / W8A16) for GLM-130B projection shapes, on NVIDIA B200 (sm_100a).
+ *
+ * The operations are those of the GLM-130B paper's weight-only quantization
+ * ("GLM-130B: An Open Bilingual Pre-trained Model"):
+ *   - wikillm.com paper card, "Method": every output row of a linear layer gets
+ *     one scale, its absolute maximum divided by 7; weights are rounded to
+ *     integers in [-7, 7], two INT4 values per byte; at run time the weights are
+ *     dequantized (quant * scale[:, None]) and multiplied by FP16 activations.
+ *   - same card, "Paper vs code", quantization-scale bullet: the divisor is
+ *     2^(b-1) - 1 (7 for INT4, 127 for INT8) and the scale is computed per
+ *     output row in FP16.
+ *   - paperlayer.ai summary, "INT4 Quantization for RTX 3090s/2080s": only the
+ *     linear-layer weights are quantized, activations stay FP16 and weights are
+ *     converted to FP16 at run time.
+ *
+ * Readings this library fixes where the pages are silent:
+ *   scale  s[n] = fp16_rn( fp32(max_k |W[n,k]|) / d ),  d = 7 (INT4) or 127 (INT8)
+ *   code   q[n,k] = clamp( round_half_even( fp32(W[n,k]) / fp32(s[n]) ), -d, d ),
+ *          and q[n,:] = 0 on a row whose scale rounds to 0
+ *   INT4   byte j of row n = (q[n,2j] & 0xF) | ((q[n,2j+1] & 0xF) << 4)
+ *          (low nibble = even k, 4-bit two's complement; 0x8 never occurs)
+ *   INT8   byte k of row n = q[n,k] as a two's-complement int8
+ *   linear Y[m,n] = fp16_rn( s[n] * sum_k X[m,k] * q[n,k] ), products exact,
+ *          sum accumulated in fp32 (the scale factors out of the k-sum).
+ *
+ * Conventions for every entry point:
+ *   - All tensors are dense, row-major, in DEVICE memory of the current CUDA
+ *     device, allocated and owned by the caller; the library never allocates,
+ *     frees or retains them. Every pointer must be 16-byte aligned.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *     stream). Calls only enqueue work on that stream and return without
+ *     synchronizing; results are visible after the stream reaches that point.
+ *   - Arguments are validated before anything is enqueued; a call that returns
+ *     an error status has enqueued nothing. No entry point aborts or throws.
+ *   - Shapes: N >= 0 rows (out_features), K in_features with K > 0,
+ *     K % 64 == 0 and K <= GLMQ_MAX_K; M >= 0 activation rows. N == 0 or
+ *     M == 0 is an empty problem: GLMQ_OK, nothing is enqueued, pointers may
+ *     be NULL.
+ *   - Inputs are finite fp16 values; NaN or Inf inputs are outside the contract.
+ *   - Calls that overlap on the GPU and write the same output race; distinct
+ *     calls share no library-owned state except the device status word.
+ */
+#ifndef GLMQ_H
+#define GLMQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define GLMQ_API __attribute__((visibility("default")))
+#else
+#define GLMQ_API
+#endif
+
+#define GLMQ_ABI_VERSION 1
+#define GLMQ_MAX_K 65536
+/* Largest M served by the decode (register-dequant GEMV) kernel in glmq_gemm. */
+#define GLMQ_DECODE_MAX_M 16
+
+typedef enum glmq_status {
+  GLMQ_OK = 0,
+  GLMQ_ERR_NULL_POINTER = 1,      /* a required pointer is NULL                       */
+  GLMQ_ERR_BAD_BITS = 2,          /* bits is not 4 or 8                                */
+  GLMQ_ERR_BAD_SHAPE = 3,         /* a size is negative, K % 64 != 0, K > GLMQ_MAX_K,
+                                     or a size exceeds a kernel's limit               */
+  GLMQ_ERR_MISALIGNED = 4,        /* a pointer is not 16-byte aligned                 */
+  GLMQ_ERR_CUDA = 5,              /* a CUDA runtime call failed (see glmq_last_cuda_error) */
+  GLMQ_ERR_DEVICE = 6,            /* a kernel reported a device-side error            */
+  GLMQ_ERR_UNSUPPORTED_DEVICE = 7 /* the current device is not compute capability 10.0 */
+} glmq_status;
+
+/* The ABI version this library was built with (GLMQ_ABI_VERSION). */
+GLMQ_API int glmq_abi_version(void);
+
+/* Bytes of packed weight storage for an [N, K] weight at `bits` bits:
+ * N*K/2 for INT4, N*K for INT8. Returns 0 for invalid arguments. Host-only. */
+GLMQ_API size_t glmq_packed_bytes(int64_t N, int64_t K, int bits);
+
+/*
+ * One-shot weight quantization (paper card, "Method": quantize_linear_int4;
+ * "Paper vs code": per-row absmax / (2^(b-1)-1), FP16 scale).
+ *   W       in : fp16 [N, K], row n = output feature n
+ *   packed  out: uint8 [N, K*bits/8] (glmq_packed_bytes(N, K, bits) bytes)
+ *   scale   out: fp16 [N]
+ * Packed codes and scales are a pure function of W (bit-for-bit reproducible).
+ * Limits: N <= 2^31 - 1.
+ */
+GLMQ_API glmq_status glmq_quantize(const void* W, int64_t N, int64_t K, int bits, void* packed, void* scale,
+                          void* stream);
+
+/*
+ * Dequantizing linear layer (paper card, "Method": linear_forward):
+ *   Y[m,n] = fp16_rn( s[n] * sum_k X[m,k] * q[n,k] ), fp32 accumulation.
+ *   X       in : fp16 [M, K] activations
+ *   packed  in : codes from glmq_quantize (same N, K, bits)
+ *   scale   in : fp16 [N]
+ *   Y       out: fp16 [M, N]; must not overlap any input
+ * Dispatch: M <= GLMQ_DECODE_MAX_M runs the decode kernel (HBM-bound stream of
+ * the packed weights, register dequantization); larger M runs the tensor-core
+ * prefill kernel. Both give results within the documented accuracy.
+ */
+GLMQ_API glmq_status glmq_gemm(const void* X, int64_t M, const void* packed, const void* scale, int64_t N,
+                      int64_t K, int bits, void* Y, void* stream);
+
+/* glmq_gemm forced onto the decode kernel. Requires M <= GLMQ_DECODE_MAX_M. */
+GLMQ_API glmq_status glmq_gemm_decode(const void* X, int64_t M, const void* packed, const void* scale,
+                             int64_t N, int64_t K, int bits, void* Y, void* stream);
+
+/* glmq_gemm forced onto the tensor-core prefill kernel (any M >= 0). */
+GLMQ_API glmq_status glmq_gemm_prefill(const void* X, int64_t M, const void* packed, const void* scale,
+                              int64_t N, int64_t K, int bits, void* Y, void* stream);
+
+/* Static description of a status code. Never NULL. */
+GLMQ_API const char* glmq_status_string(int status);
+
+/* The cudaError_t value (as int) of the last failed CUDA call in this thread,
+ * 0 if none. */
+GLMQ_API int glmq_last_cuda_error(void);
+
+/*
+ * Synchronizes `stream`, then reads and clears the current device's status
+ * word, which kernels set when a bounded internal wait gives up (instead of
+ * hanging). Returns GLMQ_OK if the word was 0, else GLMQ_ERR_DEVICE and, if
+ * `flags` is not NULL, stores the word's bits there. For tests and debugging:
+ * it blocks the calling thread.
+ */
+GLMQ_API glmq_status glmq_last_device_error(void* stream, uint32_t* flags);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GLMQ_H */

@@ -6,6 +6,7 @@ GLM-130B projection layers. See :mod:`inputs.synthetic`.
 """
 from .synthetic import (  # noqa: F401
     GLM_PROJECTIONS,
+    PROJECTION_ORDER,
     TINY_N,
     TINY_K,
     TINY_M,

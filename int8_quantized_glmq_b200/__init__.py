@@ -1,0 +1,21 @@
+"""B200-native weight-only INT4/INT8 quantization and W4A16/W8A16 GEMM for GLM-130B shapes.
+
+The compute lives in ``libglmq.so`` (CUDA C++ for sm_100a, C ABI in
+``include/glmq.h``); this package is its Python binding.
+"""
+from ._binding import (  # noqa: F401
+    DECODE_MAX_M,
+    MAX_K,
+    GlmqError,
+    abi_version,
+    gemm,
+    gemm_decode,
+    gemm_prefill,
+    last_device_error,
+    lib,
+    packed_bytes,
+    quantize,
+    raw_gemm,
+    raw_quantize,
+    status_string,
+)

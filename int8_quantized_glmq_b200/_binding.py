@@ -1,0 +1,176 @@
+"""ctypes binding for libglmq.so: the C ABI declared in include/glmq.h.
+
+Argument marshalling only: every step of quantization and of the dequantizing
+linear layer runs in the library's CUDA kernels. PyTorch is used for device
+memory and streams. There is no CPU fallback: if the library is missing or the
+device is not an sm_100 GPU, calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+PKG_DIR = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG_DIR, "libglmq.so")
+
+# glmq_status values (include/glmq.h)
+OK = 0
+ERR_NULL_POINTER = 1
+ERR_BAD_BITS = 2
+ERR_BAD_SHAPE = 3
+ERR_MISALIGNED = 4
+ERR_CUDA = 5
+ERR_DEVICE = 6
+ERR_UNSUPPORTED_DEVICE = 7
+
+DECODE_MAX_M = 16
+MAX_K = 65536
+
+#: every symbol include/glmq.h declares, with (restype, argtypes)
+_c_int64 = ctypes.c_int64
+_vp = ctypes.c_void_p
+SIGNATURES = {
+    "glmq_abi_version": (ctypes.c_int, []),
+    "glmq_packed_bytes": (ctypes.c_size_t, [_c_int64, _c_int64, ctypes.c_int]),
+    "glmq_quantize": (ctypes.c_int, [_vp, _c_int64, _c_int64, ctypes.c_int, _vp, _vp, _vp]),
+    "glmq_gemm": (ctypes.c_int, [_vp, _c_int64, _vp, _vp, _c_int64, _c_int64, ctypes.c_int, _vp, _vp]),
+    "glmq_gemm_decode": (ctypes.c_int, [_vp, _c_int64, _vp, _vp, _c_int64, _c_int64, ctypes.c_int, _vp, _vp]),
+    "glmq_gemm_prefill": (ctypes.c_int, [_vp, _c_int64, _vp, _vp, _c_int64, _c_int64, ctypes.c_int, _vp, _vp]),
+    "glmq_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "glmq_last_cuda_error": (ctypes.c_int, []),
+    "glmq_last_device_error": (ctypes.c_int, [_vp, ctypes.POINTER(ctypes.c_uint32)]),
+}
+
+_lib = None
+_lock = threading.Lock()
+
+
+class GlmqError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = f"{where}: glmq status {status} ({status_string(status)})"
+        if status == ERR_CUDA:
+            msg += f", cudaError {lib().glmq_last_cuda_error()}"
+        super().__init__(msg)
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded library (loaded once). Raises if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(
+                    f"{LIB_PATH} is missing: build it with `python -m int8_quantized_glmq_b200.build` "
+                    "(there is no CPU fallback)")
+            handle = ctypes.CDLL(LIB_PATH)
+            for name, (res, args) in SIGNATURES.items():
+                fn = getattr(handle, name)
+                fn.restype = res
+                fn.argtypes = args
+            _lib = handle
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().glmq_status_string(int(status)).decode()
+
+
+def abi_version() -> int:
+    return lib().glmq_abi_version()
+
+
+def packed_bytes(N: int, K: int, bits: int) -> int:
+    return lib().glmq_packed_bytes(N, K, bits)
+
+
+def _check(status: int, where: str) -> None:
+    if status != OK:
+        raise GlmqError(status, where)
+
+
+# ----------------------------------------------------------------- raw-pointer calls
+def raw_quantize(W: int, N: int, K: int, bits: int, packed: int, scale: int, stream: int = 0) -> int:
+    return lib().glmq_quantize(W, N, K, bits, packed, scale, stream)
+
+
+def raw_gemm(X: int, M: int, packed: int, scale: int, N: int, K: int, bits: int, Y: int, stream: int = 0,
+             route: str = "auto") -> int:
+    fn = {"auto": lib().glmq_gemm, "decode": lib().glmq_gemm_decode, "prefill": lib().glmq_gemm_prefill}[route]
+    return fn(X, M, packed, scale, N, K, bits, Y, stream)
+
+
+def last_device_error(stream: int = 0):
+    """(status, flags): synchronizes the stream and reads/clears the device status word."""
+    flags = ctypes.c_uint32(0)
+    st = lib().glmq_last_device_error(stream, ctypes.byref(flags))
+    return st, flags.value
+
+
+# ----------------------------------------------------------------- torch-tensor calls
+def _torch():
+    import torch  # noqa: WPS433 (plumbing only)
+    return torch
+
+
+def _stream_ptr(stream=None) -> int:
+    torch = _torch()
+    s = torch.cuda.current_stream() if stream is None else stream
+    return int(s.cuda_stream)
+
+
+def _require(t, dtype, ndim, name):
+    torch = _torch()
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must be on a CUDA device (no CPU path exists)")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != ndim or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous {ndim}-D tensor")
+
+
+def quantize(W, bits: int = 4, stream=None, out=None):
+    """One-shot quantization of fp16 W[N, K] -> (packed uint8 [N, K*bits/8], scale fp16 [N])."""
+    torch = _torch()
+    _require(W, torch.float16, 2, "W")
+    N, K = W.shape
+    if out is None:
+        packed = torch.empty((N, K * bits // 8), dtype=torch.uint8, device=W.device)
+        scale = torch.empty((N,), dtype=torch.float16, device=W.device)
+    else:
+        packed, scale = out
+    with torch.cuda.device(W.device):
+        st = raw_quantize(W.data_ptr(), N, K, bits, packed.data_ptr(), scale.data_ptr(), _stream_ptr(stream))
+    _check(st, "glmq_quantize")
+    return packed, scale
+
+
+def gemm(X, packed, scale, bits: int = 4, stream=None, out=None, route: str = "auto"):
+    """Y[M, N] = fp16(s[n] * sum_k X[m,k] q[n,k]) for packed weights from :func:`quantize`."""
+    torch = _torch()
+    _require(X, torch.float16, 2, "X")
+    _require(packed, torch.uint8, 2, "packed")
+    _require(scale, torch.float16, 1, "scale")
+    M, K = X.shape
+    N = packed.shape[0]
+    if packed.shape[1] * 8 != K * bits or scale.shape[0] != N:
+        raise ValueError("packed/scale shapes do not match X and bits")
+    Y = torch.empty((M, N), dtype=torch.float16, device=X.device) if out is None else out
+    with torch.cuda.device(X.device):
+        st = raw_gemm(X.data_ptr(), M, packed.data_ptr(), scale.data_ptr(), N, K, bits, Y.data_ptr(),
+                      _stream_ptr(stream), route)
+    _check(st, f"glmq_gemm({route})")
+    return Y
+
+
+def gemm_decode(X, packed, scale, bits: int = 4, stream=None, out=None):
+    return gemm(X, packed, scale, bits, stream, out, route="decode")
+
+
+def gemm_prefill(X, packed, scale, bits: int = 4, stream=None, out=None):
+    return gemm(X, packed, scale, bits, stream, out, route="prefill")

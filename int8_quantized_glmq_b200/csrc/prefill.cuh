@@ -1,0 +1,351 @@
+// Prefill-regime W4A16 / W8A16 GEMM on the 5th-generation tensor cores (tcgen05).
+//
+//   Y[m,n] = fp16( s[n] * sum_k X[m,k] q[n,k] )
+//
+// GLM-130B paper card (wikillm.com), "Method": linear_forward with weight =
+// quant * scale[:, None] and FP16 activations; paperlayer summary, "INT4
+// Quantization for RTX 3090s/2080s": weights are converted to FP16 at run time.
+// With M up to a 2048-token prompt the product is a dense contraction, so it runs
+// on tcgen05.mma (kind::f16, fp32 accumulation in tensor memory).
+//
+// The MMA is issued "swapped": the 128 weight rows of a tile are the MMA's M
+// dimension (operand A) and BN tokens its N dimension (operand B), so the per-row
+// scale s[n] belongs to one TMEM lane and is applied once per output in the
+// epilogue. Warp roles (persistent CTAs, one per SM, static round-robin tiles,
+// the BN-token tiles of one weight tile consecutive so the packed rows are read
+// from HBM once and then hit in L2):
+//   warp 12      TMA producer: 2-D tensor copies of the X tile (BN x 64 fp16,
+//                128-byte swizzle) and of the packed weight tile (128 rows of
+//                32 / 64 bytes, 32- / 64-byte swizzle) into a kStages ring;
+//   warps 0..7   dequantizers: each thread turns 32 codes of one row into fp16
+//                and writes them into the A tile in the canonical K-major
+//                128-byte-swizzled layout, then fences the generic->async proxy;
+//   warp 13      MMA issuer: one thread issues 4 tcgen05.mma (K=16) per 64-wide
+//                K block into one of two TMEM accumulators and commits each stage
+//                back to the producer;
+//   warps 8..11  epilogue: tcgen05.ld of its 32 TMEM lanes, times s[n], fp16
+//                stores; frees the accumulator for the next-but-one tile.
+// No TMA multicast is used anywhere.
+#pragma once
+
+#include <cuda.h>
+
+#include "glmq_ptx.cuh"
+
+namespace glmq {
+
+constexpr int kPrefillDequantWarps = 8;
+constexpr int kPrefillEpilogueWarp0 = 8;
+constexpr int kPrefillProducerWarp = 12;
+constexpr int kPrefillMmaWarp = 13;
+constexpr int kPrefillThreads = 14 * 32;
+constexpr int kPrefillStages = 4;
+
+template <int BITS, int BN>
+struct PrefillCfg {
+  static constexpr int kBits = BITS;
+  static constexpr int kBN = BN;
+  static constexpr int BM = 128;
+  static constexpr int BK = 64;
+  static constexpr int X_BYTES = BN * BK * 2;           // B operand tile
+  static constexpr int A_BYTES = BM * BK * 2;           // dequantized A tile
+  static constexpr int WROW = BK * BITS / 8;            // packed bytes per row per K block (32 or 64)
+  static constexpr int W_BYTES = BM * WROW;
+  static constexpr int STAGE_BYTES = X_BYTES + A_BYTES + W_BYTES;
+  static constexpr int TMEM_COLS = (2 * BN <= 256) ? 256 : 512;
+  static constexpr int SMEM_BYTES = kPrefillStages * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+  static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N for M=128");
+  static_assert(X_BYTES % 1024 == 0, "swizzle atoms stay 1024-byte aligned");
+  // kind::f16, fp32 accumulator, fp16 A and B, both K-major, N = BN, M = 128
+  static constexpr uint32_t IDESC = (1u << 4) | (uint32_t(BN >> 3) << 17) | (uint32_t(BM >> 4) << 24);
+};
+
+struct PrefillArgs {
+  const __half* scale;
+  __half* Y;
+  int M;
+  int N;
+  int K;
+  int tiles_m;
+  int tiles;
+};
+
+// ---------------------------------------------------------------- tcgen05 / TMA wrappers
+__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t smem_addr) {
+  // K-major, 128-byte swizzle: LBO = 1 (16 B units, unused), SBO = 1024 B between
+  // 8-row groups, descriptor version 1, layout type 2 (SWIZZLE_128B).
+  return static_cast<uint64_t>((smem_addr >> 4) & 0x3FFFu) | (1ull << 16) | (64ull << 32) | (1ull << 46) |
+         (2ull << 61);
+}
+
+__device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+        "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
+        "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]),
+        "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+      "[%4];" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
+// Byte offset of 16-byte chunk `c` (8 fp16 along K) of row `row` in a K-major,
+// 128-byte-swizzled tile whose rows are 128 bytes (64 fp16).
+__device__ __forceinline__ uint32_t sw128_off(int row, int c) {
+  return static_cast<uint32_t>((row >> 3) * 1024 + (row & 7) * 128 + ((c ^ (row & 7)) << 4));
+}
+
+// INT4 packed word (8 codes, k = 0..7) -> 4 words of fp16 pairs in natural k order.
+__device__ __forceinline__ uint4 dequant_int4_natural(uint32_t w) {
+  const __half2 kBias0 = __halves2half2(__ushort_as_half(0xE408), __ushort_as_half(0xE408));  // -1032
+  const __half2 kOne16 = __halves2half2(__ushort_as_half(0x2C00), __ushort_as_half(0x2C00));  // 1/16
+  const __half2 kBias1 = __halves2half2(__ushort_as_half(0xD480), __ushort_as_half(0xD480));  // -72
+  const uint32_t w8 = w >> 8;
+  uint32_t h0 = lop3_and_xor(w, 0x000F000Fu, 0x64086408u);   // (0, 4)
+  uint32_t h1 = lop3_and_xor(w, 0x00F000F0u, 0x64806480u);   // (1, 5) * 16
+  uint32_t h2 = lop3_and_xor(w8, 0x000F000Fu, 0x64086408u);  // (2, 6)
+  uint32_t h3 = lop3_and_xor(w8, 0x00F000F0u, 0x64806480u);  // (3, 7) * 16
+  __half2 r0 = __hadd2(*reinterpret_cast<__half2*>(&h0), kBias0);
+  __half2 r1 = __hfma2(*reinterpret_cast<__half2*>(&h1), kOne16, kBias1);
+  __half2 r2 = __hadd2(*reinterpret_cast<__half2*>(&h2), kBias0);
+  __half2 r3 = __hfma2(*reinterpret_cast<__half2*>(&h3), kOne16, kBias1);
+  const uint32_t p0 = *reinterpret_cast<uint32_t*>(&r0), p1 = *reinterpret_cast<uint32_t*>(&r1);
+  const uint32_t p2 = *reinterpret_cast<uint32_t*>(&r2), p3 = *reinterpret_cast<uint32_t*>(&r3);
+  return make_uint4(prmt(p0, p1, 0x5410u), prmt(p2, p3, 0x5410u), prmt(p0, p1, 0x7632u), prmt(p2, p3, 0x7632u));
+}
+
+__device__ __forceinline__ uint2 dequant_int8_natural(uint32_t w) {
+  const __half2 kBias = __halves2half2(__ushort_as_half(0xE480), __ushort_as_half(0xE480));  // -1152
+  const uint32_t x = w ^ 0x80808080u;
+  uint32_t lo = prmt(x, 0x64646464u, 0x4140u);
+  uint32_t hi = prmt(x, 0x64646464u, 0x4342u);
+  __half2 a = __hadd2(*reinterpret_cast<__half2*>(&lo), kBias);
+  __half2 b = __hadd2(*reinterpret_cast<__half2*>(&hi), kBias);
+  return make_uint2(*reinterpret_cast<uint32_t*>(&a), *reinterpret_cast<uint32_t*>(&b));
+}
+
+// ---------------------------------------------------------------- the kernel
+template <class C>
+__global__ void __launch_bounds__(kPrefillThreads, 1)
+    prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
+                   const PrefillArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kPrefillStages * C::STAGE_BYTES);
+  uint64_t* full = bars;                           // TMA bytes landed          (count 1 + tx)
+  uint64_t* afull = bars + kPrefillStages;         // A tile dequantized        (count 8 warps)
+  uint64_t* empty = bars + 2 * kPrefillStages;     // MMAs of the stage done    (tcgen05.commit)
+  uint64_t* accfull = bars + 3 * kPrefillStages;   // accumulator ready         (tcgen05.commit), x2
+  uint64_t* accempty = accfull + 2;                // accumulator drained       (count 4 warps), x2
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accempty + 2);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int num_kb = a.K / C::BK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kPrefillStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&afull[s], kPrefillDequantWarps);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&accfull[b], 1);
+      mbar_init(&accempty[b], 4);
+    }
+    fence_barrier_init();
+  }
+  if (warp == kPrefillMmaWarp) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(C::TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int G = gridDim.x;
+  bool ok = true;
+
+  if (warp == kPrefillProducerWarp) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      uint32_t armed[kPrefillStages] = {};
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int tile = blockIdx.x; tile < a.tiles && ok; tile += G) {
+        const int nt = tile / a.tiles_m;
+        const int mt = tile - nt * a.tiles_m;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1)) { ok = false; break; }
+          uint8_t* st = smem + stage * C::STAGE_BYTES;
+          mbar_arrive_expect_tx(&full[stage], C::X_BYTES + C::W_BYTES);
+          armed[stage] = phase + 1;
+          tma_load_2d(st, &tmap_x, kb * C::BK, mt * C::kBN, &full[stage]);
+          tma_load_2d(st + C::X_BYTES + C::A_BYTES, &tmap_w, kb * C::WROW, nt * C::BM, &full[stage]);
+          if (++stage == kPrefillStages) { stage = 0; phase ^= 1; }
+        }
+      }
+      bool drained = true;
+      for (int s = 0; s < kPrefillStages; ++s)
+        if (armed[s] && !mbar_wait(&full[s], armed[s] - 1)) drained = false;
+      if (!ok || !drained) report_error(kErrPrefillWait);
+    }
+  } else if (warp < kPrefillDequantWarps) {
+    // ------------------------------------------------------------ dequantizers
+    const int row = threadIdx.x & 127;   // tile row (TMEM lane / weight row)
+    const int half = threadIdx.x >> 7;   // which 32 codes of the 64-wide K block
+    int stage = 0;
+    uint32_t phase = 0;
+    for (int tile = blockIdx.x; tile < a.tiles && ok; tile += G) {
+      for (int kb = 0; kb < num_kb; ++kb) {
+        if (!mbar_wait_warp(&full[stage], phase)) { ok = false; break; }
+        uint8_t* st = smem + stage * C::STAGE_BYTES;
+        const uint32_t a_tile = smem_u32(st + C::X_BYTES);
+        const uint32_t w_tile = smem_u32(st + C::X_BYTES + C::A_BYTES);
+        if constexpr (C::kBits == 4) {
+          // 32-byte rows, 32-byte swizzle: 16-byte unit u sits at u ^ ((row >> 2) & 1)
+          const uint4 v = lds_v4(w_tile + row * 32 + ((half ^ ((row >> 2) & 1)) << 4));
+          const uint32_t words[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint4 o = dequant_int4_natural(words[j]);
+            st_shared_v4(a_tile + sw128_off(row, 4 * half + j), o.x, o.y, o.z, o.w);
+          }
+        } else {
+          // 64-byte rows, 64-byte swizzle: unit u sits at u ^ ((row >> 1) & 3)
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            const int u = 2 * half + q;
+            const uint4 v = lds_v4(w_tile + row * 64 + ((u ^ ((row >> 1) & 3)) << 4));
+            const uint2 lo0 = dequant_int8_natural(v.x), lo1 = dequant_int8_natural(v.y);
+            const uint2 hi0 = dequant_int8_natural(v.z), hi1 = dequant_int8_natural(v.w);
+            st_shared_v4(a_tile + sw128_off(row, 2 * u), lo0.x, lo0.y, lo1.x, lo1.y);
+            st_shared_v4(a_tile + sw128_off(row, 2 * u + 1), hi0.x, hi0.y, hi1.x, hi1.y);
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&afull[stage]);
+        if (++stage == kPrefillStages) { stage = 0; phase ^= 1; }
+      }
+    }
+    if (!ok && lane == 0) report_error(kErrPrefillWait);
+  } else if (warp == kPrefillMmaWarp) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      uint32_t acc_armed[2] = {};
+      for (int tile = blockIdx.x; tile < a.tiles && ok; tile += G, ++it) {
+        const int ab = it & 1;
+        const uint32_t aphase = (it >> 1) & 1;
+        if (!mbar_wait(&accempty[ab], aphase ^ 1)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + ab * C::kBN;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(&afull[stage], phase)) { ok = false; break; }
+          tc_fence_after();
+          uint8_t* st = smem + stage * C::STAGE_BYTES;
+          const uint32_t x_addr = smem_u32(st);
+          const uint32_t a_addr = smem_u32(st + C::X_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < C::BK / 16; ++kk) {
+            umma_f16(d_tmem, umma_desc_sw128(a_addr + kk * 32), umma_desc_sw128(x_addr + kk * 32), C::IDESC,
+                     (kb | kk) != 0);
+          }
+          umma_commit(&empty[stage]);
+          if (++stage == kPrefillStages) { stage = 0; phase ^= 1; }
+        }
+        if (!ok) break;
+        umma_commit(&accfull[ab]);
+        acc_armed[ab] = aphase + 1;
+      }
+      // make sure no MMA is still writing TMEM before the allocation is released
+      bool drained = true;
+      for (int b = 0; b < 2; ++b)
+        if (acc_armed[b] && !mbar_wait(&accfull[b], acc_armed[b] - 1)) drained = false;
+      if (!ok || !drained) report_error(kErrPrefillWait);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue warps 8..11
+    const int quarter = warp & 3;   // TMEM lanes 32*quarter .. 32*quarter+31
+    int it = 0;
+    for (int tile = blockIdx.x; tile < a.tiles && ok; tile += G, ++it) {
+      const int ab = it & 1;
+      const uint32_t aphase = (it >> 1) & 1;
+      if (!mbar_wait_warp(&accfull[ab], aphase)) { ok = false; break; }
+      tc_fence_after();
+      const int nt = tile / a.tiles_m;
+      const int mt = tile - nt * a.tiles_m;
+      const int n = nt * C::BM + quarter * 32 + lane;
+      const float s = (n < a.N) ? __half2float(a.scale[n]) : 0.0f;
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + ab * C::kBN;
+#pragma unroll 1
+      for (int cb = 0; cb < C::kBN / 32; ++cb) {
+        const int m0 = mt * C::kBN + cb * 32;
+        if (m0 >= a.M) break;   // warp-uniform
+        uint32_t v[32];
+        tmem_ld32(t_row + cb * 32, v);
+        if (n < a.N) {
+          __half* yp = a.Y + static_cast<long long>(m0) * a.N + n;
+          const int mend = min(32, a.M - m0);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            if (j < mend) yp[static_cast<long long>(j) * a.N] = __float2half_rn(s * __uint_as_float(v[j]));
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&accempty[ab]);
+    }
+    if (!ok && lane == 0) report_error(kErrPrefillWait);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kPrefillMmaWarp) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(C::TMEM_COLS)
+                 : "memory");
+  }
+}
+
+}  // namespace glmq

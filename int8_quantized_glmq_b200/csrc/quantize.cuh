@@ -1,0 +1,154 @@
+// One-shot weight quantization: fp16 W[N,K] -> packed INT4/INT8 codes + fp16 scale[N].
+//
+// GLM-130B paper card (wikillm.com), "Method": each output row of a linear
+// layer gets one scale, absmax / 7, and the weights are rounded to integers in
+// [-7, 7], two per byte. "Paper vs code": the divisor is 2^(b-1)-1, so INT8 uses
+// absmax / 127, and the scale is computed per output row in FP16.
+//
+// Readings fixed by this library (the same ones the oracle states):
+//   s = fp16_rn(fp32(a) / d),  q = clamp(rint(fp32(w) / fp32(s)), -d, d),
+//   q = 0 on rows whose scale rounds to 0, round half to even,
+//   INT4 byte j = (q[2j] & 0xF) | (q[2j+1] << 4)  (low nibble = even k).
+//
+// Kernel shape (HBM-bound): one CTA of 256 threads per row. Each thread loads
+// its 16-byte chunks of the row once with streaming 128-bit loads and keeps them
+// in registers; the row absmax is an integer max over |w| bit patterns (a warp
+// reduce, then 8 warps through shared memory); the codes are formed from the
+// registers and written with coalesced 4- or 8-byte stores. W is read exactly once.
+//
+// Exact rounding without a per-element IEEE divide: with r = 1/s rounded to
+// nearest, t = fma(w, r, 1.5*2^23) leaves RNE(w*r) in the low mantissa bits of t.
+// Let e = w*r - k (one fma). Because |w*r - w/s| <= (w/s)*2^-24 < 2^-16 for the
+// quotients that occur (|w/s| < 192), |e| < 1/2 - 2^-15 proves k = RNE(w/s). The
+// rare elements with |e| at or above that margin, and every element of a row
+// whose scale is subnormal (where the clamp can fire), take an exact path that
+// compares 2|w| with (2k +- 1)s; those products have at most 20 significant bits
+// and are exact in fp32.
+#pragma once
+
+#include "glmq_ptx.cuh"
+
+namespace glmq {
+
+constexpr int kQuantThreads = 256;
+
+template <int BITS>
+__device__ __forceinline__ int exact_code(float w, float sf, float kf) {
+  constexpr int D = (1 << (BITS - 1)) - 1;
+  const float aw = fabsf(w);
+  const int k0 = static_cast<int>(fabsf(kf));
+  const float aw2 = aw + aw;                                   // exact
+  const float hi = static_cast<float>(2 * k0 + 1) * sf;        // exact: <= 9 x 11 significant bits
+  const float lo = static_cast<float>(2 * k0 - 1) * sf;        // exact
+  int k = k0;
+  if (aw2 > hi || (aw2 == hi && (k0 & 1))) {
+    k = k0 + 1;
+  } else if (aw2 < lo || (aw2 == lo && (k0 & 1))) {
+    k = k0 - 1;
+  }
+  k = min(k, D);
+  return (w < 0.0f) ? -k : k;
+}
+
+// Codes for the 8 halves of one 16-byte chunk, as 32-bit words whose low bits hold
+// the two's-complement code. Returns nothing; writes u[8].
+template <int BITS>
+__device__ __forceinline__ void chunk_codes(const uint4 v, float sf, float r, bool exact_all, uint32_t (&u)[8]) {
+  const uint32_t words[4] = {v.x, v.y, v.z, v.w};
+  float w[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const __half2 h = *reinterpret_cast<const __half2*>(&words[i]);
+    const float2 f = __half22float2(h);
+    w[2 * i] = f.x;
+    w[2 * i + 1] = f.y;
+  }
+  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+  constexpr float kMargin = 0.5f - 0x1p-15f;
+  float kf[8];
+  bool near = exact_all;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float t = fmaf(w[i], r, kMagic);
+    kf[i] = t - kMagic;
+    const float e = fmaf(w[i], r, -kf[i]);
+    near |= fabsf(e) >= kMargin;
+    u[i] = __float_as_uint(t);
+  }
+  if (near) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) u[i] = static_cast<uint32_t>(exact_code<BITS>(w[i], sf, kf[i]));
+  }
+}
+
+template <int BITS, int CPT>
+__global__ void __launch_bounds__(kQuantThreads) quantize_kernel(const __half* __restrict__ W, int K,
+                                                                  uint8_t* __restrict__ packed,
+                                                                  __half* __restrict__ scale) {
+  constexpr int D = (1 << (BITS - 1)) - 1;
+  const long long row = blockIdx.x;
+  const int nchunks = K >> 3;
+  const uint4* src = reinterpret_cast<const uint4*>(W + row * static_cast<long long>(K));
+
+  uint4 v[CPT];
+  uint32_t m = 0;
+#pragma unroll
+  for (int i = 0; i < CPT; ++i) {
+    const int c = threadIdx.x + i * kQuantThreads;
+    if (c < nchunks) {
+      v[i] = ld_stream_v4(src + c);
+      m = __vmaxu2(m, v[i].x & 0x7fff7fffu);
+      m = __vmaxu2(m, v[i].y & 0x7fff7fffu);
+      m = __vmaxu2(m, v[i].z & 0x7fff7fffu);
+      m = __vmaxu2(m, v[i].w & 0x7fff7fffu);
+    } else {
+      v[i] = make_uint4(0, 0, 0, 0);
+    }
+  }
+  m = max(m & 0xffffu, m >> 16);
+  m = __reduce_max_sync(0xffffffffu, m);
+
+  __shared__ uint32_t warp_max[kQuantThreads / 32];
+  const int warp = threadIdx.x >> 5;
+  if ((threadIdx.x & 31) == 0) warp_max[warp] = m;
+  __syncthreads();
+  uint32_t a_bits = warp_max[0];
+#pragma unroll
+  for (int i = 1; i < kQuantThreads / 32; ++i) a_bits = max(a_bits, warp_max[i]);
+
+  // a2: s = fp16_rn(fp32(a) / d)
+  const float af = __half2float(__ushort_as_half(static_cast<unsigned short>(a_bits)));
+  const __half s = __float2half_rn(__fdiv_rn(af, static_cast<float>(D)));
+  const float sf = __half2float(s);
+  if (threadIdx.x == 0) scale[row] = s;
+
+  const bool zero_row = (sf == 0.0f);
+  const bool exact_all = sf < 0x1p-14f;  // subnormal scale: the clamp can fire
+  const float r = zero_row ? 0.0f : __frcp_rn(sf);
+
+#pragma unroll
+  for (int i = 0; i < CPT; ++i) {
+    const int c = threadIdx.x + i * kQuantThreads;
+    if (c >= nchunks) continue;
+    uint32_t u[8];
+    if (zero_row) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) u[j] = 0;
+    } else {
+      chunk_codes<BITS>(v[i], sf, r, exact_all, u);
+    }
+    if constexpr (BITS == 4) {
+      uint32_t word = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) word |= (u[j] & 0xFu) << (4 * j);
+      reinterpret_cast<uint32_t*>(packed + row * static_cast<long long>(K / 2))[c] = word;
+    } else {
+      uint2 out;
+      out.x = (u[0] & 0xFFu) | ((u[1] & 0xFFu) << 8) | ((u[2] & 0xFFu) << 16) | ((u[3] & 0xFFu) << 24);
+      out.y = (u[4] & 0xFFu) | ((u[5] & 0xFFu) << 8) | ((u[6] & 0xFFu) << 16) | ((u[7] & 0xFFu) << 24);
+      reinterpret_cast<uint2*>(packed + row * static_cast<long long>(K))[c] = out;
+    }
+  }
+}
+
+}  // namespace glmq

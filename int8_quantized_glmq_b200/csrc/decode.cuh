@@ -9,82 +9,77 @@
 //
 // With M <= 16 the packed weights are the whole working set: the kernel is an
 // HBM stream. Design:
-//  * persistent CTAs (one per SM), each owning the row tiles b, b+G, b+2G, ...
-//    (R = 16*ROWG rows per tile), processed in groups of up to kTileGroup tiles;
-//  * warp 8 is a producer: it copies the packed rows of each stage (R rows x
-//    SB bytes) with cp.async.bulk into a kStages-deep shared-memory ring (row
-//    pitch padded so the consumers' 16-byte reads are bank-conflict free), with
-//    an L2 evict-first hint, and the activation rows of the current K pass into
-//    a padded X buffer (double-buffered when X does not fit at once);
-//  * warps 0..7 are consumers: warp w takes segment w (SEGB bytes per row) of
-//    every stage for all R rows, dequantizes codes in registers with exponent
+//  * Work units are (row tile of 32 rows, K part) pairs, enumerated K-part major;
+//    each persistent CTA takes one contiguous range of units, so the load is
+//    balanced to within one unit and a CTA changes K part (and so restages its
+//    activation slice) at most a few times.
+//  * Warp 16 is the producer: one lane issues, per stage, eight 2-D TMA tile
+//    loads of 32 rows x 128 bytes (one per K segment, 128-byte swizzle) into a
+//    kDecodeStages-deep ring, with an L2 evict-first hint. Rows past N and bytes
+//    past K are zero-filled by the TMA unit.
+//  * Warps 0..15 are consumers: warp w owns K segment (w % 8) of every stage for
+//    the 16-row group (w / 8). Codes are dequantized in registers with exponent-
 //    bias tricks (a code c becomes the fp16 number 1024 + (c ^ 8) by OR-ing it
-//    into the mantissa, then one subtraction), and feeds mma.sync m16n8k16 with
-//    the weights as the A operand straight from registers and X as B. The K
-//    order inside each MMA is permuted identically on both operands so that
-//    each 32-bit packed word feeds two MMAs without a byte shuffle;
-//  * the 8 consumer warps each hold a K-slice partial of every output; they add
-//    it into a per-tile fp32 accumulator in shared memory with red.shared.add
-//    (no barrier), and after the last K pass the tile is scaled by s[n],
-//    rounded to fp16 and stored.
+//    into the mantissa, then one subtraction) and feed mma.sync m16n8k16 as the A
+//    operand straight from registers, X being the B operand. The K order inside
+//    each MMA is permuted identically on both operands so that each 32-bit packed
+//    word feeds two MMAs without a byte shuffle; the permutation is applied once,
+//    when the consumers stage the activation slice into shared memory in exactly
+//    the order the B fragments are read.
+//  * A unit's partial sums are added across warps in shared memory
+//    (red.shared.add). A tile covered by one K part is scaled, rounded and stored
+//    directly. When the activation slice does not fit in shared memory at once,
+//    tiles are split over several K parts: each unit adds its partial sums into
+//    an fp32 scratch buffer with fire-and-forget red.global.add, and a small
+//    stream-ordered finalize kernel (decode_finalize_kernel) scales, rounds and
+//    stores Y and returns the scratch to zero for the next call.
 #pragma once
+
+#include <cuda.h>
 
 #include "glmq_ptx.cuh"
 
 namespace glmq {
 
-constexpr int kDecodeConsumerWarps = 8;
+constexpr int kDecodeConsumerWarps = 16;
 constexpr int kDecodeThreads = (kDecodeConsumerWarps + 1) * 32;
 constexpr int kDecodeStages = 4;
-constexpr int kTileGroup = 8;
+constexpr int kDecodeRows = 32;          // rows per tile
+constexpr int kDecodeSegB = 128;         // packed bytes per row per segment (one TMA box width)
+constexpr int kDecodeSegs = 8;           // segments per stage
+constexpr int kDecodeBoxBytes = kDecodeRows * kDecodeSegB;            // 4 KB per TMA box
+constexpr int kDecodeStageBytes = kDecodeSegs * kDecodeBoxBytes;      // 32 KB per stage
+constexpr int kDecodeAccBytes = kDecodeRows * 16 * 4;
+// ring + unit accumulator + barriers; the activation slice follows
+constexpr int kDecodeFixedSmem = kDecodeStages * kDecodeStageBytes + kDecodeAccBytes + 256;
 
-template <int BITS, int NB, int SEGB, int ROWG>
+template <int BITS, int MP>
 struct DecodeCfg {
   static constexpr int kBits = BITS;
-  static constexpr int kNB = NB;            // n8 token blocks: 1 for M <= 8, 2 for M <= 16
-  static constexpr int kSegB = SEGB;        // packed bytes per row per consumer warp per stage
-  static constexpr int kRowG = ROWG;        // 16-row groups per tile
-  static constexpr int R = 16 * ROWG;       // rows per tile
-  static constexpr int SB = SEGB * kDecodeConsumerWarps;  // packed bytes per row per stage
-  static constexpr int KPB = (BITS == 4) ? 2 : 1;         // codes per byte
-  static constexpr int SK = SB * KPB;       // k per stage
-  static constexpr int SEGK = SEGB * KPB;   // k per segment
-  static constexpr int TB = SEGB / 4;       // packed bytes per thread per row per segment
-  static constexpr int TK = TB * KPB;       // k per thread per segment
-  static constexpr int TW = TB / 4;         // 32-bit words per thread per row per segment
-  static constexpr int WPAD = (SEGB == 128) ? 16 : 64;
-  static constexpr int WPITCH = SB + WPAD;
-  static constexpr int STAGE_BYTES = R * WPITCH;
-  // X row pitch must shift a token's bank group by this many 16-byte units.
-  static constexpr int XSHIFT = (BITS == 4) ? ((SEGB == 128) ? 4 : 2) : ((SEGB == 128) ? 2 : 1);
-  static constexpr int ACC_BYTES = kTileGroup * R * 16 * 4;
-  static constexpr int FIXED_SMEM = kDecodeStages * STAGE_BYTES + ACC_BYTES + 256;
-  static_assert(TB == 16 || TB == 32, "thread slice is one or two 16-byte loads");
-  static_assert(R <= 64, "producer lanes cover at most two rows each");
+  static constexpr int kMP = MP;                    // token capacity of the activation layout (M <= MP)
+  static constexpr int kNB = (MP + 7) / 8;          // n8 token blocks of the MMA
+  static constexpr int KPB = (BITS == 4) ? 2 : 1;   // codes per byte
+  static constexpr int SEGK = kDecodeSegB * KPB;    // k per segment
+  static constexpr int SK = kDecodeSegs * SEGK;     // k per stage
+  static constexpr int TB = kDecodeSegB / 4;        // packed bytes per thread per row per segment (32)
+  static constexpr int TK = TB * KPB;               // k per thread per segment
+  static constexpr int TW = TB / 4;                 // 32-bit words per thread per row per segment (8)
+  static constexpr int XU = TK / 8;                 // 16-byte activation units per thread per segment
+  static constexpr int kChains = 2;                 // independent MMA accumulator chains
 };
-
-// Byte offset of element k inside a padded X row: 16 bytes of padding after every 128.
-__host__ __device__ constexpr uint32_t x_off(uint32_t k) { return 2u * k + (k >> 6) * 16u; }
-
-__host__ __device__ constexpr uint32_t x_pitch(uint32_t kp, int xshift) {
-  const uint32_t base = x_off(kp);
-  const uint32_t want = static_cast<uint32_t>(xshift) * 16u;
-  return base + ((want + 128u - (base & 127u)) & 127u);
-}
 
 struct DecodeArgs {
   const __half* X;
-  const uint8_t* packed;
   const __half* scale;
   __half* Y;
+  float* ws;          // fp32 [M, N] scratch, zero on entry (used when parts > 1)
   int M;
   int N;
   int K;
-  int KP;       // k per pass (multiple of SK)
-  int passes;
-  int XP;       // X row pitch in shared memory (bytes)
-  int xbufs;    // 1 (X resident for the whole kernel) or 2 (double-buffered passes)
+  int KPP;            // k per part (multiple of SK)
+  int parts;
   int tiles;
+  int units;          // parts * tiles
 };
 
 // ---------------------------------------------------------------- dequantization
@@ -121,272 +116,279 @@ __device__ __forceinline__ void dequant_int8_word(uint32_t w, uint32_t (&p)[2]) 
   p[1] = *reinterpret_cast<uint32_t*>(&b);
 }
 
+__device__ __forceinline__ void tma_load_2d_hint(void* smem_dst, const CUtensorMap* map, int x, int y, uint64_t* bar,
+                                                 uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint "
+      "[%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+
+// Index (in 16-byte units) of the activation unit read by lane (n, c) for unit jj of
+// segment sg of the current K part. Consecutive lanes of a token read consecutive
+// units; the token stride is the compile-time capacity MP, so within a stage every
+// fragment address is a per-lane base plus an immediate.
+template <class C>
+__host__ __device__ constexpr uint32_t x_unit(int sg, int jj, int n, int c) {
+  return static_cast<uint32_t>(((sg * C::XU + jj) * C::kMP + n) * 4 + c);
+}
+
+// One stage of one consumer warp: its segment (TK codes per lane) of rows ra and
+// ra + 8, against the staged activations. kTail: some lanes' codes lie past K.
+template <class C, bool kTail>
+__device__ __forceinline__ void decode_segment(uint32_t box, uint32_t xseg, uint32_t wlane, uint32_t xlane0,
+                                               uint32_t xlane1, bool valid, float (&acc)[C::kChains][C::kNB][4]) {
+  constexpr uint32_t kJStride = static_cast<uint32_t>(C::kMP) * 64u;   // bytes between consecutive jj
+  uint32_t wa[C::TW], wb[C::TW];
+#pragma unroll
+  for (int q = 0; q < 2; ++q) {
+    uint4 va = make_uint4(0, 0, 0, 0), vb = make_uint4(0, 0, 0, 0);
+    if (!kTail || valid) {
+      // 128-byte swizzle: lane offsets for q = 0 / 1 are precomputed in wlane (low / high 16 bits)
+      const uint32_t off = q ? (wlane >> 16) : (wlane & 0xFFFFu);
+      va = lds_v4(box + off);
+      vb = lds_v4(box + off + 8 * kDecodeSegB);
+    }
+    wa[4 * q + 0] = va.x; wa[4 * q + 1] = va.y; wa[4 * q + 2] = va.z; wa[4 * q + 3] = va.w;
+    wb[4 * q + 0] = vb.x; wb[4 * q + 1] = vb.y; wb[4 * q + 2] = vb.z; wb[4 * q + 3] = vb.w;
+  }
+  if constexpr (C::kBits == 4) {
+#pragma unroll
+    for (int j = 0; j < C::TW; ++j) {
+      uint4 bf[C::kNB];
+#pragma unroll
+      for (int nb = 0; nb < C::kNB; ++nb) {
+        bf[nb] = make_uint4(0, 0, 0, 0);
+        if (!kTail || valid) bf[nb] = lds_v4(xseg + (nb ? xlane1 : xlane0) + j * kJStride);
+      }
+      uint32_t pa[4], pb[4];
+      dequant_int4_word(wa[j], pa);
+      dequant_int4_word(wb[j], pb);
+#pragma unroll
+      for (int nb = 0; nb < C::kNB; ++nb) {
+        mma_16816(acc[0][nb], pa[0], pb[0], pa[1], pb[1], bf[nb].x, bf[nb].y);
+        mma_16816(acc[1][nb], pa[2], pb[2], pa[3], pb[3], bf[nb].z, bf[nb].w);
+      }
+    }
+  } else {
+#pragma unroll
+    for (int j2 = 0; j2 < C::TW / 2; ++j2) {
+      uint4 bf[C::kNB];
+#pragma unroll
+      for (int nb = 0; nb < C::kNB; ++nb) {
+        bf[nb] = make_uint4(0, 0, 0, 0);
+        if (!kTail || valid) bf[nb] = lds_v4(xseg + (nb ? xlane1 : xlane0) + j2 * kJStride);
+      }
+      uint32_t pa0[2], pb0[2], pa1[2], pb1[2];
+      dequant_int8_word(wa[2 * j2], pa0);
+      dequant_int8_word(wb[2 * j2], pb0);
+      dequant_int8_word(wa[2 * j2 + 1], pa1);
+      dequant_int8_word(wb[2 * j2 + 1], pb1);
+#pragma unroll
+      for (int nb = 0; nb < C::kNB; ++nb) {
+        mma_16816(acc[0][nb], pa0[0], pb0[0], pa0[1], pb0[1], bf[nb].x, bf[nb].y);
+        mma_16816(acc[1][nb], pa1[0], pb1[0], pa1[1], pb1[1], bf[nb].z, bf[nb].w);
+      }
+    }
+  }
+}
+
 // ---------------------------------------------------------------- the kernel
 template <class C>
-__global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const DecodeArgs a) {
-  extern __shared__ __align__(128) uint8_t smem[];
+__global__ void __launch_bounds__(kDecodeThreads, 1)
+    decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const DecodeArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* wring = smem;
-  float* acc_s = reinterpret_cast<float*>(smem + kDecodeStages * C::STAGE_BYTES);
-  uint8_t* xbuf = smem + kDecodeStages * C::STAGE_BYTES + C::ACC_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(xbuf + a.xbufs * a.M * a.XP);
-  uint64_t* full = bars;
-  uint64_t* empty = bars + kDecodeStages;
-  uint64_t* xfull = bars + 2 * kDecodeStages;
-  uint64_t* xempty = xfull + 2;
+  float* acc_s = reinterpret_cast<float*>(smem + kDecodeStages * kDecodeStageBytes);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kDecodeStages * kDecodeStageBytes + kDecodeAccBytes);
+  uint64_t* empty = full + kDecodeStages;
+  uint8_t* xbuf = smem + kDecodeFixedSmem;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int M = a.M, N = a.N, K = a.K;
-  const long long row_bytes = static_cast<long long>(K) / C::KPB;
+  const int G = gridDim.x;
+  const int u_begin = static_cast<int>((static_cast<long long>(blockIdx.x) * a.units) / G);
+  const int u_end = static_cast<int>((static_cast<long long>(blockIdx.x + 1) * a.units) / G);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kDecodeStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], kDecodeConsumerWarps);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&xfull[b], 1);
-      mbar_init(&xempty[b], kDecodeConsumerWarps);
-    }
     fence_barrier_init();
   }
-  if (warp < kDecodeConsumerWarps) {
-    for (int i = threadIdx.x; i < kTileGroup * C::R * 16; i += kDecodeConsumerWarps * 32) acc_s[i] = 0.0f;
-  }
+  for (int i = threadIdx.x; i < kDecodeRows * 16; i += kDecodeThreads) acc_s[i] = 0.0f;
   __syncthreads();
-
-  const int G = gridDim.x;
-  const int multi = a.passes > 1;
 
   if (warp == kDecodeConsumerWarps) {
     // ------------------------------------------------------------ producer warp
-    const uint64_t pol = policy_evict_first();
-    int stage = 0;
-    uint32_t phase = 0;
-    int xb = 0;
-    uint32_t xphase = 0;
-    bool x_loaded = false;
-    bool ok = true;
-    // parity + 1 of the last phase each barrier was armed with (0 = never armed)
-    uint32_t armed[kDecodeStages] = {};
-    uint32_t xarmed[2] = {};
-    for (int g0 = blockIdx.x; g0 < a.tiles && ok; g0 += G * kTileGroup) {
-      for (int p = 0; p < a.passes && ok; ++p) {
-        const int pk0 = p * a.KP;
-        const int plen = min(a.KP, K - pk0);
-        if (multi || !x_loaded) {
-          if (multi && !mbar_wait_warp(&xempty[xb], xphase ^ 1)) { ok = false; break; }
-          if (lane == 0) mbar_arrive_expect_tx(&xfull[xb], static_cast<uint32_t>(M) * plen * 2u);
-          xarmed[xb] = xphase + 1;
-          __syncwarp();
-          const int pieces_per_row = plen >> 6;
-          uint8_t* xdst = xbuf + xb * M * a.XP;
-          for (int i = lane; i < M * pieces_per_row; i += 32) {
-            const int n = i / pieces_per_row;
-            const int pc = i - n * pieces_per_row;
-            bulk_g2s(xdst + n * a.XP + x_off(pc * 64),
-                     a.X + static_cast<long long>(n) * K + pk0 + pc * 64, 128u, &xfull[xb]);
-          }
-          x_loaded = true;
-          if (multi) { xb ^= 1; if (xb == 0) xphase ^= 1; }
-        }
+    if (lane == 0) {
+      const uint64_t pol = policy_evict_first();
+      const int row_bytes = K / C::KPB;
+      uint32_t armed[kDecodeStages] = {};
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int u = u_begin; u < u_end && ok; ++u) {
+        const int p = u / a.tiles;
+        const int t = u - p * a.tiles;
+        const int pk0 = p * a.KPP;
+        const int plen = min(a.KPP, K - pk0);
         const int nst = (plen + C::SK - 1) / C::SK;
-        for (int tt = 0; tt < kTileGroup && ok; ++tt) {
-          const int tile = g0 + tt * G;
-          if (tile >= a.tiles) break;
-          const int row0 = tile * C::R;
-          for (int ks = 0; ks < nst; ++ks) {
-            if (!mbar_wait_warp(&empty[stage], phase ^ 1)) { ok = false; break; }
-            const int k0 = pk0 + ks * C::SK;
-            const uint32_t bytes = static_cast<uint32_t>(min(C::SB, static_cast<int>((K - k0) / C::KPB)));
-            if (lane == 0) mbar_arrive_expect_tx(&full[stage], bytes * C::R);
-            armed[stage] = phase + 1;
-            __syncwarp();
-            uint8_t* dst = wring + stage * C::STAGE_BYTES;
-#pragma unroll
-            for (int i = lane; i < C::R; i += 32) {
-              const long long grow = min(row0 + i, N - 1);
-              bulk_g2s_stream(dst + i * C::WPITCH, a.packed + grow * row_bytes + k0 / C::KPB, bytes,
-                              &full[stage], pol);
-            }
-            if (++stage == kDecodeStages) { stage = 0; phase ^= 1; }
-          }
+        for (int ks = 0; ks < nst; ++ks) {
+          if (!mbar_wait(&empty[stage], phase ^ 1)) { ok = false; break; }
+          const int xb0 = (pk0 + ks * C::SK) / C::KPB;            // first packed byte of the stage
+          const int segs = min(kDecodeSegs, (row_bytes - xb0 + kDecodeSegB - 1) / kDecodeSegB);
+          mbar_arrive_expect_tx(&full[stage], static_cast<uint32_t>(segs * kDecodeBoxBytes));
+          armed[stage] = phase + 1;
+          uint8_t* dst = wring + stage * kDecodeStageBytes;
+          for (int sg = 0; sg < segs; ++sg)
+            tma_load_2d_hint(dst + sg * kDecodeBoxBytes, &tmap_w, xb0 + sg * kDecodeSegB, t * kDecodeRows,
+                             &full[stage], pol);
+          if (++stage == kDecodeStages) { stage = 0; phase ^= 1; }
         }
       }
+      // never leave while TMA writes into this CTA's shared memory may be in flight
+      bool drained = true;
+      for (int s = 0; s < kDecodeStages; ++s)
+        if (armed[s] && !mbar_wait(&full[s], armed[s] - 1)) drained = false;
+      if (!ok || !drained) report_error(kErrDecodeProducerWait);
     }
-    // Do not leave while copies into this CTA's shared memory may be in flight:
-    // wait (bounded) until the last phase armed on every barrier has landed.
-    bool drained = true;
-#pragma unroll
-    for (int s = 0; s < kDecodeStages; ++s)
-      if (armed[s] && !mbar_wait(&full[s], armed[s] - 1)) drained = false;
-    for (int b = 0; b < 2; ++b)
-      if (xarmed[b] && !mbar_wait(&xfull[b], xarmed[b] - 1)) drained = false;
-    if ((!ok || !drained) && lane == 0) report_error(kErrDecodeProducerWait);
     return;
   }
 
   // -------------------------------------------------------------- consumer warps
+  const int seg = warp & (kDecodeSegs - 1);
+  const int grp = warp >> 3;                 // 16-row group
   const int r = lane >> 2;
   const int c = lane & 3;
+  const int ct = threadIdx.x;                // 0 .. 511
+  constexpr int kCT = kDecodeConsumerWarps * 32;
+  const uint32_t wring_u32 = smem_u32(wring);
+  const uint32_t xbuf_u32 = smem_u32(xbuf);
+  const uint32_t acc_u32 = smem_u32(acc_s);
+  const int ra = 16 * grp + r;               // this lane's rows: ra and ra + 8 (same ra & 7)
+  // per-lane byte offsets: packed row ra, 16-byte units 2c and 2c+1 under the 128-byte swizzle
+  const uint32_t wlane = static_cast<uint32_t>(ra * kDecodeSegB + (((2 * c) ^ (ra & 7)) << 4)) |
+                         (static_cast<uint32_t>(ra * kDecodeSegB + (((2 * c + 1) ^ (ra & 7)) << 4)) << 16);
+  // activation units of this lane's tokens (clamped to a real token; results past M are discarded)
+  const uint32_t xlane0 = 16u * x_unit<C>(0, 0, min(r, M - 1), c);
+  const uint32_t xlane1 = 16u * x_unit<C>(0, 0, min(r + 8, M - 1), c);
   int stage = 0;
   uint32_t phase = 0;
-  int xb = 0;
-  uint32_t xphase = 0;
-  bool x_ready = false;
+  int cur_part = -1;
   bool ok = true;
-  const uint32_t wring_u32 = smem_u32(wring);
-  const uint32_t acc_u32 = smem_u32(acc_s);
 
-  for (int g0 = blockIdx.x; g0 < a.tiles; g0 += G * kTileGroup) {
-    for (int p = 0; p < a.passes; ++p) {
-      const int pk0 = p * a.KP;
-      const int plen = min(a.KP, K - pk0);
-      const int xcur = multi ? xb : 0;
-      if (ok && (multi || !x_ready)) {
-        if (!mbar_wait_warp(&xfull[xcur], xphase)) ok = false;
-        x_ready = true;
-      }
-      const uint32_t xrow[2] = {
-          smem_u32(xbuf + xcur * M * a.XP + min(r, M - 1) * a.XP),
-          smem_u32(xbuf + xcur * M * a.XP + min(r + 8, M - 1) * a.XP)};
-      const int nst = (plen + C::SK - 1) / C::SK;
-      for (int tt = 0; tt < kTileGroup; ++tt) {
-        const int tile = g0 + tt * G;
-        if (tile >= a.tiles) break;
-        float acc[C::kRowG][C::kNB][4];
-#pragma unroll
-        for (int g = 0; g < C::kRowG; ++g)
-#pragma unroll
-          for (int nb = 0; nb < C::kNB; ++nb)
-#pragma unroll
-            for (int i = 0; i < 4; ++i) acc[g][nb][i] = 0.0f;
-
-        for (int ks = 0; ks < nst; ++ks) {
-          if (ok && !mbar_wait_warp(&full[stage], phase)) ok = false;
-          const int kl = ks * C::SK + warp * C::SEGK;  // pass-relative k of this warp's segment
-          if (ok && pk0 + kl < K) {
-            const bool valid = pk0 + kl + c * C::TK < K;
-            const uint32_t wbase = wring_u32 + stage * C::STAGE_BYTES + warp * C::kSegB + c * C::TB;
-            // packed words of this thread: rows (16g + r) and (16g + r + 8)
-            uint32_t wa[C::kRowG][C::TW], wb[C::kRowG][C::TW];
-#pragma unroll
-            for (int g = 0; g < C::kRowG; ++g) {
-#pragma unroll
-              for (int q = 0; q < C::TW / 4; ++q) {
-                uint4 va = make_uint4(0, 0, 0, 0), vb = make_uint4(0, 0, 0, 0);
-                if (valid) {
-                  va = lds_v4(wbase + (16 * g + r) * C::WPITCH + 16 * q);
-                  vb = lds_v4(wbase + (16 * g + r + 8) * C::WPITCH + 16 * q);
-                }
-                wa[g][4 * q + 0] = va.x; wa[g][4 * q + 1] = va.y; wa[g][4 * q + 2] = va.z; wa[g][4 * q + 3] = va.w;
-                wb[g][4 * q + 0] = vb.x; wb[g][4 * q + 1] = vb.y; wb[g][4 * q + 2] = vb.z; wb[g][4 * q + 3] = vb.w;
-              }
-            }
-            const uint32_t xk = kl + c * C::TK;  // pass-relative k of this thread's slice
-            if constexpr (C::kBits == 4) {
-#pragma unroll
-              for (int j = 0; j < C::TW; ++j) {
-                uint32_t bf[C::kNB][4];
-#pragma unroll
-                for (int nb = 0; nb < C::kNB; ++nb) {
-                  uint4 xv = make_uint4(0, 0, 0, 0);
-                  if (valid) xv = lds_v4(xrow[nb] + x_off(xk + 8 * j));
-                  bf[nb][0] = prmt(xv.x, xv.z, 0x5410u);  // (x0, x4)
-                  bf[nb][1] = prmt(xv.x, xv.z, 0x7632u);  // (x1, x5)
-                  bf[nb][2] = prmt(xv.y, xv.w, 0x5410u);  // (x2, x6)
-                  bf[nb][3] = prmt(xv.y, xv.w, 0x7632u);  // (x3, x7)
-                }
-#pragma unroll
-                for (int g = 0; g < C::kRowG; ++g) {
-                  uint32_t pa[4], pb[4];
-                  dequant_int4_word(wa[g][j], pa);
-                  dequant_int4_word(wb[g][j], pb);
-#pragma unroll
-                  for (int nb = 0; nb < C::kNB; ++nb) {
-                    mma_16816(acc[g][nb], pa[0], pb[0], pa[1], pb[1], bf[nb][0], bf[nb][1]);
-                    mma_16816(acc[g][nb], pa[2], pb[2], pa[3], pb[3], bf[nb][2], bf[nb][3]);
-                  }
-                }
-              }
-            } else {
-#pragma unroll
-              for (int j2 = 0; j2 < C::TW / 2; ++j2) {
-                uint32_t bf[C::kNB][4];
-#pragma unroll
-                for (int nb = 0; nb < C::kNB; ++nb) {
-                  uint4 xv = make_uint4(0, 0, 0, 0);
-                  if (valid) xv = lds_v4(xrow[nb] + x_off(xk + 8 * j2));
-                  bf[nb][0] = xv.x; bf[nb][1] = xv.y; bf[nb][2] = xv.z; bf[nb][3] = xv.w;
-                }
-#pragma unroll
-                for (int g = 0; g < C::kRowG; ++g) {
-#pragma unroll
-                  for (int h = 0; h < 2; ++h) {
-                    uint32_t pa[2], pb[2];
-                    dequant_int8_word(wa[g][2 * j2 + h], pa);
-                    dequant_int8_word(wb[g][2 * j2 + h], pb);
-#pragma unroll
-                    for (int nb = 0; nb < C::kNB; ++nb)
-                      mma_16816(acc[g][nb], pa[0], pb[0], pa[1], pb[1], bf[nb][2 * h], bf[nb][2 * h + 1]);
-                  }
-                }
-              }
-            }
-          }
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&empty[stage]);
-          if (++stage == kDecodeStages) { stage = 0; phase ^= 1; }
+  for (int u = u_begin; u < u_end; ++u) {
+    const int p = u / a.tiles;
+    const int t = u - p * a.tiles;
+    const int pk0 = p * a.KPP;
+    const int plen = min(a.KPP, K - pk0);
+    if (p != cur_part) {
+      // stage this part's activations in fragment order (all consumers, then barrier)
+      named_barrier_sync(1, kCT);
+      const int chunks_per_row = plen >> 3;
+      for (int i = ct; i < M * chunks_per_row; i += kCT) {
+        const int n = i / chunks_per_row;
+        const int kr = (i - n * chunks_per_row) << 3;            // part-relative k of 8 values
+        const uint4 v = *reinterpret_cast<const uint4*>(a.X + static_cast<long long>(n) * K + pk0 + kr);
+        const int sg = kr / C::SEGK;
+        const int rem = kr - sg * C::SEGK;
+        const int cc = rem / C::TK;
+        const int jj = (rem - cc * C::TK) >> 3;
+        uint4 o;
+        if constexpr (C::kBits == 4) {
+          o.x = prmt(v.x, v.z, 0x5410u);  // (x0, x4)
+          o.y = prmt(v.x, v.z, 0x7632u);  // (x1, x5)
+          o.z = prmt(v.y, v.w, 0x5410u);  // (x2, x6)
+          o.w = prmt(v.y, v.w, 0x7632u);  // (x3, x7)
+        } else {
+          o = v;
         }
-        // add this warp's K-slice partial into the tile accumulator
-        const uint32_t tbase = acc_u32 + tt * (C::R * 16 * 4);
+        *reinterpret_cast<uint4*>(xbuf + 16u * x_unit<C>(sg, jj, n, cc)) = o;
+      }
+      cur_part = p;
+      named_barrier_sync(1, kCT);
+    }
+
+    float acc[C::kChains][C::kNB][4];
 #pragma unroll
-        for (int g = 0; g < C::kRowG; ++g) {
+    for (int h = 0; h < C::kChains; ++h)
 #pragma unroll
-          for (int nb = 0; nb < C::kNB; ++nb) {
-            const int t0 = 8 * nb + 2 * c;
-            const int ra = 16 * g + r;
-            if (t0 < M) {
-              red_shared_add_f32(tbase + (ra * 16 + t0) * 4, acc[g][nb][0]);
-              red_shared_add_f32(tbase + ((ra + 8) * 16 + t0) * 4, acc[g][nb][2]);
-            }
-            if (t0 + 1 < M) {
-              red_shared_add_f32(tbase + (ra * 16 + t0 + 1) * 4, acc[g][nb][1]);
-              red_shared_add_f32(tbase + ((ra + 8) * 16 + t0 + 1) * 4, acc[g][nb][3]);
-            }
-          }
+      for (int nb = 0; nb < C::kNB; ++nb)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[h][nb][i] = 0.0f;
+
+    const int nst = (plen + C::SK - 1) / C::SK;
+    for (int ks = 0; ks < nst; ++ks) {
+      if (ok && !mbar_wait_warp(&full[stage], phase)) ok = false;
+      const int kseg = ks * C::SK + seg * C::SEGK;               // part-relative k of this warp's segment
+      if (ok && pk0 + kseg < K) {
+        const int sg = ks * kDecodeSegs + seg;                    // segment index within the part
+        const uint32_t box = wring_u32 + stage * kDecodeStageBytes + seg * kDecodeBoxBytes;
+        const uint32_t xseg = xbuf_u32 + 16u * x_unit<C>(sg, 0, 0, 0);
+        if (pk0 + kseg + C::SEGK <= K) {
+          decode_segment<C, false>(box, xseg, wlane, xlane0, xlane1, true, acc);
+        } else {
+          const bool valid = pk0 + kseg + c * C::TK < K;
+          decode_segment<C, true>(box, xseg, wlane, xlane0, xlane1, valid, acc);
         }
       }
-      if (multi) {
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&xempty[xcur]);
-        xb ^= 1;
-        if (xb == 0) xphase ^= 1;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[stage]);
+      if (++stage == kDecodeStages) { stage = 0; phase ^= 1; }
+    }
+
+    // ---- unit epilogue: add the warps' partials, then store or accumulate across parts
+#pragma unroll
+    for (int nb = 0; nb < C::kNB; ++nb) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[0][nb][i] += acc[1][nb][i];
+      const int t0 = 8 * nb + 2 * c;
+      if (t0 < M) {
+        red_shared_add_f32(acc_u32 + (ra * 16 + t0) * 4, acc[0][nb][0]);
+        red_shared_add_f32(acc_u32 + ((ra + 8) * 16 + t0) * 4, acc[0][nb][2]);
+      }
+      if (t0 + 1 < M) {
+        red_shared_add_f32(acc_u32 + (ra * 16 + t0 + 1) * 4, acc[0][nb][1]);
+        red_shared_add_f32(acc_u32 + ((ra + 8) * 16 + t0 + 1) * 4, acc[0][nb][3]);
       }
     }
-    // epilogue of the tile group: scale, round to fp16, store
-    named_barrier_sync(1, kDecodeConsumerWarps * 32);
-    const int ct = threadIdx.x;
-    for (int tt = 0; tt < kTileGroup; ++tt) {
-      const int tile = g0 + tt * G;
-      if (tile >= a.tiles) break;
-      const int row0 = tile * C::R;
-      float* tacc = acc_s + tt * C::R * 16;
-      for (int i = ct; i < M * C::R; i += kDecodeConsumerWarps * 32) {
-        const int m = i / C::R;
-        const int rr = i - m * C::R;
-        const int grow = row0 + rr;
-        const float v = tacc[rr * 16 + m];
-        tacc[rr * 16 + m] = 0.0f;
-        if (grow < N) {
-          const float s = __half2float(a.scale[grow]);
-          a.Y[static_cast<long long>(m) * N + grow] = __float2half_rn(s * v);
+    named_barrier_sync(1, kCT);
+    const int row0 = t * kDecodeRows;
+    const bool split = a.parts > 1;
+    for (int i = ct; i < M * kDecodeRows; i += kCT) {
+      const int m = i / kDecodeRows;
+      const int rr = i - m * kDecodeRows;
+      const int grow = row0 + rr;
+      const float v = acc_s[rr * 16 + m];
+      acc_s[rr * 16 + m] = 0.0f;
+      if (grow < N) {
+        if (split) {
+          atomicAdd(a.ws + static_cast<long long>(m) * N + grow, v);   // result unused: a reduction
+        } else {
+          a.Y[static_cast<long long>(m) * N + grow] = __float2half_rn(__half2float(a.scale[grow]) * v);
         }
       }
     }
-    named_barrier_sync(1, kDecodeConsumerWarps * 32);
+    named_barrier_sync(1, kCT);
   }
   if (!ok && lane == 0) report_error(kErrDecodeConsumerWait);
+}
+
+// Y[m, n] = fp16(s[n] * ws[m, n]) for split decode calls; returns ws to zero.
+__global__ void __launch_bounds__(256) decode_finalize_kernel(float* __restrict__ ws, const __half* __restrict__ scale,
+                                                              __half* __restrict__ Y, int M, int N) {
+  const long long total = static_cast<long long>(M) * N;
+  for (long long i = blockIdx.x * 256LL + threadIdx.x; i < total; i += static_cast<long long>(gridDim.x) * 256) {
+    const int n = static_cast<int>(i % N);
+    const float v = __ldcg(ws + i);
+    ws[i] = 0.0f;
+    Y[i] = __float2half_rn(__half2float(scale[n]) * v);
+  }
 }
 
 }  // namespace glmq

@@ -3,6 +3,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "glmq.h"
@@ -56,11 +57,36 @@ glmq_status current_device(const DeviceInfo** out) {
   return GLMQ_OK;
 }
 
-// Per-device, per-kernel opt-in to large dynamic shared memory.
+// Per-device, per-kernel opt-in to large dynamic shared memory. The attribute is
+// raised only when a launch needs more than was granted before, so steady-state
+// calls make no extra CUDA runtime call. Entries are keyed by the kernel's
+// address (every instantiation of a kernel template has the same type).
+struct SmemGrant {
+  const void* fn;
+  int dev;
+  int bytes;
+};
+constexpr int kMaxGrants = 256;
+SmemGrant g_grants[kMaxGrants];
+int g_num_grants = 0;
+
 template <class Kernel>
 glmq_status allow_smem(Kernel kernel, int bytes) {
-  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  const void* fn = reinterpret_cast<const void*>(kernel);
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e);
+  if (dev < 0 || dev >= kMaxDevices) return GLMQ_ERR_UNSUPPORTED_DEVICE;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  if (bytes > g_devices[dev].smem_optin) return GLMQ_ERR_BAD_SHAPE;
+  SmemGrant* g = nullptr;
+  for (int i = 0; i < g_num_grants; ++i)
+    if (g_grants[i].fn == fn && g_grants[i].dev == dev) g = &g_grants[i];
+  if (g && bytes <= g->bytes) return GLMQ_OK;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (!g && g_num_grants < kMaxGrants) g = &g_grants[g_num_grants++];
+  if (g) *g = SmemGrant{fn, dev, bytes};
   return GLMQ_OK;
 }
 
@@ -108,56 +134,7 @@ glmq_status launch_quantize(const void* W, int64_t N, int64_t K, void* packed, v
   return launch_quantize_cpt<BITS, 32>(W, N, K, packed, scale, s);
 }
 
-// ---------------------------------------------------------------- decode
-template <class C>
-glmq_status launch_decode_cfg(const DeviceInfo& dev, const void* X, int M, const void* packed, const void* scale,
-                              int N, int K, void* Y, cudaStream_t s) {
-  const int barrier_bytes = 128;
-  const int avail = dev.smem_optin - (kDecodeStages * C::STAGE_BYTES + C::ACC_BYTES + barrier_bytes);
-  DecodeArgs a;
-  a.X = static_cast<const __half*>(X);
-  a.packed = static_cast<const uint8_t*>(packed);
-  a.scale = static_cast<const __half*>(scale);
-  a.Y = static_cast<__half*>(Y);
-  a.M = M;
-  a.N = N;
-  a.K = K;
-  const int k_round = (K + C::SK - 1) / C::SK * C::SK;
-  const int xp1 = static_cast<int>(x_pitch(k_round, C::XSHIFT));
-  if (static_cast<long long>(M) * xp1 <= avail) {
-    a.KP = k_round;
-    a.passes = 1;
-    a.XP = xp1;
-    a.xbufs = 1;
-  } else {
-    int kp = 0;
-    for (int cand = C::SK; cand < k_round; cand += C::SK) {
-      if (2LL * M * x_pitch(cand, C::XSHIFT) <= avail) kp = cand; else break;
-    }
-    if (kp == 0) return GLMQ_ERR_BAD_SHAPE;
-    a.KP = kp;
-    a.passes = (K + kp - 1) / kp;
-    a.XP = static_cast<int>(x_pitch(kp, C::XSHIFT));
-    a.xbufs = 2;
-  }
-  a.tiles = (N + C::R - 1) / C::R;
-  const int smem = kDecodeStages * C::STAGE_BYTES + C::ACC_BYTES + a.xbufs * M * a.XP + barrier_bytes;
-  glmq_status st = allow_smem(decode_kernel<C>, smem);
-  if (st != GLMQ_OK) return st;
-  const int grid = a.tiles < dev.sms ? a.tiles : dev.sms;
-  decode_kernel<C><<<grid, kDecodeThreads, smem, s>>>(a);
-  cudaError_t e = cudaGetLastError();
-  return e == cudaSuccess ? GLMQ_OK : cuda_fail(e);
-}
-
-template <int BITS>
-glmq_status launch_decode(const DeviceInfo& dev, const void* X, int M, const void* packed, const void* scale, int N,
-                          int K, void* Y, cudaStream_t s) {
-  if (M <= 8) return launch_decode_cfg<DecodeCfg<BITS, 1, 128, 2>>(dev, X, M, packed, scale, N, K, Y, s);
-  return launch_decode_cfg<DecodeCfg<BITS, 2, 64, 2>>(dev, X, M, packed, scale, N, K, Y, s);
-}
-
-// ---------------------------------------------------------------- prefill
+// ---------------------------------------------------------------- TMA descriptors
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                    CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
@@ -189,6 +166,109 @@ glmq_status make_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void*
   return GLMQ_OK;
 }
 
+// ---------------------------------------------------------------- decode scratch
+// fp32 [M, N] partial sums for decode calls whose tiles are split over several K
+// parts. Allocated once per device on first use (grown when a larger problem
+// arrives) and zeroed at allocation; the finalize kernel returns it to zero.
+struct DecodeScratch {
+  float* ws = nullptr;
+  size_t ws_elems = 0;
+};
+DecodeScratch g_scratch[kMaxDevices];
+
+glmq_status decode_scratch(size_t ws_elems, float** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  std::lock_guard<std::mutex> lock(g_mutex);
+  DecodeScratch& sc = g_scratch[dev];
+  if (sc.ws_elems < ws_elems) {
+    if (sc.ws) cudaFree(sc.ws);
+    sc.ws = nullptr;
+    sc.ws_elems = 0;
+    if ((e = cudaMalloc(&sc.ws, ws_elems * sizeof(float))) != cudaSuccess) return cuda_fail(e);
+    if ((e = cudaMemset(sc.ws, 0, ws_elems * sizeof(float))) != cudaSuccess) return cuda_fail(e);
+    sc.ws_elems = ws_elems;
+  }
+  *out = sc.ws;
+  return GLMQ_OK;
+}
+
+// ---------------------------------------------------------------- decode
+struct DecodePlan {
+  int KPP, parts, tiles, units, smem, grid;
+};
+
+// Choose the K-part length: the fewest parts whose activation slice fits in
+// shared memory. Splitting a tile over parts costs a second (finalize) launch and
+// a round trip of fp32 partial sums, so it is used only when X does not fit.
+template <class C>
+bool plan_decode(const DeviceInfo& dev, int N, int K, DecodePlan* pl) {
+  const int x_budget = dev.smem_optin - kDecodeFixedSmem - 1024;
+  const int k_round = (K + C::SK - 1) / C::SK * C::SK;
+  int kpp_max = x_budget / (2 * C::kMP) / C::SK * C::SK;
+  if (kpp_max < C::SK) return false;
+  if (kpp_max > k_round) kpp_max = k_round;
+  const int chunks = k_round / C::SK;
+  const int parts_min = (k_round + kpp_max - 1) / kpp_max;
+  pl->KPP = (chunks + parts_min - 1) / parts_min * C::SK;
+  pl->parts = (K + pl->KPP - 1) / pl->KPP;
+  pl->tiles = (N + kDecodeRows - 1) / kDecodeRows;
+  const long long units = static_cast<long long>(pl->parts) * pl->tiles;
+  if (units > 0x7fffffffLL) return false;
+  pl->units = static_cast<int>(units);
+  pl->grid = pl->units < dev.sms ? pl->units : dev.sms;
+  pl->smem = kDecodeFixedSmem + 1024 + 2 * C::kMP * pl->KPP;
+  return pl->smem <= dev.smem_optin;
+}
+
+template <class C>
+glmq_status launch_decode_cfg(const DeviceInfo& dev, const void* X, int M, const void* packed, const void* scale,
+                              int N, int K, void* Y, cudaStream_t s) {
+  DecodePlan pl;
+  if (!plan_decode<C>(dev, N, K, &pl)) return GLMQ_ERR_BAD_SHAPE;
+  CUtensorMap tw;
+  const uint64_t row_bytes = uint64_t(K) / C::KPB;
+  glmq_status st = make_map_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, packed, row_bytes, N, row_bytes, kDecodeSegB,
+                               kDecodeRows, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st != GLMQ_OK) return st;
+  DecodeArgs a;
+  a.X = static_cast<const __half*>(X);
+  a.scale = static_cast<const __half*>(scale);
+  a.Y = static_cast<__half*>(Y);
+  a.ws = nullptr;
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.KPP = pl.KPP;
+  a.parts = pl.parts;
+  a.tiles = pl.tiles;
+  a.units = pl.units;
+  if (pl.parts > 1 && (st = decode_scratch(static_cast<size_t>(M) * N, &a.ws)) != GLMQ_OK) return st;
+  if ((st = allow_smem(decode_kernel<C>, pl.smem)) != GLMQ_OK) return st;
+  decode_kernel<C><<<pl.grid, kDecodeThreads, pl.smem, s>>>(tw, a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (pl.parts > 1) {
+    const long long total = static_cast<long long>(M) * N;
+    const int blocks = static_cast<int>(std::min<long long>((total + 255) / 256, 4LL * dev.sms));
+    decode_finalize_kernel<<<blocks, 256, 0, s>>>(a.ws, a.scale, a.Y, M, N);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e);
+  }
+  return GLMQ_OK;
+}
+
+template <int BITS>
+glmq_status launch_decode(const DeviceInfo& dev, const void* X, int M, const void* packed, const void* scale, int N,
+                          int K, void* Y, cudaStream_t s) {
+  if (M <= 1) return launch_decode_cfg<DecodeCfg<BITS, 1>>(dev, X, M, packed, scale, N, K, Y, s);
+  if (M <= 2) return launch_decode_cfg<DecodeCfg<BITS, 2>>(dev, X, M, packed, scale, N, K, Y, s);
+  if (M <= 4) return launch_decode_cfg<DecodeCfg<BITS, 4>>(dev, X, M, packed, scale, N, K, Y, s);
+  if (M <= 8) return launch_decode_cfg<DecodeCfg<BITS, 8>>(dev, X, M, packed, scale, N, K, Y, s);
+  return launch_decode_cfg<DecodeCfg<BITS, 16>>(dev, X, M, packed, scale, N, K, Y, s);
+}
+
+// ---------------------------------------------------------------- prefill
 template <class C>
 glmq_status launch_prefill_cfg(const DeviceInfo& dev, const void* X, int M, const void* packed, const void* scale,
                                int N, int K, void* Y, cudaStream_t s) {
@@ -312,6 +392,14 @@ glmq_status glmq_last_device_error(void* stream, uint32_t* flags) {
   if (word == 0) return GLMQ_OK;
   const unsigned int zero = 0;
   if ((e = cudaMemcpyToSymbol(glmq::g_device_status, &zero, sizeof(zero))) != cudaSuccess) return cuda_fail(e);
+  // a kernel that gave up may have left decode scratch non-zero: restore the invariant
+  int dev = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return cuda_fail(e);
+  {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    DecodeScratch& sc = g_scratch[dev];
+    if (sc.ws && (e = cudaMemset(sc.ws, 0, sc.ws_elems * sizeof(float))) != cudaSuccess) return cuda_fail(e);
+  }
   return GLMQ_ERR_DEVICE;
 }
 

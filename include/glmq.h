@@ -116,6 +116,34 @@ GLMQ_API glmq_status glmq_gemm_decode(const void* X, int64_t M, const void* pack
 GLMQ_API glmq_status glmq_gemm_prefill(const void* X, int64_t M, const void* packed, const void* scale,
                               int64_t N, int64_t K, int bits, void* Y, void* stream);
 
+/*
+ * glmq_gemm_decode without any device allocation (the paper has no counterpart:
+ * this is a deployment variant of the decode kernel).
+ *
+ * Some callers cannot call cudaMalloc: code that runs while a stream is being
+ * captured into a CUDA graph (allocation is not a capturable operation), code
+ * embedded under an allocator that owns the whole device-memory budget (a
+ * framework's caching pool, a fixed-size arena on a shared serving GPU), and
+ * latency-critical paths that must not block in the driver after start-up.
+ * glmq_gemm_decode may allocate its split-K scratch on first use; this entry
+ * point never does. Its scratch is a fixed, statically allocated device array of
+ * GLMQ_NOALLOC_SCRATCH_FLOATS fp32 values (4 MiB) that every GPU which loads the
+ * library holds until the process exits.
+ *   - Same arguments, layout and results as glmq_gemm_decode (M <= 16).
+ *   - Requires M * N <= GLMQ_NOALLOC_SCRATCH_FLOATS, else GLMQ_ERR_BAD_SHAPE and
+ *     nothing is enqueued.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress, no allocation); make that first call before any
+ *     stream capture on that device.
+ *   - All calls share the one array, and it keeps the last call's contents: the
+ *     part a call needs zeroed is cleared on its stream before use. Calls that
+ *     overlap on the GPU (different streams, no ordering between them) race on
+ *     the array and may produce wrong results.
+ */
+#define GLMQ_NOALLOC_SCRATCH_FLOATS (1u << 20)
+GLMQ_API glmq_status glmq_gemm_decode_noalloc(const void* X, int64_t M, const void* packed, const void* scale,
+                                              int64_t N, int64_t K, int bits, void* Y, void* stream);
+
 /* Static description of a status code. Never NULL. */
 GLMQ_API const char* glmq_status_string(int status);
 

@@ -26,6 +26,7 @@ ERR_UNSUPPORTED_DEVICE = 7
 
 DECODE_MAX_M = 16
 MAX_K = 65536
+NOALLOC_SCRATCH_FLOATS = 1 << 20
 
 #: every symbol include/glmq.h declares, with (restype, argtypes)
 _c_int64 = ctypes.c_int64
@@ -37,6 +38,8 @@ SIGNATURES = {
     "glmq_gemm": (ctypes.c_int, [_vp, _c_int64, _vp, _vp, _c_int64, _c_int64, ctypes.c_int, _vp, _vp]),
     "glmq_gemm_decode": (ctypes.c_int, [_vp, _c_int64, _vp, _vp, _c_int64, _c_int64, ctypes.c_int, _vp, _vp]),
     "glmq_gemm_prefill": (ctypes.c_int, [_vp, _c_int64, _vp, _vp, _c_int64, _c_int64, ctypes.c_int, _vp, _vp]),
+    "glmq_gemm_decode_noalloc": (ctypes.c_int, [_vp, _c_int64, _vp, _vp, _c_int64, _c_int64, ctypes.c_int, _vp,
+                                                _vp]),
     "glmq_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "glmq_last_cuda_error": (ctypes.c_int, []),
     "glmq_last_device_error": (ctypes.c_int, [_vp, ctypes.POINTER(ctypes.c_uint32)]),
@@ -99,7 +102,8 @@ def raw_quantize(W: int, N: int, K: int, bits: int, packed: int, scale: int, str
 
 def raw_gemm(X: int, M: int, packed: int, scale: int, N: int, K: int, bits: int, Y: int, stream: int = 0,
              route: str = "auto") -> int:
-    fn = {"auto": lib().glmq_gemm, "decode": lib().glmq_gemm_decode, "prefill": lib().glmq_gemm_prefill}[route]
+    fn = {"auto": lib().glmq_gemm, "decode": lib().glmq_gemm_decode, "prefill": lib().glmq_gemm_prefill,
+          "decode_noalloc": lib().glmq_gemm_decode_noalloc}[route]
     return fn(X, M, packed, scale, N, K, bits, Y, stream)
 
 

@@ -308,6 +308,84 @@ glmq_status launch_prefill(const DeviceInfo& dev, const void* X, int M, const vo
   return launch_prefill_cfg<PrefillCfg<BITS, 256>>(dev, X, M, packed, scale, N, K, Y, s);
 }
 
+// ---------------------------------------------------------------- decode without allocation
+// Callers that must not allocate device memory (see glmq_gemm_decode_noalloc in
+// glmq.h) get the decode kernel with its split-K partial sums kept in this fixed
+// array instead of the lazily allocated scratch. It is static storage: every GPU
+// that loads the library holds it until the process exits. Host code must not use
+// the array's name as a device address: the address is obtained per device with
+// cudaGetSymbolAddress.
+constexpr size_t kNoAllocScratchFloats = size_t(1) << 20;   // 4 MiB per device
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchFloats];
+float* g_noalloc_scratch_ptr[kMaxDevices];
+
+// Device address of g_noalloc_scratch on the current device (looked up once per device).
+glmq_status noalloc_scratch(float** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (dev < 0 || dev >= kMaxDevices) return GLMQ_ERR_UNSUPPORTED_DEVICE;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  if (!g_noalloc_scratch_ptr[dev]) {
+    void* p = nullptr;
+    if ((e = cudaGetSymbolAddress(&p, g_noalloc_scratch)) != cudaSuccess) return cuda_fail(e);
+    g_noalloc_scratch_ptr[dev] = static_cast<float*>(p);
+  }
+  *out = g_noalloc_scratch_ptr[dev];
+  return GLMQ_OK;
+}
+
+template <class C>
+glmq_status launch_decode_noalloc_cfg(const DeviceInfo& dev, const void* X, int M, const void* packed,
+                                      const void* scale, int N, int K, void* Y, cudaStream_t s) {
+  DecodePlan pl;
+  if (!plan_decode<C>(dev, N, K, &pl)) return GLMQ_ERR_BAD_SHAPE;
+  CUtensorMap tw;
+  const uint64_t row_bytes = uint64_t(K) / C::KPB;
+  glmq_status st = make_map_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, packed, row_bytes, N, row_bytes, kDecodeSegB,
+                               kDecodeRows, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st != GLMQ_OK) return st;
+  DecodeArgs a;
+  a.X = static_cast<const __half*>(X);
+  a.scale = static_cast<const __half*>(scale);
+  a.Y = static_cast<__half*>(Y);
+  a.ws = nullptr;
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.KPP = pl.KPP;
+  a.parts = pl.parts;
+  a.tiles = pl.tiles;
+  a.units = pl.units;
+  cudaError_t e;
+  if (pl.parts > 1) {
+    if ((st = noalloc_scratch(&a.ws)) != GLMQ_OK) return st;
+    // the partial sums must start at zero; the array keeps whatever the last call left
+    if ((e = cudaMemsetAsync(a.ws, 0, static_cast<size_t>(M) * N * sizeof(float), s)) != cudaSuccess)
+      return cuda_fail(e);
+  }
+  if ((st = allow_smem(decode_kernel<C>, pl.smem)) != GLMQ_OK) return st;
+  decode_kernel<C><<<pl.grid, kDecodeThreads, pl.smem, s>>>(tw, a);
+  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e);
+  if (pl.parts > 1) {
+    const long long total = static_cast<long long>(M) * N;
+    const int blocks = static_cast<int>(std::min<long long>((total + 255) / 256, 4LL * dev.sms));
+    decode_finalize_kernel<<<blocks, 256, 0, s>>>(a.ws, a.scale, a.Y, M, N);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e);
+  }
+  return GLMQ_OK;
+}
+
+template <int BITS>
+glmq_status launch_decode_noalloc(const DeviceInfo& dev, const void* X, int M, const void* packed, const void* scale,
+                                  int N, int K, void* Y, cudaStream_t s) {
+  if (M <= 1) return launch_decode_noalloc_cfg<DecodeCfg<BITS, 1>>(dev, X, M, packed, scale, N, K, Y, s);
+  if (M <= 2) return launch_decode_noalloc_cfg<DecodeCfg<BITS, 2>>(dev, X, M, packed, scale, N, K, Y, s);
+  if (M <= 4) return launch_decode_noalloc_cfg<DecodeCfg<BITS, 4>>(dev, X, M, packed, scale, N, K, Y, s);
+  if (M <= 8) return launch_decode_noalloc_cfg<DecodeCfg<BITS, 8>>(dev, X, M, packed, scale, N, K, Y, s);
+  return launch_decode_noalloc_cfg<DecodeCfg<BITS, 16>>(dev, X, M, packed, scale, N, K, Y, s);
+}
+
 enum class Route { kAuto, kDecode, kPrefill };
 
 glmq_status gemm_entry(Route route, const void* X, int64_t M, const void* packed, const void* scale, int64_t N,
@@ -365,6 +443,21 @@ glmq_status glmq_gemm_decode(const void* X, int64_t M, const void* packed, const
 glmq_status glmq_gemm_prefill(const void* X, int64_t M, const void* packed, const void* scale, int64_t N, int64_t K,
                               int bits, void* Y, void* stream) {
   return gemm_entry(Route::kPrefill, X, M, packed, scale, N, K, bits, Y, stream);
+}
+
+glmq_status glmq_gemm_decode_noalloc(const void* X, int64_t M, const void* packed, const void* scale, int64_t N,
+                                     int64_t K, int bits, void* Y, void* stream) {
+  glmq_status st = check_gemm(X, M, packed, scale, N, K, bits, Y);
+  if (st != GLMQ_OK) return st;
+  if (M > GLMQ_DECODE_MAX_M) return GLMQ_ERR_BAD_SHAPE;
+  if (static_cast<size_t>(M) * static_cast<size_t>(N) > kNoAllocScratchFloats) return GLMQ_ERR_BAD_SHAPE;
+  if (M == 0 || N == 0) return GLMQ_OK;
+  const DeviceInfo* dev = nullptr;
+  if ((st = current_device(&dev)) != GLMQ_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int m = static_cast<int>(M), n = static_cast<int>(N), k = static_cast<int>(K);
+  return bits == 4 ? launch_decode_noalloc<4>(*dev, X, m, packed, scale, n, k, Y, s)
+                   : launch_decode_noalloc<8>(*dev, X, m, packed, scale, n, k, Y, s);
 }
 
 const char* glmq_status_string(int status) {

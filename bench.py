@@ -509,6 +509,33 @@ def run_sweep(args, world, rank, local):
             "gpu_launches": 4 * layers * args.steps, "clocks": clk}
 
 
+# ----------------------------------------------------------------------------- one launch (profiling)
+def run_one(args, world, rank, local):
+    """A handful of glmq_gemm (or glmq_quantize) launches on one GLM projection, for ncu captures."""
+    import torch
+    import int8_quantized_glmq_b200 as glmq
+    from inputs import GLM_PROJECTIONS
+
+    N, K = GLM_PROJECTIONS[args.proj]
+    g = torch.Generator(device="cuda").manual_seed(1000)
+    W = torch.empty((N, K), dtype=torch.float16, device="cuda").normal_(0.0, 0.02, generator=g)
+    packed, scale = glmq.quantize(W, args.bits)
+    if args.op == "gemm":
+        del W
+        X = torch.randn((args.m, K), generator=g, device="cuda", dtype=torch.float32).half()
+        Y = torch.empty((args.m, N), dtype=torch.float16, device="cuda")
+        fn = lambda: glmq.gemm(X, packed, scale, args.bits, out=Y)  # noqa: E731
+        work = {"bytes": packed.numel() + scale.numel() * 2 + X.numel() * 2 + Y.numel() * 2,
+                "flops": 2.0 * args.m * N * K}
+    else:
+        fn = lambda: glmq.quantize(W, args.bits, out=(packed, scale))  # noqa: E731
+        work = {"bytes": W.numel() * 2 + packed.numel() + scale.numel() * 2, "flops": 0.0}
+    t = time_launches(torch, fn, args.steps, warmup=args.warmup)
+    return {"workload": "one", "op": args.op, "proj": args.proj, "N": N, "K": K, "M": args.m, "bits": args.bits,
+            "us": round(t * 1e6, 2), "gbs": round(work["bytes"] / t / 1e9, 1),
+            "tflops": round(work["flops"] / t / 1e12, 1), "algorithmic_bytes": work["bytes"]}
+
+
 # ----------------------------------------------------------------------------- main
 def main():
     ap = argparse.ArgumentParser()
@@ -516,7 +543,11 @@ def main():
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="decode", choices=["decode", "sweep"])
+    ap.add_argument("--workload", default="decode", choices=["decode", "sweep", "one"])
+    ap.add_argument("--proj", default="attn_out", choices=["qkv", "attn_out", "ffn_up", "ffn_down"])
+    ap.add_argument("--op", default="gemm", choices=["gemm", "quantize"])
+    ap.add_argument("--m", type=int, default=1)
+    ap.add_argument("--bits", type=int, default=4, choices=[4, 8])
     ap.add_argument("--layers", type=int, default=70)
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -535,6 +566,8 @@ def main():
     world, rank, local = dist_setup()
     if args.workload == "sweep":
         res = run_sweep(args, world, rank, local)
+    elif args.workload == "one":
+        res = run_one(args, world, rank, local)
     else:
         res = run_decode(args, world, rank, local)
         if rank == 0 and world == 1 and not args.no_cpu_baseline:

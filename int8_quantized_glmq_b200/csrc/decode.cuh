@@ -104,6 +104,19 @@ __device__ __forceinline__ void dequant_int4_word(uint32_t w, uint32_t (&p)[4]) 
   p[3] = *reinterpret_cast<uint32_t*>(&r3);
 }
 
+// INT4, biased form: the same pairs without the final subtraction. Low nibbles give
+// the fp16 integers 1032 + q, high nibbles 1152 + 16 q; the MMA's B operand holds x
+// for low-nibble slots and x / 16 for high-nibble slots, so every product is
+// q * x + (a bias depending only on x), and the accumulated bias is removed per
+// segment (see decode_segment). Four LOP3 and one shift per 8 codes.
+__device__ __forceinline__ void dequant_int4_word_biased(uint32_t w, uint32_t (&p)[4]) {
+  const uint32_t w8 = w >> 8;
+  p[0] = lop3_and_xor(w, 0x000F000Fu, 0x64086408u);
+  p[1] = lop3_and_xor(w, 0x00F000F0u, 0x64806480u);
+  p[2] = lop3_and_xor(w8, 0x000F000Fu, 0x64086408u);
+  p[3] = lop3_and_xor(w8, 0x00F000F0u, 0x64806480u);
+}
+
 // INT8: one word (4 codes, k = 0..3) -> half2 pairs (0,1), (2,3).
 __device__ __forceinline__ void dequant_int8_word(uint32_t w, uint32_t (&p)[2]) {
   const __half2 kBias = __halves2half2(__ushort_as_half(0xE480), __ushort_as_half(0xE480));  // -1152
@@ -138,7 +151,8 @@ __host__ __device__ constexpr uint32_t x_unit(int sg, int jj, int n, int c) {
 // ra + 8, against the staged activations. kTail: some lanes' codes lie past K.
 template <class C, bool kTail>
 __device__ __forceinline__ void decode_segment(uint32_t box, uint32_t xseg, uint32_t wlane, uint32_t xlane0,
-                                               uint32_t xlane1, bool valid, float (&acc)[C::kChains][C::kNB][4]) {
+                                               uint32_t xlane1, bool valid, const float* bias_seg, int c,
+                                               float (&acc)[C::kChains][C::kNB][4]) {
   constexpr uint32_t kJStride = static_cast<uint32_t>(C::kMP) * 64u;   // bytes between consecutive jj
   uint32_t wa[C::TW], wb[C::TW];
 #pragma unroll
@@ -163,13 +177,22 @@ __device__ __forceinline__ void decode_segment(uint32_t box, uint32_t xseg, uint
         if (!kTail || valid) bf[nb] = lds_v4(xseg + (nb ? xlane1 : xlane0) + j * kJStride);
       }
       uint32_t pa[4], pb[4];
-      dequant_int4_word(wa[j], pa);
-      dequant_int4_word(wb[j], pb);
+      dequant_int4_word_biased(wa[j], pa);
+      dequant_int4_word_biased(wb[j], pb);
 #pragma unroll
       for (int nb = 0; nb < C::kNB; ++nb) {
         mma_16816(acc[0][nb], pa[0], pb[0], pa[1], pb[1], bf[nb].x, bf[nb].y);
         mma_16816(acc[1][nb], pa[2], pb[2], pa[3], pb[3], bf[nb].z, bf[nb].w);
       }
+    }
+    // remove the bias this segment added: bias_seg[t] = sum_k (1032 or 1152) * B[k][t]
+#pragma unroll
+    for (int nb = 0; nb < C::kNB; ++nb) {
+      const float2 b = *reinterpret_cast<const float2*>(bias_seg + 8 * nb + 2 * c);
+      acc[0][nb][0] -= b.x;
+      acc[0][nb][2] -= b.x;
+      acc[0][nb][1] -= b.y;
+      acc[0][nb][3] -= b.y;
     }
   } else {
 #pragma unroll
@@ -205,6 +228,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kDecodeStages * kDecodeStageBytes + kDecodeAccBytes);
   uint64_t* empty = full + kDecodeStages;
   uint8_t* xbuf = smem + kDecodeFixedSmem;
+  // INT4 only: per (segment, token) bias of the biased dequantization, after the activation slice
+  float* bias_s = reinterpret_cast<float*>(xbuf + 2 * C::kMP * a.KPP);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -301,14 +326,47 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         const int jj = (rem - cc * C::TK) >> 3;
         uint4 o;
         if constexpr (C::kBits == 4) {
-          o.x = prmt(v.x, v.z, 0x5410u);  // (x0, x4)
-          o.y = prmt(v.x, v.z, 0x7632u);  // (x1, x5)
-          o.z = prmt(v.y, v.w, 0x5410u);  // (x2, x6)
-          o.w = prmt(v.y, v.w, 0x7632u);  // (x3, x7)
+          // low-nibble slots (x0,x4), (x2,x6) as is; high-nibble slots (x1,x5), (x3,x7) divided by 16
+          const __half2 kSixteenth = __halves2half2(__ushort_as_half(0x2C00), __ushort_as_half(0x2C00));
+          o.x = prmt(v.x, v.z, 0x5410u);
+          uint32_t hy = prmt(v.x, v.z, 0x7632u);
+          o.z = prmt(v.y, v.w, 0x5410u);
+          uint32_t hw = prmt(v.y, v.w, 0x7632u);
+          __half2 sy = __hmul2(*reinterpret_cast<__half2*>(&hy), kSixteenth);
+          __half2 sw = __hmul2(*reinterpret_cast<__half2*>(&hw), kSixteenth);
+          o.y = *reinterpret_cast<uint32_t*>(&sy);
+          o.w = *reinterpret_cast<uint32_t*>(&sw);
         } else {
           o = v;
         }
         *reinterpret_cast<uint4*>(xbuf + 16u * x_unit<C>(sg, jj, n, cc)) = o;
+      }
+      if constexpr (C::kBits == 4) {
+        // per (segment, token) bias sum_k (1032 or 1152) * B[k], one warp per real pair
+        // (lane = 8-value chunk of the 256-k segment), read back from the staged slice
+        static_assert(C::SEGK == 256, "one lane per 8-value chunk of a segment");
+        named_barrier_sync(1, kCT);
+        const int nseg = a.KPP / C::SEGK;
+        const int pseg = (plen + C::SEGK - 1) / C::SEGK;
+        for (int i = ct; i < nseg * 16; i += kCT) {                // entries the pair loop never writes
+          if ((i & 15) >= M || (i >> 4) >= pseg) bias_s[i] = 0.0f;
+        }
+        for (int pair = warp; pair < pseg * M; pair += kDecodeConsumerWarps) {
+          const int sg = pair / M;
+          const int n = pair - sg * M;
+          float bias = 0.0f;
+          if (sg * C::SEGK + lane * 8 < plen) {
+            const uint4 o = *reinterpret_cast<const uint4*>(xbuf + 16u * x_unit<C>(sg, lane & 7, n, lane >> 3));
+            const float2 fx = __half22float2(*reinterpret_cast<const __half2*>(&o.x));
+            const float2 fy = __half22float2(*reinterpret_cast<const __half2*>(&o.y));
+            const float2 fz = __half22float2(*reinterpret_cast<const __half2*>(&o.z));
+            const float2 fw = __half22float2(*reinterpret_cast<const __half2*>(&o.w));
+            bias = 1032.0f * ((fx.x + fx.y) + (fz.x + fz.y)) + 1152.0f * ((fy.x + fy.y) + (fw.x + fw.y));
+          }
+#pragma unroll
+          for (int off = 16; off > 0; off >>= 1) bias += __shfl_xor_sync(0xffffffffu, bias, off);
+          if (lane == 0) bias_s[sg * 16 + n] = bias;
+        }
       }
       cur_part = p;
       named_barrier_sync(1, kCT);
@@ -330,11 +388,12 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         const int sg = ks * kDecodeSegs + seg;                    // segment index within the part
         const uint32_t box = wring_u32 + stage * kDecodeStageBytes + seg * kDecodeBoxBytes;
         const uint32_t xseg = xbuf_u32 + 16u * x_unit<C>(sg, 0, 0, 0);
+        const float* bias_seg = bias_s + sg * 16;
         if (pk0 + kseg + C::SEGK <= K) {
-          decode_segment<C, false>(box, xseg, wlane, xlane0, xlane1, true, acc);
+          decode_segment<C, false>(box, xseg, wlane, xlane0, xlane1, true, bias_seg, c, acc);
         } else {
           const bool valid = pk0 + kseg + c * C::TK < K;
-          decode_segment<C, true>(box, xseg, wlane, xlane0, xlane1, valid, acc);
+          decode_segment<C, true>(box, xseg, wlane, xlane0, xlane1, valid, bias_seg, c, acc);
         }
       }
       __syncwarp();

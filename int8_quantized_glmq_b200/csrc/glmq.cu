@@ -206,7 +206,10 @@ template <class C>
 bool plan_decode(const DeviceInfo& dev, int N, int K, DecodePlan* pl) {
   const int x_budget = dev.smem_optin - kDecodeFixedSmem - 1024;
   const int k_round = (K + C::SK - 1) / C::SK * C::SK;
-  int kpp_max = x_budget / (2 * C::kMP) / C::SK * C::SK;
+  // per k of a part: 2 * MP bytes of activations, plus (INT4) 16 floats of bias per segment
+  const int per_k = 2 * C::kMP;
+  const int per_seg_bias = (C::kBits == 4) ? 16 * 4 : 0;
+  int kpp_max = x_budget / (per_k + per_seg_bias / C::SEGK + 1) / C::SK * C::SK;
   if (kpp_max < C::SK) return false;
   if (kpp_max > k_round) kpp_max = k_round;
   const int chunks = k_round / C::SK;
@@ -218,7 +221,7 @@ bool plan_decode(const DeviceInfo& dev, int N, int K, DecodePlan* pl) {
   if (units > 0x7fffffffLL) return false;
   pl->units = static_cast<int>(units);
   pl->grid = pl->units < dev.sms ? pl->units : dev.sms;
-  pl->smem = kDecodeFixedSmem + 1024 + 2 * C::kMP * pl->KPP;
+  pl->smem = kDecodeFixedSmem + 1024 + 2 * C::kMP * pl->KPP + per_seg_bias * (pl->KPP / C::SEGK);
   return pl->smem <= dev.smem_optin;
 }
 

@@ -60,8 +60,11 @@ extern "C" {
 
 #define GLMQ_ABI_VERSION 1
 #define GLMQ_MAX_K 65536
-/* Largest M served by the decode (register-dequant GEMV) kernel in glmq_gemm. */
+/* Largest M the decode (register-dequant GEMV) kernel accepts (glmq_gemm_decode). */
 #define GLMQ_DECODE_MAX_M 16
+/* glmq_gemm sends M <= GLMQ_DECODE_AUTO_MAX_M to the decode kernel and larger M to the
+ * tensor-core kernel, which splits tiles over K when there are fewer tiles than SMs. */
+#define GLMQ_DECODE_AUTO_MAX_M 8
 
 typedef enum glmq_status {
   GLMQ_OK = 0,
@@ -101,9 +104,12 @@ GLMQ_API glmq_status glmq_quantize(const void* W, int64_t N, int64_t K, int bits
  *   packed  in : codes from glmq_quantize (same N, K, bits)
  *   scale   in : fp16 [N]
  *   Y       out: fp16 [M, N]; must not overlap any input
- * Dispatch: M <= GLMQ_DECODE_MAX_M runs the decode kernel (HBM-bound stream of
- * the packed weights, register dequantization); larger M runs the tensor-core
- * prefill kernel. Both give results within the documented accuracy.
+ * Dispatch: M <= GLMQ_DECODE_AUTO_MAX_M runs the decode kernel (HBM-bound stream
+ * of the packed weights, register dequantization, warp-level MMA); larger M runs
+ * the tcgen05 tensor-core kernel. Both give results within the documented accuracy.
+ * Either kernel may split tiles over K parts; it then accumulates fp32 partial sums
+ * in a per-device scratch buffer that the library allocates on first use (call once
+ * outside stream capture before capturing) and runs a second, finalize kernel.
  */
 GLMQ_API glmq_status glmq_gemm(const void* X, int64_t M, const void* packed, const void* scale, int64_t N,
                       int64_t K, int bits, void* Y, void* stream);

@@ -10,6 +10,7 @@
 #include "decode.cuh"
 #include "prefill.cuh"
 #include "quantize.cuh"
+#include "skinny.cuh"
 
 namespace {
 
@@ -272,6 +273,28 @@ glmq_status launch_decode(const DeviceInfo& dev, const void* X, int M, const voi
 }
 
 // ---------------------------------------------------------------- prefill
+// Choose K parts for `tiles` tiles of `num_steps` K steps each: only when there are
+// fewer tiles than SMs, the split that spreads (tile, part) units most evenly,
+// preferring fewer parts (each split tile costs a round trip of fp32 partial sums
+// through the scratch buffer and a finalize launch).
+int plan_parts(int tiles, int num_steps, int min_steps_per_part, int sms) {
+  int parts = 1;
+  if (tiles < sms) {
+    double best = 0.0;
+    for (int P = 1; P <= 16 && P * min_steps_per_part <= num_steps; ++P) {
+      const int units = tiles * P;
+      const int grid = units < sms ? units : sms;
+      const double eff = (static_cast<double>(units) / grid) / ((units + grid - 1) / grid) *
+                         (static_cast<double>(grid) / sms);
+      if (eff > best + 0.02) {
+        best = eff;
+        parts = P;
+      }
+    }
+  }
+  return parts;
+}
+
 template <class C>
 glmq_status launch_prefill_cfg(const DeviceInfo& dev, const void* X, int M, const void* packed, const void* scale,
                                int N, int K, void* Y, cudaStream_t s) {
@@ -286,27 +309,85 @@ glmq_status launch_prefill_cfg(const DeviceInfo& dev, const void* X, int M, cons
   PrefillArgs a;
   a.scale = static_cast<const __half*>(scale);
   a.Y = static_cast<__half*>(Y);
+  a.ws = nullptr;
   a.M = M;
   a.N = N;
   a.K = K;
   a.tiles_m = (M + C::kBN - 1) / C::kBN;
   const long long tiles = static_cast<long long>((N + C::BM - 1) / C::BM) * a.tiles_m;
-  if (tiles > 0x7fffffffLL) return GLMQ_ERR_BAD_SHAPE;
+  if (tiles > 0x7fffffffLL / 64) return GLMQ_ERR_BAD_SHAPE;
   a.tiles = static_cast<int>(tiles);
+  const int num_kb = K / C::BK;
+  const int parts = plan_parts(a.tiles, num_kb, 4, dev.sms);
+  a.kbp = (num_kb + parts - 1) / parts;
+  a.parts = (num_kb + a.kbp - 1) / a.kbp;
+  a.units = a.tiles * a.parts;
+  if (a.parts > 1 && (st = decode_scratch(static_cast<size_t>(M) * N, &a.ws)) != GLMQ_OK) return st;
   if (C::SMEM_BYTES > dev.smem_optin) return GLMQ_ERR_BAD_SHAPE;
-  st = allow_smem(prefill_kernel<C>, C::SMEM_BYTES);
-  if (st != GLMQ_OK) return st;
-  const int grid = a.tiles < dev.sms ? a.tiles : dev.sms;
+  if ((st = allow_smem(prefill_kernel<C>, C::SMEM_BYTES)) != GLMQ_OK) return st;
+  const int grid = a.units < dev.sms ? a.units : dev.sms;
   prefill_kernel<C><<<grid, kPrefillThreads, C::SMEM_BYTES, s>>>(tx, tw, a);
   cudaError_t e = cudaGetLastError();
-  return e == cudaSuccess ? GLMQ_OK : cuda_fail(e);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (a.parts > 1) {
+    const long long total = static_cast<long long>(M) * N;
+    const int blocks = static_cast<int>(std::min<long long>((total + 255) / 256, 4LL * dev.sms));
+    decode_finalize_kernel<<<blocks, 256, 0, s>>>(a.ws, a.scale, a.Y, M, N);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e);
+  }
+  return GLMQ_OK;
+}
+
+template <class C>
+glmq_status launch_skinny_cfg(const DeviceInfo& dev, const void* X, int M, const void* packed, const void* scale,
+                              int N, int K, void* Y, cudaStream_t s) {
+  CUtensorMap tx, tw;
+  glmq_status st = make_map_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, X, K, M, uint64_t(K) * 2, 64, C::kBN,
+                               CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st != GLMQ_OK) return st;
+  const uint64_t row_bytes = uint64_t(K) / C::KPB;
+  st = make_map_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, packed, row_bytes, N, row_bytes, C::WB, C::BM,
+                   CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st != GLMQ_OK) return st;
+  PrefillArgs a;
+  a.scale = static_cast<const __half*>(scale);
+  a.Y = static_cast<__half*>(Y);
+  a.ws = nullptr;
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.tiles_m = (M + C::kBN - 1) / C::kBN;
+  const long long tiles = static_cast<long long>((N + C::BM - 1) / C::BM) * a.tiles_m;
+  if (tiles > 0x7fffffffLL / 64) return GLMQ_ERR_BAD_SHAPE;
+  a.tiles = static_cast<int>(tiles);
+  const int num_st = (K + C::SK - 1) / C::SK;
+  const int parts = plan_parts(a.tiles, num_st, 2, dev.sms);
+  a.kbp = (num_st + parts - 1) / parts;          // stages per part
+  a.parts = (num_st + a.kbp - 1) / a.kbp;
+  a.units = a.tiles * a.parts;
+  if (a.parts > 1 && (st = decode_scratch(static_cast<size_t>(M) * N, &a.ws)) != GLMQ_OK) return st;
+  if (C::SMEM_BYTES > dev.smem_optin) return GLMQ_ERR_BAD_SHAPE;
+  if ((st = allow_smem(skinny_kernel<C>, C::SMEM_BYTES)) != GLMQ_OK) return st;
+  const int grid = a.units < dev.sms ? a.units : dev.sms;
+  skinny_kernel<C><<<grid, kSkinnyThreads, C::SMEM_BYTES, s>>>(tx, tw, a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (a.parts > 1) {
+    const long long total = static_cast<long long>(M) * N;
+    const int blocks = static_cast<int>(std::min<long long>((total + 255) / 256, 4LL * dev.sms));
+    decode_finalize_kernel<<<blocks, 256, 0, s>>>(a.ws, a.scale, a.Y, M, N);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e);
+  }
+  return GLMQ_OK;
 }
 
 template <int BITS>
 glmq_status launch_prefill(const DeviceInfo& dev, const void* X, int M, const void* packed, const void* scale, int N,
                            int K, void* Y, cudaStream_t s) {
-  if (M <= 32) return launch_prefill_cfg<PrefillCfg<BITS, 32>>(dev, X, M, packed, scale, N, K, Y, s);
-  if (M <= 64) return launch_prefill_cfg<PrefillCfg<BITS, 64>>(dev, X, M, packed, scale, N, K, Y, s);
+  // up to 64 tokens: the skinny kernel (wide weight stream, A operand in tensor memory)
+  if (M <= 16) return launch_skinny_cfg<SkinnyCfg<BITS, 16>>(dev, X, M, packed, scale, N, K, Y, s);
+  if (M <= 32) return launch_skinny_cfg<SkinnyCfg<BITS, 32>>(dev, X, M, packed, scale, N, K, Y, s);
+  if (M <= 64) return launch_skinny_cfg<SkinnyCfg<BITS, 64>>(dev, X, M, packed, scale, N, K, Y, s);
   if (M <= 128) return launch_prefill_cfg<PrefillCfg<BITS, 128>>(dev, X, M, packed, scale, N, K, Y, s);
   return launch_prefill_cfg<PrefillCfg<BITS, 256>>(dev, X, M, packed, scale, N, K, Y, s);
 }
@@ -400,7 +481,7 @@ glmq_status gemm_entry(Route route, const void* X, int64_t M, const void* packed
   const DeviceInfo* dev = nullptr;
   if ((st = current_device(&dev)) != GLMQ_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const bool decode = route == Route::kDecode || (route == Route::kAuto && M <= GLMQ_DECODE_MAX_M);
+  const bool decode = route == Route::kDecode || (route == Route::kAuto && M <= GLMQ_DECODE_AUTO_MAX_M);
   const int m = static_cast<int>(M), n = static_cast<int>(N), k = static_cast<int>(K);
   if (decode) {
     return bits == 4 ? launch_decode<4>(*dev, X, m, packed, scale, n, k, Y, s)

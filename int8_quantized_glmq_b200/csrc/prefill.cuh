@@ -14,17 +14,28 @@
 // epilogue. Warp roles (persistent CTAs, one per SM, static round-robin tiles,
 // the BN-token tiles of one weight tile consecutive so the packed rows are read
 // from HBM once and then hit in L2):
-//   warp 12      TMA producer: 2-D tensor copies of the X tile (BN x 64 fp16,
+//   warp 20      TMA producer: 2-D tensor copies of the X tile (BN x 64 fp16,
 //                128-byte swizzle) and of the packed weight tile (128 rows of
 //                32 / 64 bytes, 32- / 64-byte swizzle) into a kStages ring;
-//   warps 0..7   dequantizers: each thread turns 32 codes of one row into fp16
-//                and writes them into the A tile in the canonical K-major
-//                128-byte-swizzled layout, then fences the generic->async proxy;
-//   warp 13      MMA issuer: one thread issues 4 tcgen05.mma (K=16) per 64-wide
+//   warps 0..15  dequantizers, four independent groups of 128 threads (one weight
+//                row per thread); group g takes every fourth K block, so four K
+//                blocks are dequantized at once. A thread turns its row's 64 codes
+//                into fp16, writes them into the A tile in the canonical K-major
+//                128-byte-swizzled layout and fences the generic->async proxy;
+//   warp 21      MMA issuer: one thread issues 4 tcgen05.mma (K=16) per 64-wide
 //                K block into one of two TMEM accumulators and commits each stage
 //                back to the producer;
-//   warps 8..11  epilogue: tcgen05.ld of its 32 TMEM lanes, times s[n], fp16
+//   warps 16..19 epilogue: tcgen05.ld of its 32 TMEM lanes, times s[n], fp16
 //                stores; frees the accumulator for the next-but-one tile.
+// Work units are (tile, K part) pairs. Large problems use one part per tile; when
+// there are fewer tiles than SMs (small M), tiles are split over K parts so every
+// SM has work, each unit adds its fp32 partial tile into a scratch buffer with
+// red.global.add and a stream-ordered finalize kernel scales, rounds and stores Y.
+// For small token tiles (INT4, BN <= 32) the dequantizers write each 8-code group
+// in the order the register dequantization produces it, (0,4,1,5,2,6,3,7), and
+// permute the activation tile identically in place after it lands, which saves the
+// byte shuffles per packed word; the MMA's k order is immaterial when both
+// operands use the same one.
 // No TMA multicast is used anywhere.
 #pragma once
 
@@ -34,12 +45,14 @@
 
 namespace glmq {
 
-constexpr int kPrefillDequantWarps = 8;
-constexpr int kPrefillEpilogueWarp0 = 8;
-constexpr int kPrefillProducerWarp = 12;
-constexpr int kPrefillMmaWarp = 13;
-constexpr int kPrefillThreads = 14 * 32;
-constexpr int kPrefillStages = 4;
+constexpr int kPrefillDequantWarps = 16;
+constexpr int kPrefillDequantGroups = 4;     // groups of 4 warps; group g dequantizes K blocks g, g+4, ...
+constexpr int kPrefillEpilogueWarp0 = 16;
+constexpr int kPrefillProducerWarp = 20;
+constexpr int kPrefillMmaWarp = 21;
+constexpr int kPrefillThreads = 22 * 32;
+constexpr int kPrefillMaxStages = 8;
+constexpr int kPrefillSmemBudget = 232448 - 1024 /*alignment*/ - 512 /*barriers*/;
 
 template <int BITS, int BN>
 struct PrefillCfg {
@@ -52,10 +65,15 @@ struct PrefillCfg {
   static constexpr int WROW = BK * BITS / 8;            // packed bytes per row per K block (32 or 64)
   static constexpr int W_BYTES = BM * WROW;
   static constexpr int STAGE_BYTES = X_BYTES + A_BYTES + W_BYTES;
-  static constexpr int TMEM_COLS = (2 * BN <= 256) ? 256 : 512;
-  static constexpr int SMEM_BYTES = kPrefillStages * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+  static constexpr int kStages = (kPrefillSmemBudget / STAGE_BYTES) < kPrefillMaxStages
+                                     ? (kPrefillSmemBudget / STAGE_BYTES) : kPrefillMaxStages;
+  static constexpr int kPermX = (BITS == 4 && BN <= 32) ? 1 : 0;   // permuted k order (see above)
+  static constexpr int TMEM_COLS = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64 : (2 * BN <= 128) ? 128
+                                 : (2 * BN <= 256) ? 256 : 512;
+  static constexpr int SMEM_BYTES = kStages * STAGE_BYTES + 1024 /*align*/ + 512 /*barriers*/;
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N for M=128");
   static_assert(X_BYTES % 1024 == 0, "swizzle atoms stay 1024-byte aligned");
+  static_assert(kStages >= 2, "at least double buffering");
   // kind::f16, fp32 accumulator, fp16 A and B, both K-major, N = BN, M = 128
   static constexpr uint32_t IDESC = (1u << 4) | (uint32_t(BN >> 3) << 17) | (uint32_t(BM >> 4) << 24);
 };
@@ -63,11 +81,15 @@ struct PrefillCfg {
 struct PrefillArgs {
   const __half* scale;
   __half* Y;
+  float* ws;      // fp32 [M, N] scratch, zero on entry (used when parts > 1)
   int M;
   int N;
   int K;
   int tiles_m;
   int tiles;
+  int parts;      // K parts per tile
+  int kbp;        // K blocks per part
+  int units;      // tiles * parts
 };
 
 // ---------------------------------------------------------------- tcgen05 / TMA wrappers
@@ -110,6 +132,16 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+        "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
 __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
   asm volatile(
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
@@ -147,6 +179,25 @@ __device__ __forceinline__ uint4 dequant_int4_natural(uint32_t w) {
   return make_uint4(prmt(p0, p1, 0x5410u), prmt(p2, p3, 0x5410u), prmt(p0, p1, 0x7632u), prmt(p2, p3, 0x7632u));
 }
 
+// INT4 packed word -> 4 words of fp16 pairs (0,4), (1,5), (2,6), (3,7): the k order
+// (0,4,1,5,2,6,3,7) within the 8-code group, matched by a permuted activation tile.
+__device__ __forceinline__ uint4 dequant_int4_paired(uint32_t w) {
+  const __half2 kBias0 = __halves2half2(__ushort_as_half(0xE408), __ushort_as_half(0xE408));  // -1032
+  const __half2 kOne16 = __halves2half2(__ushort_as_half(0x2C00), __ushort_as_half(0x2C00));  // 1/16
+  const __half2 kBias1 = __halves2half2(__ushort_as_half(0xD480), __ushort_as_half(0xD480));  // -72
+  const uint32_t w8 = w >> 8;
+  uint32_t h0 = lop3_and_xor(w, 0x000F000Fu, 0x64086408u);
+  uint32_t h1 = lop3_and_xor(w, 0x00F000F0u, 0x64806480u);
+  uint32_t h2 = lop3_and_xor(w8, 0x000F000Fu, 0x64086408u);
+  uint32_t h3 = lop3_and_xor(w8, 0x00F000F0u, 0x64806480u);
+  __half2 r0 = __hadd2(*reinterpret_cast<__half2*>(&h0), kBias0);
+  __half2 r1 = __hfma2(*reinterpret_cast<__half2*>(&h1), kOne16, kBias1);
+  __half2 r2 = __hadd2(*reinterpret_cast<__half2*>(&h2), kBias0);
+  __half2 r3 = __hfma2(*reinterpret_cast<__half2*>(&h3), kOne16, kBias1);
+  return make_uint4(*reinterpret_cast<uint32_t*>(&r0), *reinterpret_cast<uint32_t*>(&r1),
+                    *reinterpret_cast<uint32_t*>(&r2), *reinterpret_cast<uint32_t*>(&r3));
+}
+
 __device__ __forceinline__ uint2 dequant_int8_natural(uint32_t w) {
   const __half2 kBias = __halves2half2(__ushort_as_half(0xE480), __ushort_as_half(0xE480));  // -1152
   const uint32_t x = w ^ 0x80808080u;
@@ -162,14 +213,15 @@ template <class C>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                    const PrefillArgs a) {
+  constexpr int S = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kPrefillStages * C::STAGE_BYTES);
-  uint64_t* full = bars;                           // TMA bytes landed          (count 1 + tx)
-  uint64_t* afull = bars + kPrefillStages;         // A tile dequantized        (count 8 warps)
-  uint64_t* empty = bars + 2 * kPrefillStages;     // MMAs of the stage done    (tcgen05.commit)
-  uint64_t* accfull = bars + 3 * kPrefillStages;   // accumulator ready         (tcgen05.commit), x2
-  uint64_t* accempty = accfull + 2;                // accumulator drained       (count 4 warps), x2
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::STAGE_BYTES);
+  uint64_t* full = bars;                  // TMA bytes landed          (count 1 + tx)
+  uint64_t* afull = bars + S;             // A tile dequantized        (count 4 warps)
+  uint64_t* empty = bars + 2 * S;         // MMAs of the stage done    (tcgen05.commit)
+  uint64_t* accfull = bars + 3 * S;       // accumulator ready         (tcgen05.commit), x2
+  uint64_t* accempty = accfull + 2;       // accumulator drained       (count 4 warps), x2
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accempty + 2);
 
   const int warp = threadIdx.x >> 5;
@@ -177,9 +229,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   const int num_kb = a.K / C::BK;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kPrefillStages; ++s) {
+    for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&afull[s], kPrefillDequantWarps);
+      mbar_init(&afull[s], kPrefillDequantWarps / kPrefillDequantGroups);
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -205,64 +257,83 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   if (warp == kPrefillProducerWarp) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      uint32_t armed[kPrefillStages] = {};
+      uint32_t armed[S] = {};
       int stage = 0;
       uint32_t phase = 0;
-      for (int tile = blockIdx.x; tile < a.tiles && ok; tile += G) {
-        const int nt = tile / a.tiles_m;
-        const int mt = tile - nt * a.tiles_m;
-        for (int kb = 0; kb < num_kb; ++kb) {
+      for (int u = blockIdx.x; u < a.units && ok; u += G) {
+        const int p = u / a.tiles;
+        const int t = u - p * a.tiles;
+        const int nt = t / a.tiles_m;
+        const int mt = t - nt * a.tiles_m;
+        const int kb1 = min(num_kb, (p + 1) * a.kbp);
+        for (int kb = p * a.kbp; kb < kb1; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1)) { ok = false; break; }
           uint8_t* st = smem + stage * C::STAGE_BYTES;
           mbar_arrive_expect_tx(&full[stage], C::X_BYTES + C::W_BYTES);
           armed[stage] = phase + 1;
           tma_load_2d(st, &tmap_x, kb * C::BK, mt * C::kBN, &full[stage]);
           tma_load_2d(st + C::X_BYTES + C::A_BYTES, &tmap_w, kb * C::WROW, nt * C::BM, &full[stage]);
-          if (++stage == kPrefillStages) { stage = 0; phase ^= 1; }
+          if (++stage == S) { stage = 0; phase ^= 1; }
         }
       }
       bool drained = true;
-      for (int s = 0; s < kPrefillStages; ++s)
+      for (int s = 0; s < S; ++s)
         if (armed[s] && !mbar_wait(&full[s], armed[s] - 1)) drained = false;
       if (!ok || !drained) report_error(kErrPrefillWait);
     }
   } else if (warp < kPrefillDequantWarps) {
     // ------------------------------------------------------------ dequantizers
     const int row = threadIdx.x & 127;   // tile row (TMEM lane / weight row)
-    const int half = threadIdx.x >> 7;   // which 32 codes of the 64-wide K block
+    const int grp = threadIdx.x >> 7;    // dequant group: K blocks with sequence number % 4 == grp
     int stage = 0;
     uint32_t phase = 0;
-    for (int tile = blockIdx.x; tile < a.tiles && ok; tile += G) {
-      for (int kb = 0; kb < num_kb; ++kb) {
-        if (!mbar_wait_warp(&full[stage], phase)) { ok = false; break; }
-        uint8_t* st = smem + stage * C::STAGE_BYTES;
-        const uint32_t a_tile = smem_u32(st + C::X_BYTES);
-        const uint32_t w_tile = smem_u32(st + C::X_BYTES + C::A_BYTES);
-        if constexpr (C::kBits == 4) {
-          // 32-byte rows, 32-byte swizzle: 16-byte unit u sits at u ^ ((row >> 2) & 1)
-          const uint4 v = lds_v4(w_tile + row * 32 + ((half ^ ((row >> 2) & 1)) << 4));
-          const uint32_t words[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const uint4 o = dequant_int4_natural(words[j]);
-            st_shared_v4(a_tile + sw128_off(row, 4 * half + j), o.x, o.y, o.z, o.w);
+    int seq = 0;                         // K-block sequence number across this CTA's units
+    for (int u = blockIdx.x; u < a.units && ok; u += G) {
+      const int p = u / a.tiles;
+      const int kb1 = min(num_kb, (p + 1) * a.kbp);
+      for (int kb = p * a.kbp; kb < kb1; ++kb, ++seq) {
+        if ((seq & (kPrefillDequantGroups - 1)) == grp) {
+          if (!mbar_wait_warp(&full[stage], phase)) { ok = false; break; }
+          uint8_t* st = smem + stage * C::STAGE_BYTES;
+          const uint32_t x_tile = smem_u32(st);
+          const uint32_t a_tile = smem_u32(st + C::X_BYTES);
+          const uint32_t w_tile = smem_u32(st + C::X_BYTES + C::A_BYTES);
+          if constexpr (C::kPermX) {
+            // permute each 16-byte unit of the activation tile to (0,4,1,5,2,6,3,7) in place
+            for (int i = row; i < C::kBN * 8; i += 128) {
+              const uint4 v = lds_v4(x_tile + 16 * i);
+              st_shared_v4(x_tile + 16 * i, prmt(v.x, v.z, 0x5410u), prmt(v.x, v.z, 0x7632u),
+                           prmt(v.y, v.w, 0x5410u), prmt(v.y, v.w, 0x7632u));
+            }
           }
-        } else {
-          // 64-byte rows, 64-byte swizzle: unit u sits at u ^ ((row >> 1) & 3)
+          if constexpr (C::kBits == 4) {
+            // 32-byte rows, 32-byte swizzle: 16-byte unit u sits at u ^ ((row >> 2) & 1)
 #pragma unroll
-          for (int q = 0; q < 2; ++q) {
-            const int u = 2 * half + q;
-            const uint4 v = lds_v4(w_tile + row * 64 + ((u ^ ((row >> 1) & 3)) << 4));
-            const uint2 lo0 = dequant_int8_natural(v.x), lo1 = dequant_int8_natural(v.y);
-            const uint2 hi0 = dequant_int8_natural(v.z), hi1 = dequant_int8_natural(v.w);
-            st_shared_v4(a_tile + sw128_off(row, 2 * u), lo0.x, lo0.y, lo1.x, lo1.y);
-            st_shared_v4(a_tile + sw128_off(row, 2 * u + 1), hi0.x, hi0.y, hi1.x, hi1.y);
+            for (int h = 0; h < 2; ++h) {
+              const uint4 v = lds_v4(w_tile + row * 32 + ((h ^ ((row >> 2) & 1)) << 4));
+              const uint32_t words[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                const uint4 o = C::kPermX ? dequant_int4_paired(words[j]) : dequant_int4_natural(words[j]);
+                st_shared_v4(a_tile + sw128_off(row, 4 * h + j), o.x, o.y, o.z, o.w);
+              }
+            }
+          } else {
+            // 64-byte rows, 64-byte swizzle: unit u sits at u ^ ((row >> 1) & 3)
+#pragma unroll
+            for (int uu = 0; uu < 4; ++uu) {
+              const uint4 v = lds_v4(w_tile + row * 64 + ((uu ^ ((row >> 1) & 3)) << 4));
+              const uint2 lo0 = dequant_int8_natural(v.x), lo1 = dequant_int8_natural(v.y);
+              const uint2 hi0 = dequant_int8_natural(v.z), hi1 = dequant_int8_natural(v.w);
+              st_shared_v4(a_tile + sw128_off(row, 2 * uu), lo0.x, lo0.y, lo1.x, lo1.y);
+              st_shared_v4(a_tile + sw128_off(row, 2 * uu + 1), hi0.x, hi0.y, hi1.x, hi1.y);
+            }
           }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&afull[stage]);
         }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&afull[stage]);
-        if (++stage == kPrefillStages) { stage = 0; phase ^= 1; }
+        if (++stage == S) { stage = 0; phase ^= 1; }
       }
     }
     if (!ok && lane == 0) report_error(kErrPrefillWait);
@@ -273,13 +344,16 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       uint32_t phase = 0;
       int it = 0;
       uint32_t acc_armed[2] = {};
-      for (int tile = blockIdx.x; tile < a.tiles && ok; tile += G, ++it) {
+      for (int u = blockIdx.x; u < a.units && ok; u += G, ++it) {
+        const int p = u / a.tiles;
+        const int kb0 = p * a.kbp;
+        const int kb1 = min(num_kb, kb0 + a.kbp);
         const int ab = it & 1;
         const uint32_t aphase = (it >> 1) & 1;
         if (!mbar_wait(&accempty[ab], aphase ^ 1)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + ab * C::kBN;
-        for (int kb = 0; kb < num_kb; ++kb) {
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&afull[stage], phase)) { ok = false; break; }
           tc_fence_after();
           uint8_t* st = smem + stage * C::STAGE_BYTES;
@@ -288,10 +362,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < C::BK / 16; ++kk) {
             umma_f16(d_tmem, umma_desc_sw128(a_addr + kk * 32), umma_desc_sw128(x_addr + kk * 32), C::IDESC,
-                     (kb | kk) != 0);
+                     (kb > kb0 || kk > 0) ? 1u : 0u);
           }
           umma_commit(&empty[stage]);
-          if (++stage == kPrefillStages) { stage = 0; phase ^= 1; }
+          if (++stage == S) { stage = 0; phase ^= 1; }
         }
         if (!ok) break;
         umma_commit(&accfull[ab]);
@@ -306,29 +380,39 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   } else {
     // ------------------------------------------------------------ epilogue warps 8..11
     const int quarter = warp & 3;   // TMEM lanes 32*quarter .. 32*quarter+31
+    const bool split = a.parts > 1;
     int it = 0;
-    for (int tile = blockIdx.x; tile < a.tiles && ok; tile += G, ++it) {
+    for (int u = blockIdx.x; u < a.units && ok; u += G, ++it) {
       const int ab = it & 1;
       const uint32_t aphase = (it >> 1) & 1;
       if (!mbar_wait_warp(&accfull[ab], aphase)) { ok = false; break; }
       tc_fence_after();
-      const int nt = tile / a.tiles_m;
-      const int mt = tile - nt * a.tiles_m;
+      const int t = u % a.tiles;
+      const int nt = t / a.tiles_m;
+      const int mt = t - nt * a.tiles_m;
       const int n = nt * C::BM + quarter * 32 + lane;
       const float s = (n < a.N) ? __half2float(a.scale[n]) : 0.0f;
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + ab * C::kBN;
+      constexpr int kChunk = (C::kBN < 32) ? C::kBN : 32;
 #pragma unroll 1
-      for (int cb = 0; cb < C::kBN / 32; ++cb) {
-        const int m0 = mt * C::kBN + cb * 32;
+      for (int cb = 0; cb < C::kBN / kChunk; ++cb) {
+        const int m0 = mt * C::kBN + cb * kChunk;
         if (m0 >= a.M) break;   // warp-uniform
         uint32_t v[32];
-        tmem_ld32(t_row + cb * 32, v);
+        if constexpr (kChunk == 16) tmem_ld16(t_row + cb * kChunk, v);
+        else tmem_ld32(t_row + cb * kChunk, v);
         if (n < a.N) {
-          __half* yp = a.Y + static_cast<long long>(m0) * a.N + n;
-          const int mend = min(32, a.M - m0);
+          const int mend = min(kChunk, a.M - m0);
+          if (split) {
+            float* wp = a.ws + static_cast<long long>(m0) * a.N + n;
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            if (j < mend) yp[static_cast<long long>(j) * a.N] = __float2half_rn(s * __uint_as_float(v[j]));
+            for (int j = 0; j < kChunk; ++j)
+              if (j < mend) atomicAdd(wp + static_cast<long long>(j) * a.N, __uint_as_float(v[j]));
+          } else {
+            __half* yp = a.Y + static_cast<long long>(m0) * a.N + n;
+#pragma unroll
+            for (int j = 0; j < kChunk; ++j)
+              if (j < mend) yp[static_cast<long long>(j) * a.N] = __float2half_rn(s * __uint_as_float(v[j]));
           }
         }
       }

@@ -1,0 +1,356 @@
+// Tensor-core W4A16 / W8A16 GEMM for a skinny activation matrix (M <= 64 tokens):
+//
+//   Y[m,n] = fp16( s[n] * sum_k X[m,k] q[n,k] )
+//
+// GLM-130B paper card (wikillm.com), "Method": linear_forward with weight =
+// quant * scale[:, None] and FP16 activations; paperlayer summary, "INT4
+// Quantization for RTX 3090s/2080s": weights are converted to FP16 at run time.
+//
+// With few tokens the packed weights are the working set, so the kernel is built
+// around a wide weight stream and cheap dequantization:
+//  * Stages hold one TMA box of 128 weight rows x 128 packed bytes (256 k for INT4,
+//    128 k for INT8; 128-byte swizzle) plus the matching activation tiles
+//    (BN tokens x 64 k each, 128-byte swizzle). Wide box rows matter: the TMA
+//    path serves a roughly fixed number of box rows per microsecond, so 128-byte
+//    rows stream several times faster than the 32-byte rows of a 64-wide K block.
+//  * The dequantized weights never touch shared memory: they are the MMA's A
+//    operand in tensor memory. Four dequantizer groups of 128 threads (thread =
+//    weight row = TMEM lane) take the 64-wide K blocks of the stream round-robin
+//    (group g: blocks g, g+4, ...), turn 64 codes into fp16 in registers and write
+//    them with one tcgen05.st into a ring of A slots.
+//  * One thread issues tcgen05.mma (kind::f16, A from TMEM, B from shared memory,
+//    fp32 accumulator in TMEM); the epilogue warps read the accumulator with
+//    tcgen05.ld, multiply by s[n] and store fp16 (or add into the split-K scratch).
+//  * INT4 codes are dequantized in the order (0,4,1,5,2,6,3,7) within each group
+//    of 8, which costs no byte shuffle; the activation tile is permuted the same
+//    way in place after it lands (the MMA's k order is immaterial when both
+//    operands share it).
+//  * Work units are (128-row tile, K part) pairs exactly as in the prefill kernel,
+//    with the same split-K scratch and finalize kernel.
+// No TMA multicast is used anywhere.
+#pragma once
+
+#include <cuda.h>
+
+#include "glmq_ptx.cuh"
+#include "prefill.cuh"
+
+namespace glmq {
+
+constexpr int kSkinnyDequantWarps = 16;    // 4 groups of 4 warps
+constexpr int kSkinnyGroups = 4;
+constexpr int kSkinnyEpilogueWarp0 = 16;   // warps 16..19
+constexpr int kSkinnyProducerWarp = 20;
+constexpr int kSkinnyMmaWarp = 21;
+constexpr int kSkinnyThreads = 22 * 32;
+constexpr int kSkinnyASlots = 8;           // A operand slots in TMEM (one 64-wide K block each)
+
+template <int BITS, int BN>
+struct SkinnyCfg {
+  static constexpr int kBits = BITS;
+  static constexpr int kBN = BN;
+  static constexpr int BM = 128;
+  static constexpr int WB = 128;                          // packed bytes per row per stage
+  static constexpr int KPB = (BITS == 4) ? 2 : 1;
+  static constexpr int SK = WB * KPB;                     // k per stage
+  static constexpr int KB = SK / 64;                      // 64-wide K blocks per stage (4 or 2)
+  static constexpr int W_BYTES = BM * WB;                 // 16 KB
+  static constexpr int XT_BYTES = BN * 128;               // one activation tile (BN x 64 fp16)
+  static constexpr int STAGE_BYTES = W_BYTES + KB * XT_BYTES;
+  static constexpr int kStages = (kPrefillSmemBudget / STAGE_BYTES) < kPrefillMaxStages
+                                     ? (kPrefillSmemBudget / STAGE_BYTES) : kPrefillMaxStages;
+  static constexpr int kPermX = (BITS == 4) ? 1 : 0;
+  static constexpr int ACC_COLS = 2 * BN;                 // two accumulators of BN fp32 columns
+  static constexpr int TMEM_COLS = 512;
+  static constexpr int SMEM_BYTES = kStages * STAGE_BYTES + 1024 /*align*/ + 512 /*barriers*/;
+  static_assert(BN == 16 || BN == 32 || BN == 64, "skinny token tiles");
+  static_assert(XT_BYTES % 1024 == 0, "swizzle atoms stay 1024-byte aligned");
+  static_assert(kStages >= 3, "pipeline depth");
+  static_assert(ACC_COLS + kSkinnyASlots * 32 <= TMEM_COLS, "tensor memory budget");
+  // kind::f16, fp32 accumulator, fp16 A (tensor memory) and B (shared memory), K-major, N = BN, M = 128
+  static constexpr uint32_t IDESC = (1u << 4) | (uint32_t(BN >> 3) << 17) | (uint32_t(BM >> 4) << 24);
+};
+
+__device__ __forceinline__ void umma_f16_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                                uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
+      "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]),
+      "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]),
+      "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+      : "memory");
+}
+
+// Valid 64-wide K blocks of the stage that starts at k0.
+__device__ __forceinline__ int skinny_stage_kblocks(int k0, int K, int KB) { return min(KB, (K - k0) >> 6); }
+
+template <class C>
+__global__ void __launch_bounds__(kSkinnyThreads, 1)
+    skinny_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
+                  const PrefillArgs a) {
+  constexpr int S = C::kStages;
+  constexpr int NA = kSkinnyASlots;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::STAGE_BYTES);
+  uint64_t* full = bars;                  // stage bytes landed            (count 1 + tx)
+  uint64_t* empty = bars + S;             // stage's MMAs done             (tcgen05.commit)
+  uint64_t* afull = bars + 2 * S;         // A slot written                (count 4 warps)
+  uint64_t* aempty = afull + NA;          // A slot's MMAs done            (tcgen05.commit)
+  uint64_t* accfull = aempty + NA;        // accumulator ready             (tcgen05.commit), x2
+  uint64_t* accempty = accfull + 2;       // accumulator drained           (count 4 warps), x2
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accempty + 2);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int K = a.K;
+  const int num_st = (K + C::SK - 1) / C::SK;     // stages along K
+  const int G = gridDim.x;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int i = 0; i < NA; ++i) {
+      mbar_init(&afull[i], kSkinnyDequantWarps / kSkinnyGroups);
+      mbar_init(&aempty[i], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&accfull[b], 1);
+      mbar_init(&accempty[b], 4);
+    }
+    fence_barrier_init();
+  }
+  if (warp == kSkinnyMmaWarp) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(C::TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  bool ok = true;
+
+  if (warp == kSkinnyProducerWarp) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      uint32_t armed[S] = {};
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int u = blockIdx.x; u < a.units && ok; u += G) {
+        const int p = u / a.tiles;
+        const int t = u - p * a.tiles;
+        const int nt = t / a.tiles_m;
+        const int mt = t - nt * a.tiles_m;
+        const int st1 = min(num_st, (p + 1) * a.kbp);
+        for (int ks = p * a.kbp; ks < st1; ++ks) {
+          if (!mbar_wait(&empty[stage], phase ^ 1)) { ok = false; break; }
+          const int k0 = ks * C::SK;
+          const int nkb = skinny_stage_kblocks(k0, K, C::KB);
+          uint8_t* st = smem + stage * C::STAGE_BYTES;
+          mbar_arrive_expect_tx(&full[stage], C::W_BYTES + nkb * C::XT_BYTES);
+          armed[stage] = phase + 1;
+          tma_load_2d(st, &tmap_w, k0 / C::KPB, nt * C::BM, &full[stage]);
+          for (int j = 0; j < nkb; ++j)
+            tma_load_2d(st + C::W_BYTES + j * C::XT_BYTES, &tmap_x, k0 + 64 * j, mt * C::kBN, &full[stage]);
+          if (++stage == S) { stage = 0; phase ^= 1; }
+        }
+      }
+      bool drained = true;
+      for (int s = 0; s < S; ++s)
+        if (armed[s] && !mbar_wait(&full[s], armed[s] - 1)) drained = false;
+      if (!ok || !drained) report_error(kErrPrefillWait);
+    }
+  } else if (warp < kSkinnyDequantWarps) {
+    // ------------------------------------------------------------ dequantizer groups
+    const int grp = warp >> 2;                      // K blocks with sequence number % 4 == grp
+    const int row = ((warp & 3) << 5) + lane;       // weight row of the tile = TMEM lane
+    const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    int stage = 0;
+    uint32_t phase = 0;
+    int kseq = 0;
+    for (int u = blockIdx.x; u < a.units && ok; u += G) {
+      const int p = u / a.tiles;
+      const int st1 = min(num_st, (p + 1) * a.kbp);
+      for (int ks = p * a.kbp; ks < st1 && ok; ++ks) {
+        const int nkb = skinny_stage_kblocks(ks * C::SK, K, C::KB);
+        bool waited = false;
+        for (int j = 0; j < nkb; ++j, ++kseq) {
+          if ((kseq & (kSkinnyGroups - 1)) != grp) continue;
+          if (!waited) {
+            if (!mbar_wait_warp(&full[stage], phase)) { ok = false; break; }
+            waited = true;
+          }
+          const int slot = kseq % NA;
+          if (!mbar_wait_warp(&aempty[slot], ((kseq / NA) & 1) ^ 1)) { ok = false; break; }
+          tc_fence_after();
+          uint8_t* st = smem + stage * C::STAGE_BYTES;
+          const uint32_t w_tile = smem_u32(st);
+          if constexpr (C::kPermX) {
+            // permute the activation tile of this K block to (0,4,1,5,2,6,3,7) per 8 values, in place
+            const uint32_t x_tile = smem_u32(st + C::W_BYTES + j * C::XT_BYTES);
+            for (int i = row; i < C::kBN * 8; i += 128) {
+              const uint4 v = lds_v4(x_tile + 16 * i);
+              st_shared_v4(x_tile + 16 * i, prmt(v.x, v.z, 0x5410u), prmt(v.x, v.z, 0x7632u),
+                           prmt(v.y, v.w, 0x5410u), prmt(v.y, v.w, 0x7632u));
+            }
+            fence_proxy_async_smem();
+          }
+          uint32_t h[32];
+          if constexpr (C::kBits == 4) {
+            // bytes [32j, 32j+32) of this row: 16-byte units 2j and 2j+1, 128-byte swizzle
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+              const uint32_t unit = static_cast<uint32_t>((2 * j + q) ^ (row & 7));
+              const uint4 v = lds_v4(w_tile + row * 128 + (unit << 4));
+              const uint32_t words[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+              for (int wv = 0; wv < 4; ++wv) {
+                const uint4 o = dequant_int4_paired(words[wv]);
+                h[16 * q + 4 * wv + 0] = o.x;
+                h[16 * q + 4 * wv + 1] = o.y;
+                h[16 * q + 4 * wv + 2] = o.z;
+                h[16 * q + 4 * wv + 3] = o.w;
+              }
+            }
+          } else {
+            // bytes [64j, 64j+64) of this row: units 4j .. 4j+3
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const uint32_t unit = static_cast<uint32_t>((4 * j + q) ^ (row & 7));
+              const uint4 v = lds_v4(w_tile + row * 128 + (unit << 4));
+              const uint2 d0 = dequant_int8_natural(v.x), d1 = dequant_int8_natural(v.y);
+              const uint2 d2 = dequant_int8_natural(v.z), d3 = dequant_int8_natural(v.w);
+              h[8 * q + 0] = d0.x; h[8 * q + 1] = d0.y; h[8 * q + 2] = d1.x; h[8 * q + 3] = d1.y;
+              h[8 * q + 4] = d2.x; h[8 * q + 5] = d2.y; h[8 * q + 6] = d3.x; h[8 * q + 7] = d3.y;
+            }
+          }
+          tmem_st32(tmem_base + lane_addr + C::ACC_COLS + slot * 32, h);
+          asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&afull[slot]);
+        }
+        if (++stage == S) { stage = 0; phase ^= 1; }
+      }
+    }
+    if (!ok && lane == 0) report_error(kErrPrefillWait);
+  } else if (warp == kSkinnyMmaWarp) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int kseq = 0;
+      int it = 0;
+      uint32_t acc_armed[2] = {};
+      for (int u = blockIdx.x; u < a.units && ok; u += G, ++it) {
+        const int p = u / a.tiles;
+        const int st0 = p * a.kbp;
+        const int st1 = min(num_st, st0 + a.kbp);
+        const int ab = it & 1;
+        const uint32_t aphase = (it >> 1) & 1;
+        if (!mbar_wait(&accempty[ab], aphase ^ 1)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + ab * C::kBN;
+        bool first = true;
+        for (int ks = st0; ks < st1 && ok; ++ks) {
+          const int nkb = skinny_stage_kblocks(ks * C::SK, K, C::KB);
+          uint8_t* st = smem + stage * C::STAGE_BYTES;
+          for (int j = 0; j < nkb; ++j, ++kseq) {
+            const int slot = kseq % NA;
+            if (!mbar_wait(&afull[slot], (kseq / NA) & 1)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t x_addr = smem_u32(st + C::W_BYTES + j * C::XT_BYTES);
+            const uint32_t a_tmem = tmem_base + C::ACC_COLS + slot * 32;
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              umma_f16_tmem_a(d_tmem, a_tmem + kk * 8, umma_desc_sw128(x_addr + kk * 32), C::IDESC,
+                              first ? 0u : 1u);
+              first = false;
+            }
+            umma_commit(&aempty[slot]);
+          }
+          if (!ok) break;
+          umma_commit(&empty[stage]);
+          if (++stage == S) { stage = 0; phase ^= 1; }
+        }
+        if (!ok) break;
+        umma_commit(&accfull[ab]);
+        acc_armed[ab] = aphase + 1;
+      }
+      bool drained = true;
+      for (int b = 0; b < 2; ++b)
+        if (acc_armed[b] && !mbar_wait(&accfull[b], acc_armed[b] - 1)) drained = false;
+      if (!ok || !drained) report_error(kErrPrefillWait);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue warps 16..19
+    const int quarter = warp & 3;
+    const bool split = a.parts > 1;
+    int it = 0;
+    for (int u = blockIdx.x; u < a.units && ok; u += G, ++it) {
+      const int ab = it & 1;
+      const uint32_t aphase = (it >> 1) & 1;
+      if (!mbar_wait_warp(&accfull[ab], aphase)) { ok = false; break; }
+      tc_fence_after();
+      const int t = u % a.tiles;
+      const int nt = t / a.tiles_m;
+      const int mt = t - nt * a.tiles_m;
+      const int n = nt * C::BM + quarter * 32 + lane;
+      const float s = (n < a.N) ? __half2float(a.scale[n]) : 0.0f;
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + ab * C::kBN;
+      constexpr int kChunk = (C::kBN < 32) ? C::kBN : 32;
+#pragma unroll 1
+      for (int cb = 0; cb < C::kBN / kChunk; ++cb) {
+        const int m0 = mt * C::kBN + cb * kChunk;
+        if (m0 >= a.M) break;   // warp-uniform
+        uint32_t v[32];
+        if constexpr (kChunk == 16) tmem_ld16(t_row + cb * kChunk, v);
+        else tmem_ld32(t_row + cb * kChunk, v);
+        if (n < a.N) {
+          const int mend = min(kChunk, a.M - m0);
+          if (split) {
+            float* wp = a.ws + static_cast<long long>(m0) * a.N + n;
+#pragma unroll
+            for (int jj = 0; jj < kChunk; ++jj)
+              if (jj < mend) atomicAdd(wp + static_cast<long long>(jj) * a.N, __uint_as_float(v[jj]));
+          } else {
+            __half* yp = a.Y + static_cast<long long>(m0) * a.N + n;
+#pragma unroll
+            for (int jj = 0; jj < kChunk; ++jj)
+              if (jj < mend) yp[static_cast<long long>(jj) * a.N] = __float2half_rn(s * __uint_as_float(v[jj]));
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&accempty[ab]);
+    }
+    if (!ok && lane == 0) report_error(kErrPrefillWait);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kSkinnyMmaWarp) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(C::TMEM_COLS)
+                 : "memory");
+  }
+}
+
+}  // namespace glmq

@@ -35,6 +35,7 @@ def test_library_exports_every_declared_symbol():
 def test_header_constants_match_binding():
     text = open(HEADER).read()
     assert int(re.search(r"#define GLMQ_DECODE_MAX_M (\d+)", text).group(1)) == B.DECODE_MAX_M
+    assert int(re.search(r"#define GLMQ_DECODE_AUTO_MAX_M (\d+)", text).group(1)) == B.DECODE_AUTO_MAX_M
     assert int(re.search(r"#define GLMQ_MAX_K (\d+)", text).group(1)) == B.MAX_K
     for name, val in [("GLMQ_OK", B.OK), ("GLMQ_ERR_BAD_SHAPE", B.ERR_BAD_SHAPE),
                       ("GLMQ_ERR_MISALIGNED", B.ERR_MISALIGNED), ("GLMQ_ERR_DEVICE", B.ERR_DEVICE)]:

@@ -524,14 +524,15 @@ def run_one(args, world, rank, local):
         del W
         X = torch.randn((args.m, K), generator=g, device="cuda", dtype=torch.float32).half()
         Y = torch.empty((args.m, N), dtype=torch.float16, device="cuda")
-        fn = lambda: glmq.gemm(X, packed, scale, args.bits, out=Y)  # noqa: E731
+        fn = lambda: glmq.gemm(X, packed, scale, args.bits, out=Y, route=args.route)  # noqa: E731
         work = {"bytes": packed.numel() + scale.numel() * 2 + X.numel() * 2 + Y.numel() * 2,
                 "flops": 2.0 * args.m * N * K}
     else:
         fn = lambda: glmq.quantize(W, args.bits, out=(packed, scale))  # noqa: E731
         work = {"bytes": W.numel() * 2 + packed.numel() + scale.numel() * 2, "flops": 0.0}
     t = time_launches(torch, fn, args.steps, warmup=args.warmup)
-    return {"workload": "one", "op": args.op, "proj": args.proj, "N": N, "K": K, "M": args.m, "bits": args.bits,
+    return {"workload": "one", "op": args.op, "route": args.route, "proj": args.proj, "N": N, "K": K, "M": args.m,
+            "bits": args.bits,
             "us": round(t * 1e6, 2), "gbs": round(work["bytes"] / t / 1e9, 1),
             "tflops": round(work["flops"] / t / 1e12, 1), "algorithmic_bytes": work["bytes"]}
 
@@ -548,6 +549,8 @@ def main():
     ap.add_argument("--op", default="gemm", choices=["gemm", "quantize"])
     ap.add_argument("--m", type=int, default=1)
     ap.add_argument("--bits", type=int, default=4, choices=[4, 8])
+    ap.add_argument("--route", default="auto", choices=["auto", "decode", "prefill"],
+                    help="glmq_gemm entry point for --workload one")
     ap.add_argument("--layers", type=int, default=70)
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

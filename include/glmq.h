@@ -63,8 +63,9 @@ extern "C" {
 /* Largest M the decode (register-dequant GEMV) kernel accepts (glmq_gemm_decode). */
 #define GLMQ_DECODE_MAX_M 16
 /* glmq_gemm sends M <= GLMQ_DECODE_AUTO_MAX_M to the decode kernel and larger M to the
- * tensor-core kernel, which splits tiles over K when there are fewer tiles than SMs. */
-#define GLMQ_DECODE_AUTO_MAX_M 8
+ * tcgen05 tensor-core kernels (a skinny variant up to 64 tokens, the prefill kernel
+ * above), which split tiles over K when there are fewer tiles than SMs. */
+#define GLMQ_DECODE_AUTO_MAX_M 16
 
 typedef enum glmq_status {
   GLMQ_OK = 0,

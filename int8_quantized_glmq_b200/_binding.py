@@ -25,7 +25,7 @@ ERR_DEVICE = 6
 ERR_UNSUPPORTED_DEVICE = 7
 
 DECODE_MAX_M = 16
-DECODE_AUTO_MAX_M = 8
+DECODE_AUTO_MAX_M = 16
 MAX_K = 65536
 NOALLOC_SCRATCH_FLOATS = 1 << 20
 

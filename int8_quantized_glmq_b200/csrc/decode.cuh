@@ -9,30 +9,32 @@
 //
 // With M <= 16 the packed weights are the whole working set: the kernel is an
 // HBM stream. Design:
-//  * Work units are (row tile of 32 rows, K part) pairs, enumerated K-part major;
+//  * Work units are (row tile of 256 rows, K part) pairs, enumerated K-part major;
 //    each persistent CTA takes one contiguous range of units, so the load is
 //    balanced to within one unit and a CTA changes K part (and so restages its
-//    activation slice) at most a few times.
-//  * Warp 16 is the producer: one lane issues, per stage, eight 2-D TMA tile
-//    loads of 32 rows x 128 bytes (one per K segment, 128-byte swizzle) into a
-//    kDecodeStages-deep ring, with an L2 evict-first hint. Rows past N and bytes
-//    past K are zero-filled by the TMA unit.
-//  * Warps 0..15 are consumers: warp w owns K segment (w % 8) of every stage for
-//    the 16-row group (w / 8). Codes are dequantized in registers with exponent-
-//    bias tricks (a code c becomes the fp16 number 1024 + (c ^ 8) by OR-ing it
-//    into the mantissa, then one subtraction) and feed mma.sync m16n8k16 as the A
-//    operand straight from registers, X being the B operand. The K order inside
-//    each MMA is permuted identically on both operands so that each 32-bit packed
-//    word feeds two MMAs without a byte shuffle; the permutation is applied once,
-//    when the consumers stage the activation slice into shared memory in exactly
-//    the order the B fragments are read.
-//  * A unit's partial sums are added across warps in shared memory
-//    (red.shared.add). A tile covered by one K part is scaled, rounded and stored
-//    directly. When the activation slice does not fit in shared memory at once,
-//    tiles are split over several K parts: each unit adds its partial sums into
-//    an fp32 scratch buffer with fire-and-forget red.global.add, and a small
-//    stream-ordered finalize kernel (decode_finalize_kernel) scales, rounds and
-//    stores Y and returns the scratch to zero for the next call.
+//    activation slice) at most a few times. The number of K parts is the smallest
+//    that both fits the activation slice in shared memory and spreads the units
+//    evenly over the SMs.
+//  * Warp 16 is the producer: one lane issues, per stage, one 2-D TMA tile load of
+//    256 rows x 128 bytes (128-byte swizzle, 32 KB) into a kDecodeStages-deep
+//    ring, with an L2 evict-first hint. Rows past N and bytes past K are
+//    zero-filled by the TMA unit.
+//  * Warps 0..15 are consumers: warp w owns rows 16w .. 16w+15 of the tile and
+//    reads the whole stage's K segment for them. Codes are dequantized in
+//    registers with exponent-bias tricks (a code c becomes the fp16 number
+//    1024 + (c ^ 8) by OR-ing it into the mantissa) and feed mma.sync m16n8k16
+//    as the A operand straight from registers, X being the B operand. The K order
+//    inside each MMA is permuted identically on both operands so that each 32-bit
+//    packed word feeds two MMAs without a byte shuffle; the permutation is applied
+//    once, when the consumers stage the activation slice into shared memory in
+//    exactly the order the B fragments are read.
+//  * A warp's sums stay in registers for the whole unit, so a unit ends without
+//    any cross-warp reduction or barrier: the warp scales, rounds and stores its
+//    own 16 rows. When a tile is split over several K parts each warp instead adds
+//    its partial sums into an fp32 scratch buffer with fire-and-forget
+//    red.global.add, and a small stream-ordered finalize kernel
+//    (decode_finalize_kernel) scales, rounds and stores Y and returns the scratch
+//    to zero for the next call.
 #pragma once
 
 #include <cuda.h>
@@ -44,14 +46,11 @@ namespace glmq {
 constexpr int kDecodeConsumerWarps = 16;
 constexpr int kDecodeThreads = (kDecodeConsumerWarps + 1) * 32;
 constexpr int kDecodeStages = 4;
-constexpr int kDecodeRows = 32;          // rows per tile
-constexpr int kDecodeSegB = 128;         // packed bytes per row per segment (one TMA box width)
-constexpr int kDecodeSegs = 8;           // segments per stage
-constexpr int kDecodeBoxBytes = kDecodeRows * kDecodeSegB;            // 4 KB per TMA box
-constexpr int kDecodeStageBytes = kDecodeSegs * kDecodeBoxBytes;      // 32 KB per stage
-constexpr int kDecodeAccBytes = kDecodeRows * 16 * 4;
-// ring + unit accumulator + barriers; the activation slice follows
-constexpr int kDecodeFixedSmem = kDecodeStages * kDecodeStageBytes + kDecodeAccBytes + 256;
+constexpr int kDecodeRows = 16 * kDecodeConsumerWarps;                // rows per tile (256)
+constexpr int kDecodeSegB = 128;         // packed bytes per row per stage (one TMA box width)
+constexpr int kDecodeStageBytes = kDecodeRows * kDecodeSegB;          // 32 KB: one TMA box per stage
+// ring + barriers; the activation slice follows
+constexpr int kDecodeFixedSmem = kDecodeStages * kDecodeStageBytes + 256;
 
 template <int BITS, int MP>
 struct DecodeCfg {
@@ -60,7 +59,7 @@ struct DecodeCfg {
   static constexpr int kNB = (MP + 7) / 8;          // n8 token blocks of the MMA
   static constexpr int KPB = (BITS == 4) ? 2 : 1;   // codes per byte
   static constexpr int SEGK = kDecodeSegB * KPB;    // k per segment
-  static constexpr int SK = kDecodeSegs * SEGK;     // k per stage
+  static constexpr int SK = SEGK;                   // k per stage (one segment)
   static constexpr int TB = kDecodeSegB / 4;        // packed bytes per thread per row per segment (32)
   static constexpr int TK = TB * KPB;               // k per thread per segment
   static constexpr int TW = TB / 4;                 // 32-bit words per thread per row per segment (8)
@@ -224,8 +223,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* wring = smem;
-  float* acc_s = reinterpret_cast<float*>(smem + kDecodeStages * kDecodeStageBytes);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kDecodeStages * kDecodeStageBytes + kDecodeAccBytes);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kDecodeStages * kDecodeStageBytes);
   uint64_t* empty = full + kDecodeStages;
   uint8_t* xbuf = smem + kDecodeFixedSmem;
   // INT4 only: per (segment, token) bias of the biased dequantization, after the activation slice
@@ -245,14 +243,12 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     }
     fence_barrier_init();
   }
-  for (int i = threadIdx.x; i < kDecodeRows * 16; i += kDecodeThreads) acc_s[i] = 0.0f;
   __syncthreads();
 
   if (warp == kDecodeConsumerWarps) {
     // ------------------------------------------------------------ producer warp
     if (lane == 0) {
       const uint64_t pol = policy_evict_first();
-      const int row_bytes = K / C::KPB;
       uint32_t armed[kDecodeStages] = {};
       int stage = 0;
       uint32_t phase = 0;
@@ -266,13 +262,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         for (int ks = 0; ks < nst; ++ks) {
           if (!mbar_wait(&empty[stage], phase ^ 1)) { ok = false; break; }
           const int xb0 = (pk0 + ks * C::SK) / C::KPB;            // first packed byte of the stage
-          const int segs = min(kDecodeSegs, (row_bytes - xb0 + kDecodeSegB - 1) / kDecodeSegB);
-          mbar_arrive_expect_tx(&full[stage], static_cast<uint32_t>(segs * kDecodeBoxBytes));
+          mbar_arrive_expect_tx(&full[stage], static_cast<uint32_t>(kDecodeStageBytes));
           armed[stage] = phase + 1;
-          uint8_t* dst = wring + stage * kDecodeStageBytes;
-          for (int sg = 0; sg < segs; ++sg)
-            tma_load_2d_hint(dst + sg * kDecodeBoxBytes, &tmap_w, xb0 + sg * kDecodeSegB, t * kDecodeRows,
-                             &full[stage], pol);
+          tma_load_2d_hint(wring + stage * kDecodeStageBytes, &tmap_w, xb0, t * kDecodeRows, &full[stage], pol);
           if (++stage == kDecodeStages) { stage = 0; phase ^= 1; }
         }
       }
@@ -286,22 +278,20 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   }
 
   // -------------------------------------------------------------- consumer warps
-  const int seg = warp & (kDecodeSegs - 1);
-  const int grp = warp >> 3;                 // 16-row group
   const int r = lane >> 2;
   const int c = lane & 3;
   const int ct = threadIdx.x;                // 0 .. 511
   constexpr int kCT = kDecodeConsumerWarps * 32;
   const uint32_t wring_u32 = smem_u32(wring);
   const uint32_t xbuf_u32 = smem_u32(xbuf);
-  const uint32_t acc_u32 = smem_u32(acc_s);
-  const int ra = 16 * grp + r;               // this lane's rows: ra and ra + 8 (same ra & 7)
+  const int ra = 16 * warp + r;              // this lane's rows: ra and ra + 8 (same ra & 7)
   // per-lane byte offsets: packed row ra, 16-byte units 2c and 2c+1 under the 128-byte swizzle
   const uint32_t wlane = static_cast<uint32_t>(ra * kDecodeSegB + (((2 * c) ^ (ra & 7)) << 4)) |
                          (static_cast<uint32_t>(ra * kDecodeSegB + (((2 * c + 1) ^ (ra & 7)) << 4)) << 16);
   // activation units of this lane's tokens (clamped to a real token; results past M are discarded)
   const uint32_t xlane0 = 16u * x_unit<C>(0, 0, min(r, M - 1), c);
   const uint32_t xlane1 = 16u * x_unit<C>(0, 0, min(r + 8, M - 1), c);
+  const bool split = a.parts > 1;
   int stage = 0;
   uint32_t phase = 0;
   int cur_part = -1;
@@ -383,16 +373,15 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     const int nst = (plen + C::SK - 1) / C::SK;
     for (int ks = 0; ks < nst; ++ks) {
       if (ok && !mbar_wait_warp(&full[stage], phase)) ok = false;
-      const int kseg = ks * C::SK + seg * C::SEGK;               // part-relative k of this warp's segment
-      if (ok && pk0 + kseg < K) {
-        const int sg = ks * kDecodeSegs + seg;                    // segment index within the part
-        const uint32_t box = wring_u32 + stage * kDecodeStageBytes + seg * kDecodeBoxBytes;
-        const uint32_t xseg = xbuf_u32 + 16u * x_unit<C>(sg, 0, 0, 0);
-        const float* bias_seg = bias_s + sg * 16;
-        if (pk0 + kseg + C::SEGK <= K) {
+      if (ok) {
+        const uint32_t box = wring_u32 + stage * kDecodeStageBytes;
+        const uint32_t xseg = xbuf_u32 + 16u * x_unit<C>(ks, 0, 0, 0);
+        const float* bias_seg = bias_s + ks * 16;
+        const int kseg = pk0 + ks * C::SK;                        // absolute k of this stage
+        if (kseg + C::SK <= K) {
           decode_segment<C, false>(box, xseg, wlane, xlane0, xlane1, true, bias_seg, c, acc);
         } else {
-          const bool valid = pk0 + kseg + c * C::TK < K;
+          const bool valid = kseg + c * C::TK < K;
           decode_segment<C, true>(box, xseg, wlane, xlane0, xlane1, valid, bias_seg, c, acc);
         }
       }
@@ -401,39 +390,26 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       if (++stage == kDecodeStages) { stage = 0; phase ^= 1; }
     }
 
-    // ---- unit epilogue: add the warps' partials, then store or accumulate across parts
+    // ---- unit epilogue, per warp: rows ra and ra + 8, tokens 8 nb + 2 c (+1)
+    const int row_a = t * kDecodeRows + ra;
+    const int row_b = row_a + 8;
+    const float sa = (!split && row_a < N) ? __half2float(a.scale[row_a]) : 0.0f;
+    const float sb = (!split && row_b < N) ? __half2float(a.scale[row_b]) : 0.0f;
 #pragma unroll
     for (int nb = 0; nb < C::kNB; ++nb) {
 #pragma unroll
       for (int i = 0; i < 4; ++i) acc[0][nb][i] += acc[1][nb][i];
-      const int t0 = 8 * nb + 2 * c;
-      if (t0 < M) {
-        red_shared_add_f32(acc_u32 + (ra * 16 + t0) * 4, acc[0][nb][0]);
-        red_shared_add_f32(acc_u32 + ((ra + 8) * 16 + t0) * 4, acc[0][nb][2]);
-      }
-      if (t0 + 1 < M) {
-        red_shared_add_f32(acc_u32 + (ra * 16 + t0 + 1) * 4, acc[0][nb][1]);
-        red_shared_add_f32(acc_u32 + ((ra + 8) * 16 + t0 + 1) * 4, acc[0][nb][3]);
-      }
-    }
-    named_barrier_sync(1, kCT);
-    const int row0 = t * kDecodeRows;
-    const bool split = a.parts > 1;
-    for (int i = ct; i < M * kDecodeRows; i += kCT) {
-      const int m = i / kDecodeRows;
-      const int rr = i - m * kDecodeRows;
-      const int grow = row0 + rr;
-      const float v = acc_s[rr * 16 + m];
-      acc_s[rr * 16 + m] = 0.0f;
-      if (grow < N) {
-        if (split) {
-          atomicAdd(a.ws + static_cast<long long>(m) * N + grow, v);   // result unused: a reduction
-        } else {
-          a.Y[static_cast<long long>(m) * N + grow] = __float2half_rn(__half2float(a.scale[grow]) * v);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int m = 8 * nb + 2 * c + (i & 1);
+        const int row = (i < 2) ? row_a : row_b;
+        if (m < M && row < N) {
+          const long long idx = static_cast<long long>(m) * N + row;
+          if (split) atomicAdd(a.ws + idx, acc[0][nb][i]);   // result unused: a reduction
+          else a.Y[idx] = __float2half_rn(((i < 2) ? sa : sb) * acc[0][nb][i]);
         }
       }
     }
-    named_barrier_sync(1, kCT);
   }
   if (!ok && lane == 0) report_error(kErrDecodeConsumerWait);
 }

@@ -200,29 +200,42 @@ struct DecodePlan {
   int KPP, parts, tiles, units, smem, grid;
 };
 
-// Choose the K-part length: the fewest parts whose activation slice fits in
-// shared memory. Splitting a tile over parts costs a second (finalize) launch and
-// a round trip of fp32 partial sums, so it is used only when X does not fit.
+// Choose the K-part length. A part's activation slice (and, for INT4, its bias
+// table) must fit in shared memory beside the weight ring; among the part counts
+// that fit, take the one that spreads the (tile, part) units most evenly over the
+// SMs, preferring fewer parts (each split tile costs a round trip of fp32 partial
+// sums through the scratch buffer and a finalize launch).
 template <class C>
 bool plan_decode(const DeviceInfo& dev, int N, int K, DecodePlan* pl) {
   const int x_budget = dev.smem_optin - kDecodeFixedSmem - 1024;
-  const int k_round = (K + C::SK - 1) / C::SK * C::SK;
-  // per k of a part: 2 * MP bytes of activations, plus (INT4) 16 floats of bias per segment
-  const int per_k = 2 * C::kMP;
-  const int per_seg_bias = (C::kBits == 4) ? 16 * 4 : 0;
-  int kpp_max = x_budget / (per_k + per_seg_bias / C::SEGK + 1) / C::SK * C::SK;
-  if (kpp_max < C::SK) return false;
-  if (kpp_max > k_round) kpp_max = k_round;
-  const int chunks = k_round / C::SK;
-  const int parts_min = (k_round + kpp_max - 1) / kpp_max;
-  pl->KPP = (chunks + parts_min - 1) / parts_min * C::SK;
-  pl->parts = (K + pl->KPP - 1) / pl->KPP;
-  pl->tiles = (N + kDecodeRows - 1) / kDecodeRows;
-  const long long units = static_cast<long long>(pl->parts) * pl->tiles;
-  if (units > 0x7fffffffLL) return false;
-  pl->units = static_cast<int>(units);
+  const int stages = (K + C::SK - 1) / C::SK;
+  const int per_stage = 2 * C::kMP * C::SK + ((C::kBits == 4) ? 16 * 4 : 0);
+  const int max_spp = x_budget / per_stage;
+  if (max_spp < 1 || stages < 1) return false;
+  const int parts_min = (stages + max_spp - 1) / max_spp;
+  const long long tiles = (static_cast<long long>(N) + kDecodeRows - 1) / kDecodeRows;
+  if (tiles * stages > 0x7fffffffLL) return false;
+  int parts = parts_min;
+  double best = -1.0;
+  for (int P = parts_min; P <= stages && P <= parts_min + 16; ++P) {
+    const int spp = (stages + P - 1) / P;
+    if ((stages + spp - 1) / spp != P) continue;      // not a distinct split into equal-length parts
+    const long long units = tiles * P;
+    const long long grid = units < dev.sms ? units : dev.sms;
+    const double eff = (static_cast<double>(units) / grid) / ((units + grid - 1) / grid) *
+                       (static_cast<double>(grid) / dev.sms);
+    if (eff > best + 0.02) {
+      best = eff;
+      parts = P;
+    }
+  }
+  const int spp = (stages + parts - 1) / parts;
+  pl->KPP = spp * C::SK;
+  pl->parts = (stages + spp - 1) / spp;
+  pl->tiles = static_cast<int>(tiles);
+  pl->units = pl->parts * pl->tiles;
   pl->grid = pl->units < dev.sms ? pl->units : dev.sms;
-  pl->smem = kDecodeFixedSmem + 1024 + 2 * C::kMP * pl->KPP + per_seg_bias * (pl->KPP / C::SEGK);
+  pl->smem = kDecodeFixedSmem + 1024 + spp * per_stage;
   return pl->smem <= dev.smem_optin;
 }
 

@@ -159,6 +159,15 @@ GLMQ_API const char* glmq_status_string(int status);
 GLMQ_API int glmq_last_cuda_error(void);
 
 /*
+ * Number of kernels this library has enqueued since it was loaded, over all
+ * devices and threads: quantize, decode, tensor-core and finalize kernels. The
+ * stream memset of glmq_gemm_decode_noalloc is not a kernel and is not counted.
+ * A launch recorded into a CUDA graph during stream capture counts once, when it
+ * is captured; replays of the graph do not count. Host-only; never fails.
+ */
+GLMQ_API uint64_t glmq_kernel_launches(void);
+
+/*
  * Synchronizes `stream`, then reads and clears the current device's status
  * word, which kernels set when a bounded internal wait gives up (instead of
  * hanging). Returns GLMQ_OK if the word was 0, else GLMQ_ERR_DEVICE and, if

@@ -11,6 +11,7 @@ from ._binding import (  # noqa: F401
     gemm,
     gemm_decode,
     gemm_prefill,
+    kernel_launches,
     last_device_error,
     lib,
     packed_bytes,

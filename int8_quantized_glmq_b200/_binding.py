@@ -43,6 +43,7 @@ SIGNATURES = {
                                                 _vp]),
     "glmq_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "glmq_last_cuda_error": (ctypes.c_int, []),
+    "glmq_kernel_launches": (ctypes.c_uint64, []),
     "glmq_last_device_error": (ctypes.c_int, [_vp, ctypes.POINTER(ctypes.c_uint32)]),
 }
 
@@ -108,6 +109,11 @@ def raw_gemm(X: int, M: int, packed: int, scale: int, N: int, K: int, bits: int,
     return fn(X, M, packed, scale, N, K, bits, Y, stream)
 
 
+def kernel_launches() -> int:
+    """Kernels the library has enqueued since it was loaded (graph replays not included)."""
+    return int(lib().glmq_kernel_launches())
+
+
 def last_device_error(stream: int = 0):
     """(status, flags): synchronizes the stream and reads/clears the device status word."""
     flags = ctypes.c_uint32(0)
@@ -139,6 +145,24 @@ def _require(t, dtype, ndim, name):
         raise ValueError(f"{name} must be a contiguous {ndim}-D tensor")
 
 
+class _on_device:
+    """Makes t's device current for the call (a no-op when it already is)."""
+
+    def __init__(self, t):
+        torch = _torch()
+        idx = t.device.index
+        self._ctx = None if idx is None or idx == torch.cuda.current_device() else torch.cuda.device(idx)
+
+    def __enter__(self):
+        if self._ctx is not None:
+            self._ctx.__enter__()
+
+    def __exit__(self, *exc):
+        if self._ctx is not None:
+            self._ctx.__exit__(*exc)
+        return False
+
+
 def quantize(W, bits: int = 4, stream=None, out=None):
     """One-shot quantization of fp16 W[N, K] -> (packed uint8 [N, K*bits/8], scale fp16 [N])."""
     torch = _torch()
@@ -149,7 +173,7 @@ def quantize(W, bits: int = 4, stream=None, out=None):
         scale = torch.empty((N,), dtype=torch.float16, device=W.device)
     else:
         packed, scale = out
-    with torch.cuda.device(W.device):
+    with _on_device(W):
         st = raw_quantize(W.data_ptr(), N, K, bits, packed.data_ptr(), scale.data_ptr(), _stream_ptr(stream))
     _check(st, "glmq_quantize")
     return packed, scale
@@ -166,7 +190,7 @@ def gemm(X, packed, scale, bits: int = 4, stream=None, out=None, route: str = "a
     if packed.shape[1] * 8 != K * bits or scale.shape[0] != N:
         raise ValueError("packed/scale shapes do not match X and bits")
     Y = torch.empty((M, N), dtype=torch.float16, device=X.device) if out is None else out
-    with torch.cuda.device(X.device):
+    with _on_device(X):
         st = raw_gemm(X.data_ptr(), M, packed.data_ptr(), scale.data_ptr(), N, K, bits, Y.data_ptr(),
                       _stream_ptr(stream), route)
     _check(st, f"glmq_gemm({route})")

@@ -52,8 +52,9 @@ constexpr int kDecodeStageBytes = kDecodeRows * kDecodeSegB;          // 32 KB: 
 // ring + barriers; the activation slice follows
 constexpr int kDecodeFixedSmem = kDecodeStages * kDecodeStageBytes + 256;
 
-template <int BITS, int MP>
+template <int BITS, int MP, int CHAINS = 2>
 struct DecodeCfg {
+  static_assert(CHAINS == 2 || CHAINS == 4, "accumulator chains");
   static constexpr int kBits = BITS;
   static constexpr int kMP = MP;                    // token capacity of the activation layout (M <= MP)
   static constexpr int kNB = (MP + 7) / 8;          // n8 token blocks of the MMA
@@ -64,7 +65,7 @@ struct DecodeCfg {
   static constexpr int TK = TB * KPB;               // k per thread per segment
   static constexpr int TW = TB / 4;                 // 32-bit words per thread per row per segment (8)
   static constexpr int XU = TK / 8;                 // 16-byte activation units per thread per segment
-  static constexpr int kChains = 2;                 // independent MMA accumulator chains
+  static constexpr int kChains = CHAINS;            // independent MMA accumulator chains per token block
 };
 
 struct DecodeArgs {
@@ -178,10 +179,11 @@ __device__ __forceinline__ void decode_segment(uint32_t box, uint32_t xseg, uint
       uint32_t pa[4], pb[4];
       dequant_int4_word_biased(wa[j], pa);
       dequant_int4_word_biased(wb[j], pb);
+      const int h0 = (C::kChains == 4) ? 2 * (j & 1) : 0;
 #pragma unroll
       for (int nb = 0; nb < C::kNB; ++nb) {
-        mma_16816(acc[0][nb], pa[0], pb[0], pa[1], pb[1], bf[nb].x, bf[nb].y);
-        mma_16816(acc[1][nb], pa[2], pb[2], pa[3], pb[3], bf[nb].z, bf[nb].w);
+        mma_16816(acc[h0][nb], pa[0], pb[0], pa[1], pb[1], bf[nb].x, bf[nb].y);
+        mma_16816(acc[h0 + 1][nb], pa[2], pb[2], pa[3], pb[3], bf[nb].z, bf[nb].w);
       }
     }
     // remove the bias this segment added: bias_seg[t] = sum_k (1032 or 1152) * B[k][t]
@@ -207,11 +209,62 @@ __device__ __forceinline__ void decode_segment(uint32_t box, uint32_t xseg, uint
       dequant_int8_word(wb[2 * j2], pb0);
       dequant_int8_word(wa[2 * j2 + 1], pa1);
       dequant_int8_word(wb[2 * j2 + 1], pb1);
+      const int h0 = (C::kChains == 4) ? 2 * (j2 & 1) : 0;
 #pragma unroll
       for (int nb = 0; nb < C::kNB; ++nb) {
-        mma_16816(acc[0][nb], pa0[0], pb0[0], pa0[1], pb0[1], bf[nb].x, bf[nb].y);
-        mma_16816(acc[1][nb], pa1[0], pb1[0], pa1[1], pb1[1], bf[nb].z, bf[nb].w);
+        mma_16816(acc[h0][nb], pa0[0], pb0[0], pa0[1], pb0[1], bf[nb].x, bf[nb].y);
+        mma_16816(acc[h0 + 1][nb], pa1[0], pb1[0], pa1[1], pb1[1], bf[nb].z, bf[nb].w);
       }
+    }
+  }
+}
+
+// Copies the activation slice X[:, pk0 : pk0 + plen] into shared memory in the order
+// the B fragments are read (x_unit), INT4 slots permuted and high-nibble slots
+// divided by 16 (see dequant_int4_word_biased). Units of tokens >= M and of k past
+// plen are not written (no fragment of a real token reads them).
+template <class C>
+__device__ __forceinline__ void stage_activations(const __half* __restrict__ X, int K, int M, int pk0, int plen,
+                                                  uint8_t* xbuf, int ct) {
+  constexpr int kCT = kDecodeConsumerWarps * 32;
+  constexpr int kBatch = 8;
+  const int nseg = (plen + C::SEGK - 1) / C::SEGK;
+  const int total = nseg * C::XU * C::kMP * 4;                  // 16-byte units of the slice
+  for (int d0 = ct; d0 < total; d0 += kCT * kBatch) {
+    uint4 v[kBatch];
+    bool live[kBatch];
+#pragma unroll
+    for (int b = 0; b < kBatch; ++b) {
+      const int d = d0 + b * kCT;
+      const int cc = d & 3;
+      const int n = (d >> 2) % C::kMP;
+      const int rest = (d >> 2) / C::kMP;
+      const int jj = rest % C::XU;
+      const int sg = rest / C::XU;
+      const int kr = sg * C::SEGK + cc * C::TK + jj * 8;        // part-relative k of the 8 values
+      live[b] = d < total && n < M && kr < plen;
+      v[b] = make_uint4(0, 0, 0, 0);
+      if (live[b]) v[b] = __ldg(reinterpret_cast<const uint4*>(X + static_cast<long long>(n) * K + pk0 + kr));
+    }
+#pragma unroll
+    for (int b = 0; b < kBatch; ++b) {
+      if (!live[b]) continue;
+      uint4 o;
+      if constexpr (C::kBits == 4) {
+        // low-nibble slots (x0,x4), (x2,x6) as is; high-nibble slots (x1,x5), (x3,x7) divided by 16
+        const __half2 kSixteenth = __halves2half2(__ushort_as_half(0x2C00), __ushort_as_half(0x2C00));
+        o.x = prmt(v[b].x, v[b].z, 0x5410u);
+        uint32_t hy = prmt(v[b].x, v[b].z, 0x7632u);
+        o.z = prmt(v[b].y, v[b].w, 0x5410u);
+        uint32_t hw = prmt(v[b].y, v[b].w, 0x7632u);
+        __half2 sy = __hmul2(*reinterpret_cast<__half2*>(&hy), kSixteenth);
+        __half2 sw = __hmul2(*reinterpret_cast<__half2*>(&hw), kSixteenth);
+        o.y = *reinterpret_cast<uint32_t*>(&sy);
+        o.w = *reinterpret_cast<uint32_t*>(&sw);
+      } else {
+        o = v[b];
+      }
+      *reinterpret_cast<uint4*>(xbuf + 16u * static_cast<uint32_t>(d0 + b * kCT)) = o;
     }
   }
 }
@@ -303,34 +356,11 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     const int pk0 = p * a.KPP;
     const int plen = min(a.KPP, K - pk0);
     if (p != cur_part) {
-      // stage this part's activations in fragment order (all consumers, then barrier)
+      // stage this part's activations in fragment order (all consumers, then barrier).
+      // Thread i fills shared 16-byte unit i (conflict-free stores); each thread first
+      // issues all its global loads of a batch through the read-only path, then stores.
       named_barrier_sync(1, kCT);
-      const int chunks_per_row = plen >> 3;
-      for (int i = ct; i < M * chunks_per_row; i += kCT) {
-        const int n = i / chunks_per_row;
-        const int kr = (i - n * chunks_per_row) << 3;            // part-relative k of 8 values
-        const uint4 v = *reinterpret_cast<const uint4*>(a.X + static_cast<long long>(n) * K + pk0 + kr);
-        const int sg = kr / C::SEGK;
-        const int rem = kr - sg * C::SEGK;
-        const int cc = rem / C::TK;
-        const int jj = (rem - cc * C::TK) >> 3;
-        uint4 o;
-        if constexpr (C::kBits == 4) {
-          // low-nibble slots (x0,x4), (x2,x6) as is; high-nibble slots (x1,x5), (x3,x7) divided by 16
-          const __half2 kSixteenth = __halves2half2(__ushort_as_half(0x2C00), __ushort_as_half(0x2C00));
-          o.x = prmt(v.x, v.z, 0x5410u);
-          uint32_t hy = prmt(v.x, v.z, 0x7632u);
-          o.z = prmt(v.y, v.w, 0x5410u);
-          uint32_t hw = prmt(v.y, v.w, 0x7632u);
-          __half2 sy = __hmul2(*reinterpret_cast<__half2*>(&hy), kSixteenth);
-          __half2 sw = __hmul2(*reinterpret_cast<__half2*>(&hw), kSixteenth);
-          o.y = *reinterpret_cast<uint32_t*>(&sy);
-          o.w = *reinterpret_cast<uint32_t*>(&sw);
-        } else {
-          o = v;
-        }
-        *reinterpret_cast<uint4*>(xbuf + 16u * x_unit<C>(sg, jj, n, cc)) = o;
-      }
+      stage_activations<C>(a.X, K, M, pk0, plen, xbuf, ct);
       if constexpr (C::kBits == 4) {
         // per (segment, token) bias sum_k (1032 or 1152) * B[k], one warp per real pair
         // (lane = 8-value chunk of the 256-k segment), read back from the staged slice
@@ -398,7 +428,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
 #pragma unroll
     for (int nb = 0; nb < C::kNB; ++nb) {
 #pragma unroll
-      for (int i = 0; i < 4; ++i) acc[0][nb][i] += acc[1][nb][i];
+      for (int h = 1; h < C::kChains; ++h)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[0][nb][i] += acc[h][nb][i];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int m = 8 * nb + 2 * c + (i & 1);

@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 
 #include "glmq.h"
@@ -32,6 +33,17 @@ std::mutex g_mutex;
 glmq_status cuda_fail(cudaError_t e) {
   t_last_cuda_error = static_cast<int>(e);
   return GLMQ_ERR_CUDA;
+}
+
+// Kernels enqueued by this library since it was loaded (glmq_kernel_launches).
+std::atomic<unsigned long long> g_kernel_launches{0};
+
+// Status of the kernel launch just made on this thread; an accepted launch is counted.
+glmq_status launched() {
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e);
+  g_kernel_launches.fetch_add(1, std::memory_order_relaxed);
+  return GLMQ_OK;
 }
 
 // Current device's properties (queried once per device). Returns an error
@@ -117,8 +129,7 @@ template <int BITS, int CPT>
 glmq_status launch_quantize_cpt(const void* W, int64_t N, int64_t K, void* packed, void* scale, cudaStream_t s) {
   quantize_kernel<BITS, CPT><<<static_cast<unsigned>(N), kQuantThreads, 0, s>>>(
       static_cast<const __half*>(W), static_cast<int>(K), static_cast<uint8_t*>(packed), static_cast<__half*>(scale));
-  cudaError_t e = cudaGetLastError();
-  return e == cudaSuccess ? GLMQ_OK : cuda_fail(e);
+  return launched();
 }
 
 template <int BITS>
@@ -264,13 +275,12 @@ glmq_status launch_decode_cfg(const DeviceInfo& dev, const void* X, int M, const
   if (pl.parts > 1 && (st = decode_scratch(static_cast<size_t>(M) * N, &a.ws)) != GLMQ_OK) return st;
   if ((st = allow_smem(decode_kernel<C>, pl.smem)) != GLMQ_OK) return st;
   decode_kernel<C><<<pl.grid, kDecodeThreads, pl.smem, s>>>(tw, a);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_fail(e);
+  if ((st = launched()) != GLMQ_OK) return st;
   if (pl.parts > 1) {
     const long long total = static_cast<long long>(M) * N;
     const int blocks = static_cast<int>(std::min<long long>((total + 255) / 256, 4LL * dev.sms));
     decode_finalize_kernel<<<blocks, 256, 0, s>>>(a.ws, a.scale, a.Y, M, N);
-    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e);
+    if ((st = launched()) != GLMQ_OK) return st;
   }
   return GLMQ_OK;
 }
@@ -340,13 +350,12 @@ glmq_status launch_prefill_cfg(const DeviceInfo& dev, const void* X, int M, cons
   if ((st = allow_smem(prefill_kernel<C>, C::SMEM_BYTES)) != GLMQ_OK) return st;
   const int grid = a.units < dev.sms ? a.units : dev.sms;
   prefill_kernel<C><<<grid, kPrefillThreads, C::SMEM_BYTES, s>>>(tx, tw, a);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_fail(e);
+  if ((st = launched()) != GLMQ_OK) return st;
   if (a.parts > 1) {
     const long long total = static_cast<long long>(M) * N;
     const int blocks = static_cast<int>(std::min<long long>((total + 255) / 256, 4LL * dev.sms));
     decode_finalize_kernel<<<blocks, 256, 0, s>>>(a.ws, a.scale, a.Y, M, N);
-    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e);
+    if ((st = launched()) != GLMQ_OK) return st;
   }
   return GLMQ_OK;
 }
@@ -383,13 +392,12 @@ glmq_status launch_skinny_cfg(const DeviceInfo& dev, const void* X, int M, const
   if ((st = allow_smem(skinny_kernel<C>, C::SMEM_BYTES)) != GLMQ_OK) return st;
   const int grid = a.units < dev.sms ? a.units : dev.sms;
   skinny_kernel<C><<<grid, kSkinnyThreads, C::SMEM_BYTES, s>>>(tx, tw, a);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_fail(e);
+  if ((st = launched()) != GLMQ_OK) return st;
   if (a.parts > 1) {
     const long long total = static_cast<long long>(M) * N;
     const int blocks = static_cast<int>(std::min<long long>((total + 255) / 256, 4LL * dev.sms));
     decode_finalize_kernel<<<blocks, 256, 0, s>>>(a.ws, a.scale, a.Y, M, N);
-    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e);
+    if ((st = launched()) != GLMQ_OK) return st;
   }
   return GLMQ_OK;
 }
@@ -463,12 +471,12 @@ glmq_status launch_decode_noalloc_cfg(const DeviceInfo& dev, const void* X, int 
   }
   if ((st = allow_smem(decode_kernel<C>, pl.smem)) != GLMQ_OK) return st;
   decode_kernel<C><<<pl.grid, kDecodeThreads, pl.smem, s>>>(tw, a);
-  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e);
+  if ((st = launched()) != GLMQ_OK) return st;
   if (pl.parts > 1) {
     const long long total = static_cast<long long>(M) * N;
     const int blocks = static_cast<int>(std::min<long long>((total + 255) / 256, 4LL * dev.sms));
     decode_finalize_kernel<<<blocks, 256, 0, s>>>(a.ws, a.scale, a.Y, M, N);
-    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e);
+    if ((st = launched()) != GLMQ_OK) return st;
   }
   return GLMQ_OK;
 }
@@ -572,6 +580,8 @@ const char* glmq_status_string(int status) {
 }
 
 int glmq_last_cuda_error(void) { return t_last_cuda_error; }
+
+uint64_t glmq_kernel_launches(void) { return g_kernel_launches.load(std::memory_order_relaxed); }
 
 glmq_status glmq_last_device_error(void* stream, uint32_t* flags) {
   cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));

@@ -103,3 +103,12 @@ def test_binding_rejects_cpu_tensors():
     W = torch.zeros((4, 64), dtype=torch.float16)
     with pytest.raises(ValueError):
         glmq.quantize(W, 4)
+
+
+def test_kernel_launch_counter_ignores_rejected_calls():
+    n0 = glmq.kernel_launches()
+    assert n0 >= 0
+    assert B.raw_quantize(ALIGNED, 4, 100, 4, ALIGNED, ALIGNED) == B.ERR_BAD_SHAPE
+    assert B.raw_gemm(ALIGNED, 4, ALIGNED, ALIGNED, 8, 64, 3, ALIGNED, 0, "auto") == B.ERR_BAD_BITS
+    assert B.raw_gemm(0, 0, ALIGNED, ALIGNED, 8, 64, 4, 0, 0, "auto") == B.OK     # empty: nothing enqueued
+    assert glmq.kernel_launches() == n0

@@ -191,6 +191,17 @@ def test_auto_dispatch_matches_both_kernels():
         assert oracle.relative_max_error(Y, oracle.linear_forward(X, packed, scale, 4)) <= TIGHT
 
 
+def test_kernel_launch_counter_counts_each_kernel():
+    g = glmq()
+    W = gaussian_fp16((512, 1024), 0.02, 3)
+    n0 = g.kernel_launches()
+    packed, scale = g.quantize(to_dev(W), 4)
+    assert g.kernel_launches() == n0 + 1
+    n1 = g.kernel_launches()
+    g.gemm(to_dev(gaussian_fp16((1, 1024), 1.0, 4)), packed, scale, 4)
+    assert g.kernel_launches() - n1 in (1, 2)          # the kernel, plus a finalize kernel when K is split
+
+
 def test_no_device_error_reported():
     g = glmq()
     W = gaussian_fp16((64, 256), 0.02, 1)

@@ -55,10 +55,15 @@ def measured_peaks():
                 "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
-def source_digest() -> str:
+DECODE_SOURCES = ("decode.cuh", "glmq_ptx.cuh")
+
+
+def source_digest(files=DECODE_SOURCES) -> str:
+    """First 16 hex digits of the SHA-256 of the named kernel sources (the decode kernel's
+    by default); a profile's DRAM counters are used only while this digest matches."""
     csrc = os.path.join(ROOT, "int8_quantized_glmq_b200", "csrc")
     h = hashlib.sha256()
-    for f in sorted(os.listdir(csrc)):
+    for f in sorted(files):
         with open(os.path.join(csrc, f), "rb") as fh:
             h.update(f.encode())
             h.update(fh.read())

@@ -206,6 +206,14 @@ glmq_status decode_scratch(size_t ws_elems, float** out) {
   return GLMQ_OK;
 }
 
+// Grid of decode_finalize_kernel: about four CTAs per SM, 256-column blocks spread
+// over the M token rows (the kernel loops over rows past the grid's y extent).
+dim3 finalize_grid(const DeviceInfo& dev, int M, int N) {
+  const int rows = std::min(M, 65535);
+  const int per_row = std::max(1, std::min((N + 255) / 256, (4 * dev.sms + rows - 1) / rows));
+  return dim3(static_cast<unsigned>(per_row), static_cast<unsigned>(rows));
+}
+
 // ---------------------------------------------------------------- decode
 struct DecodePlan {
   int KPP, parts, tiles, units, smem, grid;
@@ -277,9 +285,7 @@ glmq_status launch_decode_cfg(const DeviceInfo& dev, const void* X, int M, const
   decode_kernel<C><<<pl.grid, kDecodeThreads, pl.smem, s>>>(tw, a);
   if ((st = launched()) != GLMQ_OK) return st;
   if (pl.parts > 1) {
-    const long long total = static_cast<long long>(M) * N;
-    const int blocks = static_cast<int>(std::min<long long>((total + 255) / 256, 4LL * dev.sms));
-    decode_finalize_kernel<<<blocks, 256, 0, s>>>(a.ws, a.scale, a.Y, M, N);
+    decode_finalize_kernel<<<finalize_grid(dev, M, N), 256, 0, s>>>(a.ws, a.scale, a.Y, M, N);
     if ((st = launched()) != GLMQ_OK) return st;
   }
   return GLMQ_OK;
@@ -352,9 +358,7 @@ glmq_status launch_prefill_cfg(const DeviceInfo& dev, const void* X, int M, cons
   prefill_kernel<C><<<grid, kPrefillThreads, C::SMEM_BYTES, s>>>(tx, tw, a);
   if ((st = launched()) != GLMQ_OK) return st;
   if (a.parts > 1) {
-    const long long total = static_cast<long long>(M) * N;
-    const int blocks = static_cast<int>(std::min<long long>((total + 255) / 256, 4LL * dev.sms));
-    decode_finalize_kernel<<<blocks, 256, 0, s>>>(a.ws, a.scale, a.Y, M, N);
+    decode_finalize_kernel<<<finalize_grid(dev, M, N), 256, 0, s>>>(a.ws, a.scale, a.Y, M, N);
     if ((st = launched()) != GLMQ_OK) return st;
   }
   return GLMQ_OK;
@@ -394,9 +398,7 @@ glmq_status launch_skinny_cfg(const DeviceInfo& dev, const void* X, int M, const
   skinny_kernel<C><<<grid, kSkinnyThreads, C::SMEM_BYTES, s>>>(tx, tw, a);
   if ((st = launched()) != GLMQ_OK) return st;
   if (a.parts > 1) {
-    const long long total = static_cast<long long>(M) * N;
-    const int blocks = static_cast<int>(std::min<long long>((total + 255) / 256, 4LL * dev.sms));
-    decode_finalize_kernel<<<blocks, 256, 0, s>>>(a.ws, a.scale, a.Y, M, N);
+    decode_finalize_kernel<<<finalize_grid(dev, M, N), 256, 0, s>>>(a.ws, a.scale, a.Y, M, N);
     if ((st = launched()) != GLMQ_OK) return st;
   }
   return GLMQ_OK;
@@ -473,9 +475,7 @@ glmq_status launch_decode_noalloc_cfg(const DeviceInfo& dev, const void* X, int 
   decode_kernel<C><<<pl.grid, kDecodeThreads, pl.smem, s>>>(tw, a);
   if ((st = launched()) != GLMQ_OK) return st;
   if (pl.parts > 1) {
-    const long long total = static_cast<long long>(M) * N;
-    const int blocks = static_cast<int>(std::min<long long>((total + 255) / 256, 4LL * dev.sms));
-    decode_finalize_kernel<<<blocks, 256, 0, s>>>(a.ws, a.scale, a.Y, M, N);
+    decode_finalize_kernel<<<finalize_grid(dev, M, N), 256, 0, s>>>(a.ws, a.scale, a.Y, M, N);
     if ((st = launched()) != GLMQ_OK) return st;
   }
   return GLMQ_OK;

@@ -185,6 +185,8 @@ glmq_status make_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void*
 struct DecodeScratch {
   float* ws = nullptr;
   size_t ws_elems = 0;
+  uint8_t* xs = nullptr;     // skinny kernel's activation image
+  size_t xs_bytes = 0;
 };
 DecodeScratch g_scratch[kMaxDevices];
 
@@ -212,6 +214,25 @@ dim3 finalize_grid(const DeviceInfo& dev, int M, int N) {
   const int rows = std::min(M, 65535);
   const int per_row = std::max(1, std::min((N + 255) / 256, (4 * dev.sms + rows - 1) / rows));
   return dim3(static_cast<unsigned>(per_row), static_cast<unsigned>(rows));
+}
+
+// Per-device buffer for the skinny kernel's pre-swizzled activation tiles (grown on
+// demand; fully rewritten by every call before it is read, so never cleared).
+glmq_status skinny_x_scratch(size_t bytes, uint8_t** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  std::lock_guard<std::mutex> lock(g_mutex);
+  DecodeScratch& sc = g_scratch[dev];
+  if (sc.xs_bytes < bytes) {
+    if (sc.xs) cudaFree(sc.xs);
+    sc.xs = nullptr;
+    sc.xs_bytes = 0;
+    if ((e = cudaMalloc(&sc.xs, bytes)) != cudaSuccess) return cuda_fail(e);
+    sc.xs_bytes = bytes;
+  }
+  *out = sc.xs;
+  return GLMQ_OK;
 }
 
 // ---------------------------------------------------------------- decode
@@ -339,6 +360,7 @@ glmq_status launch_prefill_cfg(const DeviceInfo& dev, const void* X, int M, cons
   a.scale = static_cast<const __half*>(scale);
   a.Y = static_cast<__half*>(Y);
   a.ws = nullptr;
+  a.xs = nullptr;
   a.M = M;
   a.N = N;
   a.K = K;
@@ -367,18 +389,19 @@ glmq_status launch_prefill_cfg(const DeviceInfo& dev, const void* X, int M, cons
 template <class C>
 glmq_status launch_skinny_cfg(const DeviceInfo& dev, const void* X, int M, const void* packed, const void* scale,
                               int N, int K, void* Y, cudaStream_t s) {
-  CUtensorMap tx, tw;
-  glmq_status st = make_map_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, X, K, M, uint64_t(K) * 2, 64, C::kBN,
-                               CU_TENSOR_MAP_SWIZZLE_128B);
-  if (st != GLMQ_OK) return st;
+  if (M > C::kBN) return GLMQ_ERR_BAD_SHAPE;   // one token tile: the activation image holds BN rows
+  CUtensorMap tw;
   const uint64_t row_bytes = uint64_t(K) / C::KPB;
-  st = make_map_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, packed, row_bytes, N, row_bytes, C::WB, C::BM,
-                   CU_TENSOR_MAP_SWIZZLE_128B);
+  glmq_status st = make_map_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, packed, row_bytes, N, row_bytes, C::WB, C::BM,
+                               CU_TENSOR_MAP_SWIZZLE_128B);
   if (st != GLMQ_OK) return st;
   PrefillArgs a;
   a.scale = static_cast<const __half*>(scale);
   a.Y = static_cast<__half*>(Y);
   a.ws = nullptr;
+  uint8_t* xs = nullptr;
+  if ((st = skinny_x_scratch(static_cast<size_t>(K / 64) * C::XT_BYTES, &xs)) != GLMQ_OK) return st;
+  a.xs = xs;
   a.M = M;
   a.N = N;
   a.K = K;
@@ -395,7 +418,13 @@ glmq_status launch_skinny_cfg(const DeviceInfo& dev, const void* X, int M, const
   if (C::SMEM_BYTES > dev.smem_optin) return GLMQ_ERR_BAD_SHAPE;
   if ((st = allow_smem(skinny_kernel<C>, C::SMEM_BYTES)) != GLMQ_OK) return st;
   const int grid = a.units < dev.sms ? a.units : dev.sms;
-  skinny_kernel<C><<<grid, kSkinnyThreads, C::SMEM_BYTES, s>>>(tx, tw, a);
+  {
+    const long long units16 = static_cast<long long>(K / 64) * C::kBN * 8;
+    const int blocks = static_cast<int>(std::min<long long>((units16 + 255) / 256, 8LL * dev.sms));
+    skinny_pack_x_kernel<C><<<blocks, 256, 0, s>>>(static_cast<const __half*>(X), M, K, xs);
+    if ((st = launched()) != GLMQ_OK) return st;
+  }
+  skinny_kernel<C><<<grid, kSkinnyThreads, C::SMEM_BYTES, s>>>(tw, a);
   if ((st = launched()) != GLMQ_OK) return st;
   if (a.parts > 1) {
     decode_finalize_kernel<<<finalize_grid(dev, M, N), 256, 0, s>>>(a.ws, a.scale, a.Y, M, N);

@@ -82,6 +82,7 @@ struct PrefillArgs {
   const __half* scale;
   __half* Y;
   float* ws;      // fp32 [M, N] scratch, zero on entry (used when parts > 1)
+  const uint8_t* xs;  // skinny kernel only: activation tiles pre-swizzled by skinny_pack_x_kernel
   int M;
   int N;
   int K;

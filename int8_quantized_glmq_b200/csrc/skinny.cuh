@@ -10,9 +10,13 @@
 // around a wide weight stream and cheap dequantization:
 //  * Stages hold one TMA box of 128 weight rows x 128 packed bytes (256 k for INT4,
 //    128 k for INT8; 128-byte swizzle) plus the matching activation tiles
-//    (BN tokens x 64 k each, 128-byte swizzle). Wide box rows matter: the TMA
-//    path serves a roughly fixed number of box rows per microsecond, so 128-byte
-//    rows stream several times faster than the 32-byte rows of a 64-wide K block.
+//    (BN tokens x 64 k each). Wide box rows matter: the TMA path serves a roughly
+//    fixed number of box rows per microsecond, so 128-byte rows stream several
+//    times faster than the 32-byte rows of a 64-wide K block, and the activation
+//    tiles do not take box rows at all: a small pre-pass (skinny_pack_x_kernel)
+//    writes X once per call as the exact shared-memory image of every tile (128-byte
+//    swizzle, INT4 k order, zero rows past M), and each stage fetches its tiles with
+//    one contiguous bulk copy.
 //  * The dequantized weights never touch shared memory: they are the MMA's A
 //    operand in tensor memory. Four dequantizer groups of 128 threads (thread =
 //    weight row = TMEM lane) take the 64-wide K blocks of the stream round-robin
@@ -22,9 +26,8 @@
 //    fp32 accumulator in TMEM); the epilogue warps read the accumulator with
 //    tcgen05.ld, multiply by s[n] and store fp16 (or add into the split-K scratch).
 //  * INT4 codes are dequantized in the order (0,4,1,5,2,6,3,7) within each group
-//    of 8, which costs no byte shuffle; the activation tile is permuted the same
-//    way in place after it lands (the MMA's k order is immaterial when both
-//    operands share it).
+//    of 8, which costs no byte shuffle; the pre-pass writes the activations in the
+//    same order (the MMA's k order is immaterial when both operands share it).
 //  * Work units are (128-row tile, K part) pairs exactly as in the prefill kernel,
 //    with the same split-K scratch and finalize kernel.
 // No TMA multicast is used anywhere.
@@ -59,7 +62,6 @@ struct SkinnyCfg {
   static constexpr int STAGE_BYTES = W_BYTES + KB * XT_BYTES;
   static constexpr int kStages = (kPrefillSmemBudget / STAGE_BYTES) < kPrefillMaxStages
                                      ? (kPrefillSmemBudget / STAGE_BYTES) : kPrefillMaxStages;
-  static constexpr int kPermX = (BITS == 4) ? 1 : 0;
   static constexpr int ACC_COLS = 2 * BN;                 // two accumulators of BN fp32 columns
   static constexpr int TMEM_COLS = 512;
   static constexpr int SMEM_BYTES = kStages * STAGE_BYTES + 1024 /*align*/ + 512 /*barriers*/;
@@ -93,13 +95,40 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32
       : "memory");
 }
 
+// Pre-pass: X fp16 [M, K] -> the shared-memory image of every activation tile the
+// skinny kernel reads: for 64-wide K block b, BN rows (tokens) of 128 bytes with the
+// 128-byte swizzle (16-byte unit u of row r at (u ^ (r & 7)) * 16), rows >= M zero,
+// INT4 values of each 8-group in the order (0,4,1,5,2,6,3,7). Tiles of consecutive
+// K blocks are contiguous, so a stage's tiles are one contiguous range.
+template <class C>
+__global__ void __launch_bounds__(256) skinny_pack_x_kernel(const __half* __restrict__ X, int M, int K,
+                                                            uint8_t* __restrict__ xs) {
+  const long long total = static_cast<long long>(K / 64) * C::kBN * 8;     // 16-byte units
+  for (long long i = blockIdx.x * 256LL + threadIdx.x; i < total; i += static_cast<long long>(gridDim.x) * 256) {
+    const int u = static_cast<int>(i & 7);
+    const long long rk = i >> 3;
+    const int r = static_cast<int>(rk % C::kBN);
+    const long long kb = rk / C::kBN;
+    uint4 o = make_uint4(0, 0, 0, 0);
+    if (r < M) {
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(X + static_cast<long long>(r) * K + kb * 64 + 8 * u));
+      if constexpr (C::kBits == 4) {
+        o = make_uint4(prmt(v.x, v.z, 0x5410u), prmt(v.x, v.z, 0x7632u), prmt(v.y, v.w, 0x5410u),
+                       prmt(v.y, v.w, 0x7632u));
+      } else {
+        o = v;
+      }
+    }
+    *reinterpret_cast<uint4*>(xs + kb * C::XT_BYTES + r * 128 + ((u ^ (r & 7)) << 4)) = o;
+  }
+}
+
 // Valid 64-wide K blocks of the stage that starts at k0.
 __device__ __forceinline__ int skinny_stage_kblocks(int k0, int K, int KB) { return min(KB, (K - k0) >> 6); }
 
 template <class C>
 __global__ void __launch_bounds__(kSkinnyThreads, 1)
-    skinny_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
-                  const PrefillArgs a) {
+    skinny_kernel(const __grid_constant__ CUtensorMap tmap_w, const PrefillArgs a) {
   constexpr int S = C::kStages;
   constexpr int NA = kSkinnyASlots;
   extern __shared__ uint8_t smem_raw[];
@@ -166,8 +195,8 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
           mbar_arrive_expect_tx(&full[stage], C::W_BYTES + nkb * C::XT_BYTES);
           armed[stage] = phase + 1;
           tma_load_2d(st, &tmap_w, k0 / C::KPB, nt * C::BM, &full[stage]);
-          for (int j = 0; j < nkb; ++j)
-            tma_load_2d(st + C::W_BYTES + j * C::XT_BYTES, &tmap_x, k0 + 64 * j, mt * C::kBN, &full[stage]);
+          bulk_g2s(st + C::W_BYTES, a.xs + (static_cast<long long>(mt) * (K / 64) + k0 / 64) * C::XT_BYTES,
+                   static_cast<uint32_t>(nkb * C::XT_BYTES), &full[stage]);
           if (++stage == S) { stage = 0; phase ^= 1; }
         }
       }
@@ -201,16 +230,6 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
           tc_fence_after();
           uint8_t* st = smem + stage * C::STAGE_BYTES;
           const uint32_t w_tile = smem_u32(st);
-          if constexpr (C::kPermX) {
-            // permute the activation tile of this K block to (0,4,1,5,2,6,3,7) per 8 values, in place
-            const uint32_t x_tile = smem_u32(st + C::W_BYTES + j * C::XT_BYTES);
-            for (int i = row; i < C::kBN * 8; i += 128) {
-              const uint4 v = lds_v4(x_tile + 16 * i);
-              st_shared_v4(x_tile + 16 * i, prmt(v.x, v.z, 0x5410u), prmt(v.x, v.z, 0x7632u),
-                           prmt(v.y, v.w, 0x5410u), prmt(v.y, v.w, 0x7632u));
-            }
-            fence_proxy_async_smem();
-          }
           uint32_t h[32];
           if constexpr (C::kBits == 4) {
             // bytes [32j, 32j+32) of this row: 16-byte units 2j and 2j+1, 128-byte swizzle

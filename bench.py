@@ -248,54 +248,57 @@ def run_decode(args, world, rank, local):
     alg_bytes = sum(quant[n][0].numel() + quant[n][1].numel() * 2 + xs[(M, n)].numel() * 2 + ys[(M, n)].numel() * 2
                     for (M, n) in launches)
 
-    # Each launch is captured once into its own CUDA graph (the eager call before it sizes
-    # the library's scratch and sets kernel attributes); a step replays the 12 graphs.
-    # The graphs hold exactly the kernels the public call enqueues, decode plus finalize.
+    # The timed steps are captured into one CUDA graph: K steps of the 12 public calls,
+    # with timing-event record nodes (external events) around every call, so the replay
+    # carries per-launch device times without host launch gaps between the calls. The
+    # eager calls before capture size the library's scratch and set kernel attributes.
     for (M, n) in launches:
         glmq.gemm(xs[(M, n)], quant[n][0], quant[n][1], bits, out=ys[(M, n)])
     torch.cuda.synchronize()
     cap_stream = torch.cuda.Stream()
-    graphs = []
-    n_capture0 = glmq.kernel_launches()
-    for (M, n) in launches:
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=cap_stream):
-            glmq.gemm(xs[(M, n)], quant[n][0], quant[n][1], bits, out=ys[(M, n)])
-        graphs.append(g)
-    kernels_per_step = glmq.kernel_launches() - n_capture0
 
+    def capture(n_steps, with_events):
+        g = torch.cuda.CUDAGraph()
+        evs = [[(torch.cuda.Event(enable_timing=True, external=True),
+                 torch.cuda.Event(enable_timing=True, external=True)) for _ in launches]
+               for _ in range(n_steps)] if with_events else None
+        edge = (torch.cuda.Event(enable_timing=True, external=True),
+                torch.cuda.Event(enable_timing=True, external=True)) if with_events else None
+        n0 = glmq.kernel_launches()
+        with torch.cuda.graph(g, stream=cap_stream):
+            if with_events:
+                edge[0].record()
+            for it in range(n_steps):
+                for j, (M, n) in enumerate(launches):
+                    if with_events:
+                        evs[it][j][0].record()
+                    glmq.gemm(xs[(M, n)], quant[n][0], quant[n][1], bits, out=ys[(M, n)])
+                    if with_events:
+                        evs[it][j][1].record()
+            if with_events:
+                edge[1].record()
+        return g, evs, edge, glmq.kernel_launches() - n0
+
+    warm_graph, _, _, _ = capture(args.warmup, False)
+    timed_graph, ev, (t0, t1), kernels_timed = capture(args.steps, True)
     stream = torch.cuda.current_stream()
-    for _ in range(args.warmup):
-        for g in graphs:
-            g.replay()
+    warm_graph.replay()
     torch.cuda.synchronize()
 
-    # per-launch device time of the dominant kernel, CUDA events on the launching stream,
-    # recorded inside the timed region around each launch
-    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in launches]
-          for _ in range(args.steps)]
     clocks = ClockSampler(local)
     clocks.start()
     barrier(world)
     torch.cuda.synchronize()
-    t0 = torch.cuda.Event(enable_timing=True)
-    t1 = torch.cuda.Event(enable_timing=True)
-    t0.record(stream)
-    for it in range(args.steps):
-        for j, g in enumerate(graphs):
-            ev[it][j][0].record(stream)
-            g.replay()
-            ev[it][j][1].record(stream)
-    t1.record(stream)
+    timed_graph.replay()
     torch.cuda.synchronize()
     barrier(world)
     clk = clocks.stop()
-    gpu_launches = kernels_per_step * args.steps
+    gpu_launches = kernels_timed
     elapsed = t0.elapsed_time(t1) / 1e3
     per_launch_s = [sum(ev[it][j][0].elapsed_time(ev[it][j][1]) for it in range(args.steps)) / 1e3 / args.steps
                     for j in range(len(launches))]
     value, elapsed_max = whole_job_rate(weight_bytes / 1e9, args.steps, elapsed, world)
-    del graphs
+    del warm_graph, timed_graph
 
     # e2e through the public API: pinned host X in, pinned host Y out, every step
     hx = {k: v.cpu().pin_memory() for k, v in xs.items()}

@@ -446,18 +446,4 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   if (!ok && lane == 0) report_error(kErrDecodeConsumerWait);
 }
 
-// Y[m, n] = fp16(s[n] * ws[m, n]) for split calls; returns ws to zero.
-// Grid: (column blocks, token-row blocks); rows m = blockIdx.y, blockIdx.y + gridDim.y, ...
-__global__ void __launch_bounds__(256) decode_finalize_kernel(float* __restrict__ ws, const __half* __restrict__ scale,
-                                                              __half* __restrict__ Y, int M, int N) {
-  for (int m = blockIdx.y; m < M; m += gridDim.y) {
-    const long long row = static_cast<long long>(m) * N;
-    for (int n = blockIdx.x * 256 + threadIdx.x; n < N; n += gridDim.x * 256) {
-      const float v = __ldcg(ws + row + n);
-      __stcg(ws + row + n, 0.0f);
-      Y[row + n] = __float2half_rn(__half2float(scale[n]) * v);
-    }
-  }
-}
-
 }  // namespace glmq

@@ -1,0 +1,47 @@
+// Finalize pass for GEMM calls whose tiles were split over K parts: the fp32 partial
+// sums of all parts have been added into a scratch buffer ws [M, N]; this kernel
+// applies the per-row scale, rounds to fp16 (the epilogue of the dequantizing linear
+// layer, Y = fp16(s[n] * sum_k X q)) and returns ws to zero for the next call.
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cstdint>
+
+namespace glmq {
+
+// Y[m, n] = fp16(s[n] * ws[m, n]) for split calls; returns ws to zero.
+// Grid: x covers the columns in groups of VEC per thread (one pass), y the token rows
+// (rows m = blockIdx.y, blockIdx.y + gridDim.y, ...). VEC = 4 needs N % 4 == 0, so
+// every group is 16-byte aligned in ws and 8-byte aligned in Y and scale.
+template <int VEC>
+__global__ void __launch_bounds__(256) decode_finalize_kernel(float* __restrict__ ws, const __half* __restrict__ scale,
+                                                              __half* __restrict__ Y, int M, int N) {
+  const int n = (blockIdx.x * 256 + threadIdx.x) * VEC;
+  if (n >= N) return;
+  if constexpr (VEC == 4) {
+    const uint2 sv = __ldg(reinterpret_cast<const uint2*>(scale + n));
+    const float2 s01 = __half22float2(*reinterpret_cast<const __half2*>(&sv.x));
+    const float2 s23 = __half22float2(*reinterpret_cast<const __half2*>(&sv.y));
+    for (int m = blockIdx.y; m < M; m += gridDim.y) {
+      const long long idx = static_cast<long long>(m) * N + n;
+      const float4 v = __ldcg(reinterpret_cast<const float4*>(ws + idx));
+      __stcg(reinterpret_cast<float4*>(ws + idx), make_float4(0.0f, 0.0f, 0.0f, 0.0f));
+      const __half2 y01 = __floats2half2_rn(s01.x * v.x, s01.y * v.y);
+      const __half2 y23 = __floats2half2_rn(s23.x * v.z, s23.y * v.w);
+      uint2 o;
+      o.x = *reinterpret_cast<const uint32_t*>(&y01);
+      o.y = *reinterpret_cast<const uint32_t*>(&y23);
+      *reinterpret_cast<uint2*>(Y + idx) = o;
+    }
+  } else {
+    const float sn = __half2float(scale[n]);
+    for (int m = blockIdx.y; m < M; m += gridDim.y) {
+      const long long idx = static_cast<long long>(m) * N + n;
+      const float v = __ldcg(ws + idx);
+      __stcg(ws + idx, 0.0f);
+      Y[idx] = __float2half_rn(sn * v);
+    }
+  }
+}
+
+}  // namespace glmq

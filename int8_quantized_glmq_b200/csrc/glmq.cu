@@ -9,6 +9,7 @@
 
 #include "glmq.h"
 #include "decode.cuh"
+#include "finalize.cuh"
 #include "prefill.cuh"
 #include "quantize.cuh"
 #include "skinny.cuh"
@@ -125,25 +126,28 @@ glmq_status check_gemm(const void* X, int64_t M, const void* packed, const void*
 }
 
 // ---------------------------------------------------------------- quantize
-template <int BITS, int CPT>
+template <int BITS, int CPT, int T>
 glmq_status launch_quantize_cpt(const void* W, int64_t N, int64_t K, void* packed, void* scale, cudaStream_t s) {
-  quantize_kernel<BITS, CPT><<<static_cast<unsigned>(N), kQuantThreads, 0, s>>>(
+  quantize_kernel<BITS, CPT, T><<<static_cast<unsigned>(N), T, 0, s>>>(
       static_cast<const __half*>(W), static_cast<int>(K), static_cast<uint8_t*>(packed), static_cast<__half*>(scale));
   return launched();
 }
 
+// Block size and chunks per thread from the row length (K <= GLMQ_MAX_K: at most
+// 8192 chunks of 8 values): 256 threads up to 6 chunks each, then 512 or 1024
+// threads with at most 8 chunks each.
 template <int BITS>
 glmq_status launch_quantize(const void* W, int64_t N, int64_t K, void* packed, void* scale, cudaStream_t s) {
-  const int64_t need = (K / 8 + kQuantThreads - 1) / kQuantThreads;  // 16-byte chunks per thread
-  if (need <= 1) return launch_quantize_cpt<BITS, 1>(W, N, K, packed, scale, s);
-  if (need <= 2) return launch_quantize_cpt<BITS, 2>(W, N, K, packed, scale, s);
-  if (need <= 4) return launch_quantize_cpt<BITS, 4>(W, N, K, packed, scale, s);
-  if (need <= 6) return launch_quantize_cpt<BITS, 6>(W, N, K, packed, scale, s);
-  if (need <= 8) return launch_quantize_cpt<BITS, 8>(W, N, K, packed, scale, s);
-  if (need <= 12) return launch_quantize_cpt<BITS, 12>(W, N, K, packed, scale, s);
-  if (need <= 16) return launch_quantize_cpt<BITS, 16>(W, N, K, packed, scale, s);
-  if (need <= 24) return launch_quantize_cpt<BITS, 24>(W, N, K, packed, scale, s);
-  return launch_quantize_cpt<BITS, 32>(W, N, K, packed, scale, s);
+  const int64_t chunks = K / 8;
+  if (chunks <= 256) return launch_quantize_cpt<BITS, 1, 256>(W, N, K, packed, scale, s);
+  if (chunks <= 512) return launch_quantize_cpt<BITS, 2, 256>(W, N, K, packed, scale, s);
+  if (chunks <= 1024) return launch_quantize_cpt<BITS, 4, 256>(W, N, K, packed, scale, s);
+  if (chunks <= 1536) return launch_quantize_cpt<BITS, 6, 256>(W, N, K, packed, scale, s);
+  if (chunks <= 2048) return launch_quantize_cpt<BITS, 4, 512>(W, N, K, packed, scale, s);
+  if (chunks <= 3072) return launch_quantize_cpt<BITS, 6, 512>(W, N, K, packed, scale, s);
+  if (chunks <= 4096) return launch_quantize_cpt<BITS, 8, 512>(W, N, K, packed, scale, s);
+  if (chunks <= 6144) return launch_quantize_cpt<BITS, 6, 1024>(W, N, K, packed, scale, s);
+  return launch_quantize_cpt<BITS, 8, 1024>(W, N, K, packed, scale, s);
 }
 
 // ---------------------------------------------------------------- TMA descriptors
@@ -208,12 +212,16 @@ glmq_status decode_scratch(size_t ws_elems, float** out) {
   return GLMQ_OK;
 }
 
-// Grid of decode_finalize_kernel: about four CTAs per SM, 256-column blocks spread
-// over the M token rows (the kernel loops over rows past the grid's y extent).
-dim3 finalize_grid(const DeviceInfo& dev, int M, int N) {
-  const int rows = std::min(M, 65535);
-  const int per_row = std::max(1, std::min((N + 255) / 256, (4 * dev.sms + rows - 1) / rows));
-  return dim3(static_cast<unsigned>(per_row), static_cast<unsigned>(rows));
+// Launches decode_finalize_kernel: one thread per group of 4 columns (1 when N is not
+// a multiple of 4) of every token row, all in one pass (rows beyond the grid's y
+// extent loop).
+glmq_status launch_finalize(float* ws, const __half* scale, __half* Y, int M, int N, cudaStream_t s) {
+  const bool vec = (N % 4) == 0;
+  const int groups = vec ? N / 4 : N;
+  const dim3 grid(static_cast<unsigned>((groups + 255) / 256), static_cast<unsigned>(std::min(M, 65535)));
+  if (vec) decode_finalize_kernel<4><<<grid, 256, 0, s>>>(ws, scale, Y, M, N);
+  else decode_finalize_kernel<1><<<grid, 256, 0, s>>>(ws, scale, Y, M, N);
+  return launched();
 }
 
 // Per-device buffer for the skinny kernel's pre-swizzled activation tiles (grown on
@@ -306,8 +314,7 @@ glmq_status launch_decode_cfg(const DeviceInfo& dev, const void* X, int M, const
   decode_kernel<C><<<pl.grid, kDecodeThreads, pl.smem, s>>>(tw, a);
   if ((st = launched()) != GLMQ_OK) return st;
   if (pl.parts > 1) {
-    decode_finalize_kernel<<<finalize_grid(dev, M, N), 256, 0, s>>>(a.ws, a.scale, a.Y, M, N);
-    if ((st = launched()) != GLMQ_OK) return st;
+    if ((st = launch_finalize(a.ws, a.scale, a.Y, M, N, s)) != GLMQ_OK) return st;
   }
   return GLMQ_OK;
 }
@@ -380,8 +387,7 @@ glmq_status launch_prefill_cfg(const DeviceInfo& dev, const void* X, int M, cons
   prefill_kernel<C><<<grid, kPrefillThreads, C::SMEM_BYTES, s>>>(tx, tw, a);
   if ((st = launched()) != GLMQ_OK) return st;
   if (a.parts > 1) {
-    decode_finalize_kernel<<<finalize_grid(dev, M, N), 256, 0, s>>>(a.ws, a.scale, a.Y, M, N);
-    if ((st = launched()) != GLMQ_OK) return st;
+    if ((st = launch_finalize(a.ws, a.scale, a.Y, M, N, s)) != GLMQ_OK) return st;
   }
   return GLMQ_OK;
 }
@@ -427,8 +433,7 @@ glmq_status launch_skinny_cfg(const DeviceInfo& dev, const void* X, int M, const
   skinny_kernel<C><<<grid, kSkinnyThreads, C::SMEM_BYTES, s>>>(tw, a);
   if ((st = launched()) != GLMQ_OK) return st;
   if (a.parts > 1) {
-    decode_finalize_kernel<<<finalize_grid(dev, M, N), 256, 0, s>>>(a.ws, a.scale, a.Y, M, N);
-    if ((st = launched()) != GLMQ_OK) return st;
+    if ((st = launch_finalize(a.ws, a.scale, a.Y, M, N, s)) != GLMQ_OK) return st;
   }
   return GLMQ_OK;
 }
@@ -504,8 +509,7 @@ glmq_status launch_decode_noalloc_cfg(const DeviceInfo& dev, const void* X, int 
   decode_kernel<C><<<pl.grid, kDecodeThreads, pl.smem, s>>>(tw, a);
   if ((st = launched()) != GLMQ_OK) return st;
   if (pl.parts > 1) {
-    decode_finalize_kernel<<<finalize_grid(dev, M, N), 256, 0, s>>>(a.ws, a.scale, a.Y, M, N);
-    if ((st = launched()) != GLMQ_OK) return st;
+    if ((st = launch_finalize(a.ws, a.scale, a.Y, M, N, s)) != GLMQ_OK) return st;
   }
   return GLMQ_OK;
 }

@@ -10,7 +10,9 @@
 //   q = 0 on rows whose scale rounds to 0, round half to even,
 //   INT4 byte j = (q[2j] & 0xF) | (q[2j+1] << 4)  (low nibble = even k).
 //
-// Kernel shape (HBM-bound): one CTA of 256 threads per row. Each thread loads
+// Kernel shape (HBM-bound): one CTA per row, 256 threads for rows up to 12288
+// values and 512 or 1024 for longer rows (so a thread holds at most 8 chunks and
+// enough CTAs stay resident to cover the memory latency). Each thread loads
 // its 16-byte chunks of the row once with streaming 128-bit loads and keeps them
 // in registers; the row absmax is an integer max over |w| bit patterns (a warp
 // reduce, then 8 warps through shared memory); the codes are formed from the
@@ -30,7 +32,6 @@
 
 namespace glmq {
 
-constexpr int kQuantThreads = 256;
 
 template <int BITS>
 __device__ __forceinline__ int exact_code(float w, float sf, float kf) {
@@ -81,10 +82,10 @@ __device__ __forceinline__ void chunk_codes(const uint4 v, float sf, float r, bo
   }
 }
 
-template <int BITS, int CPT>
-__global__ void __launch_bounds__(kQuantThreads) quantize_kernel(const __half* __restrict__ W, int K,
-                                                                  uint8_t* __restrict__ packed,
-                                                                  __half* __restrict__ scale) {
+// One CTA of T threads per row; each thread holds CPT 16-byte chunks of the row.
+template <int BITS, int CPT, int T>
+__global__ void __launch_bounds__(T) quantize_kernel(const __half* __restrict__ W, int K,
+                                                     uint8_t* __restrict__ packed, __half* __restrict__ scale) {
   constexpr int D = (1 << (BITS - 1)) - 1;
   const long long row = blockIdx.x;
   const int nchunks = K >> 3;
@@ -94,7 +95,7 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_kernel(const __half* _
   uint32_t m = 0;
 #pragma unroll
   for (int i = 0; i < CPT; ++i) {
-    const int c = threadIdx.x + i * kQuantThreads;
+    const int c = threadIdx.x + i * T;
     if (c < nchunks) {
       v[i] = ld_stream_v4(src + c);
       m = __vmaxu2(m, v[i].x & 0x7fff7fffu);
@@ -108,13 +109,13 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_kernel(const __half* _
   m = max(m & 0xffffu, m >> 16);
   m = __reduce_max_sync(0xffffffffu, m);
 
-  __shared__ uint32_t warp_max[kQuantThreads / 32];
+  __shared__ uint32_t warp_max[T / 32];
   const int warp = threadIdx.x >> 5;
   if ((threadIdx.x & 31) == 0) warp_max[warp] = m;
   __syncthreads();
   uint32_t a_bits = warp_max[0];
 #pragma unroll
-  for (int i = 1; i < kQuantThreads / 32; ++i) a_bits = max(a_bits, warp_max[i]);
+  for (int i = 1; i < T / 32; ++i) a_bits = max(a_bits, warp_max[i]);
 
   // a2: s = fp16_rn(fp32(a) / d)
   const float af = __half2float(__ushort_as_half(static_cast<unsigned short>(a_bits)));
@@ -128,7 +129,7 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_kernel(const __half* _
 
 #pragma unroll
   for (int i = 0; i < CPT; ++i) {
-    const int c = threadIdx.x + i * kQuantThreads;
+    const int c = threadIdx.x + i * T;
     if (c >= nchunks) continue;
     uint32_t u[8];
     if (zero_row) {

@@ -297,6 +297,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     fence_barrier_init();
   }
   __syncthreads();
+  // everything above touches only shared memory; X, W, Y and the scratch may belong
+  // to the previous kernel in the stream
+  griddep_wait();
+  if (threadIdx.x == 0) griddep_launch_dependents();
 
   if (warp == kDecodeConsumerWarps) {
     // ------------------------------------------------------------ producer warp

@@ -7,6 +7,8 @@
 #include <cuda_fp16.h>
 #include <cstdint>
 
+#include "glmq_ptx.cuh"
+
 namespace glmq {
 
 // Y[m, n] = fp16(s[n] * ws[m, n]) for split calls; returns ws to zero.
@@ -16,6 +18,7 @@ namespace glmq {
 template <int VEC>
 __global__ void __launch_bounds__(256) decode_finalize_kernel(float* __restrict__ ws, const __half* __restrict__ scale,
                                                               __half* __restrict__ Y, int M, int N) {
+  griddep_wait();   // the partial sums come from the kernel before this one
   const int n = (blockIdx.x * 256 + threadIdx.x) * VEC;
   if (n >= N) return;
   if constexpr (VEC == 4) {

@@ -47,6 +47,28 @@ glmq_status launched() {
   return GLMQ_OK;
 }
 
+// Launches kernel<<<grid, block, smem, s>>>(args...) with programmatic stream
+// serialization: it may begin (its shared-memory prologue) while the previous kernel
+// in the stream drains, and waits for that kernel (griddep_wait) before any
+// global-memory access. Counted like launched().
+template <typename... KArgs, typename... Args>
+glmq_status launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                       Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, args...);
+  if (e != cudaSuccess) return cuda_fail(e);
+  return launched();
+}
+
 // Current device's properties (queried once per device). Returns an error
 // status when the device is unusable.
 glmq_status current_device(const DeviceInfo** out) {
@@ -219,9 +241,8 @@ glmq_status launch_finalize(float* ws, const __half* scale, __half* Y, int M, in
   const bool vec = (N % 4) == 0;
   const int groups = vec ? N / 4 : N;
   const dim3 grid(static_cast<unsigned>((groups + 255) / 256), static_cast<unsigned>(std::min(M, 65535)));
-  if (vec) decode_finalize_kernel<4><<<grid, 256, 0, s>>>(ws, scale, Y, M, N);
-  else decode_finalize_kernel<1><<<grid, 256, 0, s>>>(ws, scale, Y, M, N);
-  return launched();
+  if (vec) return launch_pdl(decode_finalize_kernel<4>, grid, dim3(256), 0, s, ws, scale, Y, M, N);
+  return launch_pdl(decode_finalize_kernel<1>, grid, dim3(256), 0, s, ws, scale, Y, M, N);
 }
 
 // Per-device buffer for the skinny kernel's pre-swizzled activation tiles (grown on
@@ -311,8 +332,8 @@ glmq_status launch_decode_cfg(const DeviceInfo& dev, const void* X, int M, const
   a.units = pl.units;
   if (pl.parts > 1 && (st = decode_scratch(static_cast<size_t>(M) * N, &a.ws)) != GLMQ_OK) return st;
   if ((st = allow_smem(decode_kernel<C>, pl.smem)) != GLMQ_OK) return st;
-  decode_kernel<C><<<pl.grid, kDecodeThreads, pl.smem, s>>>(tw, a);
-  if ((st = launched()) != GLMQ_OK) return st;
+  if ((st = launch_pdl(decode_kernel<C>, dim3(pl.grid), dim3(kDecodeThreads), pl.smem, s, tw, a)) != GLMQ_OK)
+    return st;
   if (pl.parts > 1) {
     if ((st = launch_finalize(a.ws, a.scale, a.Y, M, N, s)) != GLMQ_OK) return st;
   }
@@ -506,8 +527,8 @@ glmq_status launch_decode_noalloc_cfg(const DeviceInfo& dev, const void* X, int 
       return cuda_fail(e);
   }
   if ((st = allow_smem(decode_kernel<C>, pl.smem)) != GLMQ_OK) return st;
-  decode_kernel<C><<<pl.grid, kDecodeThreads, pl.smem, s>>>(tw, a);
-  if ((st = launched()) != GLMQ_OK) return st;
+  if ((st = launch_pdl(decode_kernel<C>, dim3(pl.grid), dim3(kDecodeThreads), pl.smem, s, tw, a)) != GLMQ_OK)
+    return st;
   if (pl.parts > 1) {
     if ((st = launch_finalize(a.ws, a.scale, a.Y, M, N, s)) != GLMQ_OK) return st;
   }

@@ -91,11 +91,51 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
+// Same wait, but each try_wait may suspend the thread in hardware (up to 20 us per
+// try, still bounded by kWaitLimitNs overall) instead of returning at once, so a
+// waiting warp stops taking issue slots. Used by kernels whose waiting warps share
+// an SM sub-partition with a latency-critical issuer (the skinny kernel's MMA thread).
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(20000u)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ bool mbar_wait_suspend(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait_suspend(bar, parity)) return true;
+  const unsigned long long t0 = globaltimer_ns();
+  while (true) {
+    if (mbar_try_wait_suspend(bar, parity)) return true;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+  }
+}
+
+__device__ __forceinline__ bool mbar_wait_warp_suspend(uint64_t* bar, uint32_t parity) {
+  return __all_sync(0xffffffffu, mbar_wait_suspend(bar, parity));
+}
+
 // Warp-uniform wait: every lane waits, and the warp agrees on the outcome, so the
 // result can gate warp-collective instructions (mma.sync, tcgen05.ld, __syncwarp).
 __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity) {
   return __all_sync(0xffffffffu, mbar_wait(bar, parity));
 }
+
+// ---------------------------------------------------------------- programmatic dependent launch
+// A kernel launched with programmatic stream serialization may start while the
+// previous kernel in the stream is still running. griddep_wait() blocks until that
+// kernel has completed and its memory operations are visible; every thread calls it
+// before its first global-memory access. griddep_launch_dependents() lets the next
+// such kernel start launching once every CTA of this grid has called it or exited;
+// only single-wave grids call it (all their CTAs are resident before any dependent
+// CTA can take an SM). Both are no-ops for a kernel launched without the attribute.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" :::); }
 
 // ---------------------------------------------------------------- bulk async copy (no multicast)
 // Contiguous global -> shared copy whose completion is counted on an mbarrier

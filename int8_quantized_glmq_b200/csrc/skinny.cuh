@@ -188,7 +188,7 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
         const int mt = t - nt * a.tiles_m;
         const int st1 = min(num_st, (p + 1) * a.kbp);
         for (int ks = p * a.kbp; ks < st1; ++ks) {
-          if (!mbar_wait(&empty[stage], phase ^ 1)) { ok = false; break; }
+          if (!mbar_wait_suspend(&empty[stage], phase ^ 1)) { ok = false; break; }
           const int k0 = ks * C::SK;
           const int nkb = skinny_stage_kblocks(k0, K, C::KB);
           uint8_t* st = smem + stage * C::STAGE_BYTES;
@@ -202,7 +202,7 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
       }
       bool drained = true;
       for (int s = 0; s < S; ++s)
-        if (armed[s] && !mbar_wait(&full[s], armed[s] - 1)) drained = false;
+        if (armed[s] && !mbar_wait_suspend(&full[s], armed[s] - 1)) drained = false;
       if (!ok || !drained) report_error(kErrPrefillWait);
     }
   } else if (warp < kSkinnyDequantWarps) {
@@ -222,11 +222,11 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
         for (int j = 0; j < nkb; ++j, ++kseq) {
           if ((kseq & (kSkinnyGroups - 1)) != grp) continue;
           if (!waited) {
-            if (!mbar_wait_warp(&full[stage], phase)) { ok = false; break; }
+            if (!mbar_wait_warp_suspend(&full[stage], phase)) { ok = false; break; }
             waited = true;
           }
           const int slot = kseq % NA;
-          if (!mbar_wait_warp(&aempty[slot], ((kseq / NA) & 1) ^ 1)) { ok = false; break; }
+          if (!mbar_wait_warp_suspend(&aempty[slot], ((kseq / NA) & 1) ^ 1)) { ok = false; break; }
           tc_fence_after();
           uint8_t* st = smem + stage * C::STAGE_BYTES;
           const uint32_t w_tile = smem_u32(st);
@@ -283,7 +283,7 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
         const int st1 = min(num_st, st0 + a.kbp);
         const int ab = it & 1;
         const uint32_t aphase = (it >> 1) & 1;
-        if (!mbar_wait(&accempty[ab], aphase ^ 1)) { ok = false; break; }
+        if (!mbar_wait_suspend(&accempty[ab], aphase ^ 1)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + ab * C::kBN;
         bool first = true;
@@ -292,7 +292,7 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
           uint8_t* st = smem + stage * C::STAGE_BYTES;
           for (int j = 0; j < nkb; ++j, ++kseq) {
             const int slot = kseq % NA;
-            if (!mbar_wait(&afull[slot], (kseq / NA) & 1)) { ok = false; break; }
+            if (!mbar_wait_suspend(&afull[slot], (kseq / NA) & 1)) { ok = false; break; }
             tc_fence_after();
             const uint32_t x_addr = smem_u32(st + C::W_BYTES + j * C::XT_BYTES);
             const uint32_t a_tmem = tmem_base + C::ACC_COLS + slot * 32;
@@ -314,7 +314,7 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
       }
       bool drained = true;
       for (int b = 0; b < 2; ++b)
-        if (acc_armed[b] && !mbar_wait(&accfull[b], acc_armed[b] - 1)) drained = false;
+        if (acc_armed[b] && !mbar_wait_suspend(&accfull[b], acc_armed[b] - 1)) drained = false;
       if (!ok || !drained) report_error(kErrPrefillWait);
     }
   } else {
@@ -325,7 +325,7 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
     for (int u = blockIdx.x; u < a.units && ok; u += G, ++it) {
       const int ab = it & 1;
       const uint32_t aphase = (it >> 1) & 1;
-      if (!mbar_wait_warp(&accfull[ab], aphase)) { ok = false; break; }
+      if (!mbar_wait_warp_suspend(&accfull[ab], aphase)) { ok = false; break; }
       tc_fence_after();
       const int t = u % a.tiles;
       const int nt = t / a.tiles_m;

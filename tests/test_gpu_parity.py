@@ -191,6 +191,32 @@ def test_auto_dispatch_matches_both_kernels():
         assert oracle.relative_max_error(Y, oracle.linear_forward(X, packed, scale, 4)) <= TIGHT
 
 
+@pytest.mark.parametrize("bits,M", [(4, 1), (4, 16), (8, 4)])
+def test_chained_calls_read_the_previous_output(bits, M):
+    """Three back-to-back calls on one stream, each call's X being the previous call's Y.
+
+    The decode and finalize kernels may begin while the kernel before them is still
+    running and must wait for it before reading its output. With N = K = 4096 these
+    calls split tiles over K parts, so the chain alternates decode and finalize
+    kernels. Reference: the oracle chain (Y rounded to fp16 between layers)."""
+    import torch
+    g = glmq()
+    K = 4096
+    layers = [oracle.quantize_linear(gaussian_fp16((K, K), 0.02, 500 + i), bits) for i in range(3)]
+    dev = [(to_dev(p), to_dev(s)) for p, s in layers]
+    X = gaussian_fp16((M, K), 1.0, 600 + M)
+    x = to_dev(X)
+    torch.cuda.synchronize()
+    for p, s in dev:
+        x = g.gemm(x, p, s, bits)                    # no host work between the launches
+    Y = to_host(x)
+    ref = X
+    for p, s in layers:
+        ref = oracle.linear_forward(ref, p, s, bits)
+    assert np.all(np.isfinite(Y))
+    assert oracle.relative_max_error(Y, ref) <= TOL
+
+
 def test_kernel_launch_counter_counts_each_kernel():
     g = glmq()
     W = gaussian_fp16((512, 1024), 0.02, 3)

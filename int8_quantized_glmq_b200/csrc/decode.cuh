@@ -45,7 +45,7 @@ namespace glmq {
 
 constexpr int kDecodeConsumerWarps = 16;
 constexpr int kDecodeThreads = (kDecodeConsumerWarps + 1) * 32;
-constexpr int kDecodeStages = 4;
+constexpr int kDecodeStages = 6;
 constexpr int kDecodeRows = 16 * kDecodeConsumerWarps;                // rows per tile (256)
 constexpr int kDecodeSegB = 128;         // packed bytes per row per stage (one TMA box width)
 constexpr int kDecodeStageBytes = kDecodeRows * kDecodeSegB;          // 32 KB: one TMA box per stage

@@ -37,6 +37,7 @@ sys.path.insert(0, ROOT)
 METRIC = "W4A16 GEMM weight GB/s (decode) and TFLOP/s (prefill) vs B200 roofline"
 HIDDEN = 12288
 DECODE_MS = (1, 4, 16)
+EVENT_EVERY = 4          # timed steps that carry per-launch timing events: 0, 4, 8, ...
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 
@@ -248,10 +249,12 @@ def run_decode(args, world, rank, local):
     alg_bytes = sum(quant[n][0].numel() + quant[n][1].numel() * 2 + xs[(M, n)].numel() * 2 + ys[(M, n)].numel() * 2
                     for (M, n) in launches)
 
-    # The timed steps are captured into one CUDA graph: K steps of the 12 public calls,
-    # with timing-event record nodes (external events) around every call, so the replay
-    # carries per-launch device times without host launch gaps between the calls. The
-    # eager calls before capture size the library's scratch and set kernel attributes.
+    # The timed steps are captured into one CUDA graph: K steps of the 12 public calls.
+    # Every EVENT_EVERY-th step carries timing-event record nodes (external events)
+    # around each call; those give the per-launch device times of the roofline. The
+    # other steps run as a plain chain of kernels (event nodes between kernels add
+    # gaps and cut the programmatic-launch edges, so they are kept to a sample).
+    # The eager calls before capture size the library's scratch and set attributes.
     for (M, n) in launches:
         glmq.gemm(xs[(M, n)], quant[n][0], quant[n][1], bits, out=ys[(M, n)])
     torch.cuda.synchronize()
@@ -259,9 +262,9 @@ def run_decode(args, world, rank, local):
 
     def capture(n_steps, with_events):
         g = torch.cuda.CUDAGraph()
-        evs = [[(torch.cuda.Event(enable_timing=True, external=True),
-                 torch.cuda.Event(enable_timing=True, external=True)) for _ in launches]
-               for _ in range(n_steps)] if with_events else None
+        sampled = [it for it in range(n_steps) if with_events and it % EVENT_EVERY == 0]
+        evs = {it: [(torch.cuda.Event(enable_timing=True, external=True),
+                     torch.cuda.Event(enable_timing=True, external=True)) for _ in launches] for it in sampled}
         edge = (torch.cuda.Event(enable_timing=True, external=True),
                 torch.cuda.Event(enable_timing=True, external=True)) if with_events else None
         n0 = glmq.kernel_launches()
@@ -270,10 +273,10 @@ def run_decode(args, world, rank, local):
                 edge[0].record()
             for it in range(n_steps):
                 for j, (M, n) in enumerate(launches):
-                    if with_events:
+                    if it in evs:
                         evs[it][j][0].record()
                     glmq.gemm(xs[(M, n)], quant[n][0], quant[n][1], bits, out=ys[(M, n)])
-                    if with_events:
+                    if it in evs:
                         evs[it][j][1].record()
             if with_events:
                 edge[1].record()
@@ -295,7 +298,7 @@ def run_decode(args, world, rank, local):
     clk = clocks.stop()
     gpu_launches = kernels_timed
     elapsed = t0.elapsed_time(t1) / 1e3
-    per_launch_s = [sum(ev[it][j][0].elapsed_time(ev[it][j][1]) for it in range(args.steps)) / 1e3 / args.steps
+    per_launch_s = [sum(ev[it][j][0].elapsed_time(ev[it][j][1]) for it in ev) / 1e3 / len(ev)
                     for j in range(len(launches))]
     value, elapsed_max = whole_job_rate(weight_bytes / 1e9, args.steps, elapsed, world)
     del warm_graph, timed_graph
@@ -306,20 +309,38 @@ def run_decode(args, world, rank, local):
     h2d = sum(v.numel() * 2 for v in hx.values())
     d2h = sum(v.numel() * 2 for v in hy.values())
 
+    # H2D of each call's X on one copy stream, the call on the compute stream, D2H of
+    # its Y on another copy stream, ordered by events: copies of one call overlap the
+    # compute of the others, as a serving loop would arrange it.
+    h2d_stream, d2h_stream = torch.cuda.Stream(), torch.cuda.Stream()
+
     def e2e_step():
         for (M, n) in launches:
-            xd = hx[(M, n)].to("cuda", non_blocking=True)
+            with torch.cuda.stream(h2d_stream):
+                xd = hx[(M, n)].to("cuda", non_blocking=True)
+                x_ready = torch.cuda.Event()
+                x_ready.record(h2d_stream)
+            stream.wait_event(x_ready)
+            xd.record_stream(stream)
             y = glmq.gemm(xd, quant[n][0], quant[n][1], bits)
-            hy[(M, n)].copy_(y, non_blocking=True)
+            y_ready = torch.cuda.Event()
+            y_ready.record(stream)
+            d2h_stream.wait_event(y_ready)
+            with torch.cuda.stream(d2h_stream):
+                hy[(M, n)].copy_(y, non_blocking=True)
+            y.record_stream(d2h_stream)
 
     for _ in range(args.warmup):
         e2e_step()
+    stream.wait_stream(d2h_stream)
     barrier(world)
     torch.cuda.synchronize()
     a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a0.record(stream)
+    h2d_stream.wait_stream(stream)      # the timed copies start after a0
     for _ in range(args.steps):
         e2e_step()
+    stream.wait_stream(d2h_stream)      # a1 after the last result is in host memory
     a1.record(stream)
     torch.cuda.synchronize()
     barrier(world)

@@ -13,3 +13,11 @@ from .glmq_oracle import (  # noqa: F401
     linear_forward_rows,
     relative_max_error,
 )
+from .glmq_epilogue import (  # noqa: F401,E402
+    linear_pre,
+    linear_bias_forward,
+    gelu,
+    geglu_forward,
+    geglu_row_order,
+    quantize_linear_geglu,
+)

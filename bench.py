@@ -398,6 +398,23 @@ def run_extras(torch, glmq, W16, quant, peaks):
         out["prefill_int4_m2048"][name] = {"us": round(t * 1e6, 1), "tflops": round(tf, 1),
                                            "frac_burst": round(tf / peaks["bf16_tflops"], 4)}
         del X, Y
+    # FFN-up with the fused GeGLU epilogue (plus an fp16 bias) against the plain call
+    N, K = GLM_PROJECTIONS["ffn_up"]
+    pg, sg = glmq.quantize(W16["ffn_up"], 4, geglu=True)
+    gb = torch.Generator(device="cuda").manual_seed(5000)
+    bias = (torch.randn((N,), generator=gb, device="cuda", dtype=torch.float32) * 0.1).half()
+    out["ffn_up_geglu_int4"] = {}
+    for M in (1, 16, 2048):
+        g = torch.Generator(device="cuda").manual_seed(6000 + M)
+        X = torch.randn((M, K), generator=g, device="cuda", dtype=torch.float32).half()
+        Yg = torch.empty((M, N // 2), dtype=torch.float16, device="cuda")
+        Yp = torch.empty((M, N), dtype=torch.float16, device="cuda")
+        tg = time_launches(torch, lambda: glmq.gemm_fused(X, pg, sg, 4, bias=bias, epilogue="geglu", out=Yg), 5)
+        tp = time_launches(torch, lambda: glmq.gemm(X, pg, sg, 4, out=Yp), 5)
+        out["ffn_up_geglu_int4"][f"M={M}"] = {"fused_us": round(tg * 1e6, 1), "plain_us": round(tp * 1e6, 1),
+                                               "fused_weight_gbs": round(pg.numel() / tg / 1e9, 1)}
+        del X, Yg, Yp
+    del pg, sg
     for name in PROJECTION_ORDER:
         N, K = GLM_PROJECTIONS[name]
         p8 = torch.empty((N, K), dtype=torch.uint8, device="cuda")

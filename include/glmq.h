@@ -124,6 +124,38 @@ GLMQ_API glmq_status glmq_gemm_prefill(const void* X, int64_t M, const void* pac
                               int64_t N, int64_t K, int bits, void* Y, void* stream);
 
 /*
+ * One-shot quantization like glmq_quantize, with the packed rows (and scales) stored
+ * in the layout the fused GeGLU epilogue reads (GLM-130B paper card, "Method": the
+ * feed-forward block is a GeGLU; FFN-up holds both GLU branches, rows 0 .. N/2-1 the
+ * first and N/2 .. N-1 the second). Packed row 16g + r holds row 8g + r of W for
+ * r < 8 and row N/2 + 8g + r - 8 for r >= 8.
+ *   Same arguments and codes as glmq_quantize; only the row order differs.
+ *   Requires N % 16 == 0, else GLMQ_ERR_BAD_SHAPE.
+ */
+GLMQ_API glmq_status glmq_quantize_geglu(const void* W, int64_t N, int64_t K, int bits, void* packed, void* scale,
+                                         void* stream);
+
+/* Epilogues of glmq_gemm_fused. */
+#define GLMQ_EPILOGUE_NONE 0
+#define GLMQ_EPILOGUE_GEGLU 1
+
+/*
+ * glmq_gemm with a fused epilogue (paper card, "Paper vs code": biases stay FP16;
+ * "Method": GeGLU feed-forward block).
+ *   bias      in : fp16 [N] in the natural row order of W, or NULL; 2-byte aligned.
+ *   epilogue     : GLMQ_EPILOGUE_NONE:  Y [M, N],   Y = fp16( s[n] * sum_k X q + bias[n] )
+ *                  GLMQ_EPILOGUE_GEGLU: Y [M, N/2], with U = s * sum_k X q + bias over the
+ *                  N = 2F rows, Y[m,j] = fp16( GELU(U[m,j]) * U[m,F+j] ), GELU(u) =
+ *                  0.5 u (1 + erf(u / sqrt 2)); packed and scale must come from
+ *                  glmq_quantize_geglu, and N % 16 == 0.
+ * Other arguments, dispatch, scratch and errors as glmq_gemm; an unknown epilogue
+ * value is GLMQ_ERR_BAD_SHAPE.
+ */
+GLMQ_API glmq_status glmq_gemm_fused(const void* X, int64_t M, const void* packed, const void* scale,
+                                     const void* bias, int64_t N, int64_t K, int bits, int epilogue, void* Y,
+                                     void* stream);
+
+/*
  * glmq_gemm_decode without any device allocation (the paper has no counterpart:
  * this is a deployment variant of the decode kernel).
  *

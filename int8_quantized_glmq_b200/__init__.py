@@ -5,10 +5,13 @@ The compute lives in ``libglmq.so`` (CUDA C++ for sm_100a, C ABI in
 """
 from ._binding import (  # noqa: F401
     DECODE_MAX_M,
+    EPILOGUE_GEGLU,
+    EPILOGUE_NONE,
     MAX_K,
     GlmqError,
     abi_version,
     gemm,
+    gemm_fused,
     gemm_decode,
     gemm_prefill,
     kernel_launches,

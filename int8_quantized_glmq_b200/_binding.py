@@ -28,6 +28,8 @@ DECODE_MAX_M = 16
 DECODE_AUTO_MAX_M = 16
 MAX_K = 65536
 NOALLOC_SCRATCH_FLOATS = 1 << 20
+EPILOGUE_NONE = 0
+EPILOGUE_GEGLU = 1
 
 #: every symbol include/glmq.h declares, with (restype, argtypes)
 _c_int64 = ctypes.c_int64
@@ -36,6 +38,9 @@ SIGNATURES = {
     "glmq_abi_version": (ctypes.c_int, []),
     "glmq_packed_bytes": (ctypes.c_size_t, [_c_int64, _c_int64, ctypes.c_int]),
     "glmq_quantize": (ctypes.c_int, [_vp, _c_int64, _c_int64, ctypes.c_int, _vp, _vp, _vp]),
+    "glmq_quantize_geglu": (ctypes.c_int, [_vp, _c_int64, _c_int64, ctypes.c_int, _vp, _vp, _vp]),
+    "glmq_gemm_fused": (ctypes.c_int, [_vp, _c_int64, _vp, _vp, _vp, _c_int64, _c_int64, ctypes.c_int, ctypes.c_int,
+                                       _vp, _vp]),
     "glmq_gemm": (ctypes.c_int, [_vp, _c_int64, _vp, _vp, _c_int64, _c_int64, ctypes.c_int, _vp, _vp]),
     "glmq_gemm_decode": (ctypes.c_int, [_vp, _c_int64, _vp, _vp, _c_int64, _c_int64, ctypes.c_int, _vp, _vp]),
     "glmq_gemm_prefill": (ctypes.c_int, [_vp, _c_int64, _vp, _vp, _c_int64, _c_int64, ctypes.c_int, _vp, _vp]),
@@ -102,6 +107,15 @@ def raw_quantize(W: int, N: int, K: int, bits: int, packed: int, scale: int, str
     return lib().glmq_quantize(W, N, K, bits, packed, scale, stream)
 
 
+def raw_quantize_geglu(W: int, N: int, K: int, bits: int, packed: int, scale: int, stream: int = 0) -> int:
+    return lib().glmq_quantize_geglu(W, N, K, bits, packed, scale, stream)
+
+
+def raw_gemm_fused(X: int, M: int, packed: int, scale: int, bias: int, N: int, K: int, bits: int, epilogue: int,
+                   Y: int, stream: int = 0) -> int:
+    return lib().glmq_gemm_fused(X, M, packed, scale, bias, N, K, bits, epilogue, Y, stream)
+
+
 def raw_gemm(X: int, M: int, packed: int, scale: int, N: int, K: int, bits: int, Y: int, stream: int = 0,
              route: str = "auto") -> int:
     fn = {"auto": lib().glmq_gemm, "decode": lib().glmq_gemm_decode, "prefill": lib().glmq_gemm_prefill,
@@ -163,8 +177,11 @@ class _on_device:
         return False
 
 
-def quantize(W, bits: int = 4, stream=None, out=None):
-    """One-shot quantization of fp16 W[N, K] -> (packed uint8 [N, K*bits/8], scale fp16 [N])."""
+def quantize(W, bits: int = 4, stream=None, out=None, geglu: bool = False):
+    """One-shot quantization of fp16 W[N, K] -> (packed uint8 [N, K*bits/8], scale fp16 [N]).
+
+    geglu=True stores the rows in the layout of the fused GeGLU epilogue
+    (glmq_quantize_geglu); N must then be a multiple of 16."""
     torch = _torch()
     _require(W, torch.float16, 2, "W")
     N, K = W.shape
@@ -173,9 +190,10 @@ def quantize(W, bits: int = 4, stream=None, out=None):
         scale = torch.empty((N,), dtype=torch.float16, device=W.device)
     else:
         packed, scale = out
+    fn = raw_quantize_geglu if geglu else raw_quantize
     with _on_device(W):
-        st = raw_quantize(W.data_ptr(), N, K, bits, packed.data_ptr(), scale.data_ptr(), _stream_ptr(stream))
-    _check(st, "glmq_quantize")
+        st = fn(W.data_ptr(), N, K, bits, packed.data_ptr(), scale.data_ptr(), _stream_ptr(stream))
+    _check(st, "glmq_quantize_geglu" if geglu else "glmq_quantize")
     return packed, scale
 
 
@@ -194,6 +212,31 @@ def gemm(X, packed, scale, bits: int = 4, stream=None, out=None, route: str = "a
         st = raw_gemm(X.data_ptr(), M, packed.data_ptr(), scale.data_ptr(), N, K, bits, Y.data_ptr(),
                       _stream_ptr(stream), route)
     _check(st, f"glmq_gemm({route})")
+    return Y
+
+
+def gemm_fused(X, packed, scale, bits: int = 4, bias=None, epilogue: str = "none", stream=None, out=None):
+    """glmq_gemm_fused: Y = fp16(s * X q + bias) [M, N], or with epilogue="geglu" (packed
+    from quantize(..., geglu=True)) Y[m, j] = fp16(GELU(U[m, j]) * U[m, N/2 + j]) [M, N/2]."""
+    torch = _torch()
+    _require(X, torch.float16, 2, "X")
+    _require(packed, torch.uint8, 2, "packed")
+    _require(scale, torch.float16, 1, "scale")
+    epi = {"none": EPILOGUE_NONE, "geglu": EPILOGUE_GEGLU}[epilogue]
+    M, K = X.shape
+    N = packed.shape[0]
+    if packed.shape[1] * 8 != K * bits or scale.shape[0] != N:
+        raise ValueError("packed/scale shapes do not match X and bits")
+    if bias is not None:
+        _require(bias, torch.float16, 1, "bias")
+        if bias.shape[0] != N:
+            raise ValueError("bias must have N entries")
+    width = N // 2 if epi == EPILOGUE_GEGLU else N
+    Y = torch.empty((M, width), dtype=torch.float16, device=X.device) if out is None else out
+    with _on_device(X):
+        st = raw_gemm_fused(X.data_ptr(), M, packed.data_ptr(), scale.data_ptr(),
+                            0 if bias is None else bias.data_ptr(), N, K, bits, epi, Y.data_ptr(), _stream_ptr(stream))
+    _check(st, "glmq_gemm_fused")
     return Y
 
 

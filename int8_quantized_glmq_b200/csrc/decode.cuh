@@ -39,6 +39,7 @@
 
 #include <cuda.h>
 
+#include "epilogue.cuh"
 #include "glmq_ptx.cuh"
 
 namespace glmq {
@@ -73,6 +74,8 @@ struct DecodeArgs {
   const __half* scale;
   __half* Y;
   float* ws;          // fp32 [M, N] scratch, zero on entry (used when parts > 1)
+  const __half* bias; // fp16 [N] in the natural row order of W, or NULL (epilogue.cuh)
+  int geglu;          // 1: packed rows in the GeGLU layout, Y is [M, N / 2]
   int M;
   int N;
   int K;
@@ -427,14 +430,29 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     // ---- unit epilogue, per warp: rows ra and ra + 8, tokens 8 nb + 2 c (+1)
     const int row_a = t * kDecodeRows + ra;
     const int row_b = row_a + 8;
-    const float sa = (!split && row_a < N) ? __half2float(a.scale[row_a]) : 0.0f;
-    const float sb = (!split && row_b < N) ? __half2float(a.scale[row_b]) : 0.0f;
+    const bool live_a = row_a < N, live_b = row_b < N;
+    const float sa = (!split && live_a) ? __half2float(a.scale[row_a]) : 0.0f;
+    const float sb = (!split && live_b) ? __half2float(a.scale[row_b]) : 0.0f;
+    const float ba = (!split && live_a) ? epilogue_bias(a.bias, a.geglu, row_a, N) : 0.0f;
+    const float bb = (!split && live_b) ? epilogue_bias(a.bias, a.geglu, row_b, N) : 0.0f;
 #pragma unroll
     for (int nb = 0; nb < C::kNB; ++nb) {
 #pragma unroll
       for (int h = 1; h < C::kChains; ++h)
 #pragma unroll
         for (int i = 0; i < 4; ++i) acc[0][nb][i] += acc[h][nb][i];
+      if (!split && a.geglu) {
+        // rows row_a (first GeGLU half) and row_b (second half) of the same output column
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          const int m = 8 * nb + 2 * c + i;
+          if (m < M && live_a) {
+            const float ua = sa * acc[0][nb][i] + ba, ub = sb * acc[0][nb][i + 2] + bb;
+            a.Y[static_cast<long long>(m) * (N >> 1) + geglu_column(row_a)] = __float2half_rn(gelu_exact(ua) * ub);
+          }
+        }
+        continue;
+      }
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int m = 8 * nb + 2 * c + (i & 1);
@@ -442,7 +460,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         if (m < M && row < N) {
           const long long idx = static_cast<long long>(m) * N + row;
           if (split) atomicAdd(a.ws + idx, acc[0][nb][i]);   // result unused: a reduction
-          else a.Y[idx] = __float2half_rn(((i < 2) ? sa : sb) * acc[0][nb][i]);
+          else a.Y[idx] = __float2half_rn(((i < 2) ? sa : sb) * acc[0][nb][i] + ((i < 2) ? ba : bb));
         }
       }
     }

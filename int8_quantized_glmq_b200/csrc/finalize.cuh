@@ -7,6 +7,7 @@
 #include <cuda_fp16.h>
 #include <cstdint>
 
+#include "epilogue.cuh"
 #include "glmq_ptx.cuh"
 
 namespace glmq {
@@ -43,6 +44,45 @@ __global__ void __launch_bounds__(256) decode_finalize_kernel(float* __restrict_
       const float v = __ldcg(ws + idx);
       __stcg(ws + idx, 0.0f);
       Y[idx] = __float2half_rn(sn * v);
+    }
+  }
+}
+
+// The same pass with a fused epilogue (a bias, and/or GeGLU over a GeGLU-layout
+// weight): one thread per output column j of a token row, Y of width N (bias only) or
+// N / 2 (GeGLU). For GeGLU, output j reads packed rows pa = 16 (j / 8) + j % 8 and
+// pa + 8, and returns both scratch entries to zero.
+__global__ void __launch_bounds__(256) finalize_epilogue_kernel(float* __restrict__ ws,
+                                                                const __half* __restrict__ scale,
+                                                                const __half* __restrict__ bias, int geglu,
+                                                                __half* __restrict__ Y, int M, int N) {
+  griddep_wait();   // the partial sums come from the kernel before this one
+  const int width = geglu ? (N >> 1) : N;
+  const int j = blockIdx.x * 256 + threadIdx.x;
+  if (j >= width) return;
+  if (!geglu) {
+    const float sj = __half2float(scale[j]);
+    const float bj = bias ? __half2float(bias[j]) : 0.0f;
+    for (int m = blockIdx.y; m < M; m += gridDim.y) {
+      const long long idx = static_cast<long long>(m) * N + j;
+      const float v = __ldcg(ws + idx);
+      __stcg(ws + idx, 0.0f);
+      Y[idx] = __float2half_rn(sj * v + bj);
+    }
+  } else {
+    const int F = N >> 1;
+    const int pa = 16 * (j >> 3) + (j & 7);
+    const int pb = pa + 8;
+    const float sa = __half2float(scale[pa]), sb = __half2float(scale[pb]);
+    const float ba = bias ? __half2float(bias[j]) : 0.0f;
+    const float bb = bias ? __half2float(bias[F + j]) : 0.0f;
+    for (int m = blockIdx.y; m < M; m += gridDim.y) {
+      const long long row = static_cast<long long>(m) * N;
+      const float va = __ldcg(ws + row + pa), vb = __ldcg(ws + row + pb);
+      __stcg(ws + row + pa, 0.0f);
+      __stcg(ws + row + pb, 0.0f);
+      const float ua = sa * va + ba, ub = sb * vb + bb;
+      Y[static_cast<long long>(m) * F + j] = __float2half_rn(gelu_exact(ua) * ub);
     }
   }
 }

@@ -149,9 +149,11 @@ glmq_status check_gemm(const void* X, int64_t M, const void* packed, const void*
 
 // ---------------------------------------------------------------- quantize
 template <int BITS, int CPT, int T>
-glmq_status launch_quantize_cpt(const void* W, int64_t N, int64_t K, void* packed, void* scale, cudaStream_t s) {
+glmq_status launch_quantize_cpt(const void* W, int64_t N, int64_t K, void* packed, void* scale, int geglu_half,
+                                cudaStream_t s) {
   quantize_kernel<BITS, CPT, T><<<static_cast<unsigned>(N), T, 0, s>>>(
-      static_cast<const __half*>(W), static_cast<int>(K), static_cast<uint8_t*>(packed), static_cast<__half*>(scale));
+      static_cast<const __half*>(W), static_cast<int>(K), static_cast<uint8_t*>(packed), static_cast<__half*>(scale),
+      geglu_half);
   return launched();
 }
 
@@ -159,17 +161,18 @@ glmq_status launch_quantize_cpt(const void* W, int64_t N, int64_t K, void* packe
 // 8192 chunks of 8 values): 256 threads up to 6 chunks each, then 512 or 1024
 // threads with at most 8 chunks each.
 template <int BITS>
-glmq_status launch_quantize(const void* W, int64_t N, int64_t K, void* packed, void* scale, cudaStream_t s) {
+glmq_status launch_quantize(const void* W, int64_t N, int64_t K, void* packed, void* scale, int geglu_half,
+                            cudaStream_t s) {
   const int64_t chunks = K / 8;
-  if (chunks <= 256) return launch_quantize_cpt<BITS, 1, 256>(W, N, K, packed, scale, s);
-  if (chunks <= 512) return launch_quantize_cpt<BITS, 2, 256>(W, N, K, packed, scale, s);
-  if (chunks <= 1024) return launch_quantize_cpt<BITS, 4, 256>(W, N, K, packed, scale, s);
-  if (chunks <= 1536) return launch_quantize_cpt<BITS, 6, 256>(W, N, K, packed, scale, s);
-  if (chunks <= 2048) return launch_quantize_cpt<BITS, 4, 512>(W, N, K, packed, scale, s);
-  if (chunks <= 3072) return launch_quantize_cpt<BITS, 6, 512>(W, N, K, packed, scale, s);
-  if (chunks <= 4096) return launch_quantize_cpt<BITS, 8, 512>(W, N, K, packed, scale, s);
-  if (chunks <= 6144) return launch_quantize_cpt<BITS, 6, 1024>(W, N, K, packed, scale, s);
-  return launch_quantize_cpt<BITS, 8, 1024>(W, N, K, packed, scale, s);
+  if (chunks <= 256) return launch_quantize_cpt<BITS, 1, 256>(W, N, K, packed, scale, geglu_half, s);
+  if (chunks <= 512) return launch_quantize_cpt<BITS, 2, 256>(W, N, K, packed, scale, geglu_half, s);
+  if (chunks <= 1024) return launch_quantize_cpt<BITS, 4, 256>(W, N, K, packed, scale, geglu_half, s);
+  if (chunks <= 1536) return launch_quantize_cpt<BITS, 6, 256>(W, N, K, packed, scale, geglu_half, s);
+  if (chunks <= 2048) return launch_quantize_cpt<BITS, 4, 512>(W, N, K, packed, scale, geglu_half, s);
+  if (chunks <= 3072) return launch_quantize_cpt<BITS, 6, 512>(W, N, K, packed, scale, geglu_half, s);
+  if (chunks <= 4096) return launch_quantize_cpt<BITS, 8, 512>(W, N, K, packed, scale, geglu_half, s);
+  if (chunks <= 6144) return launch_quantize_cpt<BITS, 6, 1024>(W, N, K, packed, scale, geglu_half, s);
+  return launch_quantize_cpt<BITS, 8, 1024>(W, N, K, packed, scale, geglu_half, s);
 }
 
 // ---------------------------------------------------------------- TMA descriptors
@@ -232,6 +235,20 @@ glmq_status decode_scratch(size_t ws_elems, float** out) {
   }
   *out = sc.ws;
   return GLMQ_OK;
+}
+
+// Fused epilogue of a GEMM call (epilogue.cuh): optional bias, optional GeGLU.
+struct Epi {
+  const __half* bias = nullptr;
+  int geglu = 0;
+};
+
+// Launches finalize_epilogue_kernel: one thread per output column of every token row.
+glmq_status launch_finalize_epi(float* ws, const __half* scale, const Epi& e, __half* Y, int M, int N,
+                                cudaStream_t s) {
+  const int width = e.geglu ? N / 2 : N;
+  const dim3 grid(static_cast<unsigned>((width + 255) / 256), static_cast<unsigned>(std::min(M, 65535)));
+  return launch_pdl(finalize_epilogue_kernel, grid, dim3(256), 0, s, ws, scale, e.bias, e.geglu, Y, M, N);
 }
 
 // Launches decode_finalize_kernel: one thread per group of 4 columns (1 when N is not
@@ -310,7 +327,7 @@ bool plan_decode(const DeviceInfo& dev, int N, int K, DecodePlan* pl) {
 
 template <class C>
 glmq_status launch_decode_cfg(const DeviceInfo& dev, const void* X, int M, const void* packed, const void* scale,
-                              int N, int K, void* Y, cudaStream_t s) {
+                              int N, int K, void* Y, cudaStream_t s, const Epi& e = Epi()) {
   DecodePlan pl;
   if (!plan_decode<C>(dev, N, K, &pl)) return GLMQ_ERR_BAD_SHAPE;
   CUtensorMap tw;
@@ -323,6 +340,8 @@ glmq_status launch_decode_cfg(const DeviceInfo& dev, const void* X, int M, const
   a.scale = static_cast<const __half*>(scale);
   a.Y = static_cast<__half*>(Y);
   a.ws = nullptr;
+  a.bias = e.bias;
+  a.geglu = e.geglu;
   a.M = M;
   a.N = N;
   a.K = K;
@@ -335,19 +354,21 @@ glmq_status launch_decode_cfg(const DeviceInfo& dev, const void* X, int M, const
   if ((st = launch_pdl(decode_kernel<C>, dim3(pl.grid), dim3(kDecodeThreads), pl.smem, s, tw, a)) != GLMQ_OK)
     return st;
   if (pl.parts > 1) {
-    if ((st = launch_finalize(a.ws, a.scale, a.Y, M, N, s)) != GLMQ_OK) return st;
+    st = (e.bias || e.geglu) ? launch_finalize_epi(a.ws, a.scale, e, a.Y, M, N, s)
+                             : launch_finalize(a.ws, a.scale, a.Y, M, N, s);
+    if (st != GLMQ_OK) return st;
   }
   return GLMQ_OK;
 }
 
 template <int BITS>
 glmq_status launch_decode(const DeviceInfo& dev, const void* X, int M, const void* packed, const void* scale, int N,
-                          int K, void* Y, cudaStream_t s) {
-  if (M <= 1) return launch_decode_cfg<DecodeCfg<BITS, 1>>(dev, X, M, packed, scale, N, K, Y, s);
-  if (M <= 2) return launch_decode_cfg<DecodeCfg<BITS, 2>>(dev, X, M, packed, scale, N, K, Y, s);
-  if (M <= 4) return launch_decode_cfg<DecodeCfg<BITS, 4>>(dev, X, M, packed, scale, N, K, Y, s);
-  if (M <= 8) return launch_decode_cfg<DecodeCfg<BITS, 8>>(dev, X, M, packed, scale, N, K, Y, s);
-  return launch_decode_cfg<DecodeCfg<BITS, 16>>(dev, X, M, packed, scale, N, K, Y, s);
+                          int K, void* Y, cudaStream_t s, const Epi& e = Epi()) {
+  if (M <= 1) return launch_decode_cfg<DecodeCfg<BITS, 1>>(dev, X, M, packed, scale, N, K, Y, s, e);
+  if (M <= 2) return launch_decode_cfg<DecodeCfg<BITS, 2>>(dev, X, M, packed, scale, N, K, Y, s, e);
+  if (M <= 4) return launch_decode_cfg<DecodeCfg<BITS, 4>>(dev, X, M, packed, scale, N, K, Y, s, e);
+  if (M <= 8) return launch_decode_cfg<DecodeCfg<BITS, 8>>(dev, X, M, packed, scale, N, K, Y, s, e);
+  return launch_decode_cfg<DecodeCfg<BITS, 16>>(dev, X, M, packed, scale, N, K, Y, s, e);
 }
 
 // ---------------------------------------------------------------- prefill
@@ -375,7 +396,7 @@ int plan_parts(int tiles, int num_steps, int min_steps_per_part, int sms) {
 
 template <class C>
 glmq_status launch_prefill_cfg(const DeviceInfo& dev, const void* X, int M, const void* packed, const void* scale,
-                               int N, int K, void* Y, cudaStream_t s) {
+                               int N, int K, void* Y, cudaStream_t s, const Epi& e) {
   CUtensorMap tx, tw;
   glmq_status st = make_map_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, X, K, M, uint64_t(K) * 2, C::BK, C::kBN,
                                CU_TENSOR_MAP_SWIZZLE_128B);
@@ -389,6 +410,8 @@ glmq_status launch_prefill_cfg(const DeviceInfo& dev, const void* X, int M, cons
   a.Y = static_cast<__half*>(Y);
   a.ws = nullptr;
   a.xs = nullptr;
+  a.bias = e.bias;
+  a.geglu = e.geglu;
   a.M = M;
   a.N = N;
   a.K = K;
@@ -408,14 +431,16 @@ glmq_status launch_prefill_cfg(const DeviceInfo& dev, const void* X, int M, cons
   prefill_kernel<C><<<grid, kPrefillThreads, C::SMEM_BYTES, s>>>(tx, tw, a);
   if ((st = launched()) != GLMQ_OK) return st;
   if (a.parts > 1) {
-    if ((st = launch_finalize(a.ws, a.scale, a.Y, M, N, s)) != GLMQ_OK) return st;
+    st = (e.bias || e.geglu) ? launch_finalize_epi(a.ws, a.scale, e, a.Y, M, N, s)
+                             : launch_finalize(a.ws, a.scale, a.Y, M, N, s);
+    if (st != GLMQ_OK) return st;
   }
   return GLMQ_OK;
 }
 
 template <class C>
 glmq_status launch_skinny_cfg(const DeviceInfo& dev, const void* X, int M, const void* packed, const void* scale,
-                              int N, int K, void* Y, cudaStream_t s) {
+                              int N, int K, void* Y, cudaStream_t s, const Epi& e) {
   if (M > C::kBN) return GLMQ_ERR_BAD_SHAPE;   // one token tile: the activation image holds BN rows
   CUtensorMap tw;
   const uint64_t row_bytes = uint64_t(K) / C::KPB;
@@ -429,6 +454,8 @@ glmq_status launch_skinny_cfg(const DeviceInfo& dev, const void* X, int M, const
   uint8_t* xs = nullptr;
   if ((st = skinny_x_scratch(static_cast<size_t>(K / 64) * C::XT_BYTES, &xs)) != GLMQ_OK) return st;
   a.xs = xs;
+  a.bias = e.bias;
+  a.geglu = e.geglu;
   a.M = M;
   a.N = N;
   a.K = K;
@@ -454,20 +481,22 @@ glmq_status launch_skinny_cfg(const DeviceInfo& dev, const void* X, int M, const
   skinny_kernel<C><<<grid, kSkinnyThreads, C::SMEM_BYTES, s>>>(tw, a);
   if ((st = launched()) != GLMQ_OK) return st;
   if (a.parts > 1) {
-    if ((st = launch_finalize(a.ws, a.scale, a.Y, M, N, s)) != GLMQ_OK) return st;
+    st = (e.bias || e.geglu) ? launch_finalize_epi(a.ws, a.scale, e, a.Y, M, N, s)
+                             : launch_finalize(a.ws, a.scale, a.Y, M, N, s);
+    if (st != GLMQ_OK) return st;
   }
   return GLMQ_OK;
 }
 
 template <int BITS>
 glmq_status launch_prefill(const DeviceInfo& dev, const void* X, int M, const void* packed, const void* scale, int N,
-                           int K, void* Y, cudaStream_t s) {
+                           int K, void* Y, cudaStream_t s, const Epi& e = Epi()) {
   // up to 64 tokens: the skinny kernel (wide weight stream, A operand in tensor memory)
-  if (M <= 16) return launch_skinny_cfg<SkinnyCfg<BITS, 16>>(dev, X, M, packed, scale, N, K, Y, s);
-  if (M <= 32) return launch_skinny_cfg<SkinnyCfg<BITS, 32>>(dev, X, M, packed, scale, N, K, Y, s);
-  if (M <= 64) return launch_skinny_cfg<SkinnyCfg<BITS, 64>>(dev, X, M, packed, scale, N, K, Y, s);
-  if (M <= 128) return launch_prefill_cfg<PrefillCfg<BITS, 128>>(dev, X, M, packed, scale, N, K, Y, s);
-  return launch_prefill_cfg<PrefillCfg<BITS, 256>>(dev, X, M, packed, scale, N, K, Y, s);
+  if (M <= 16) return launch_skinny_cfg<SkinnyCfg<BITS, 16>>(dev, X, M, packed, scale, N, K, Y, s, e);
+  if (M <= 32) return launch_skinny_cfg<SkinnyCfg<BITS, 32>>(dev, X, M, packed, scale, N, K, Y, s, e);
+  if (M <= 64) return launch_skinny_cfg<SkinnyCfg<BITS, 64>>(dev, X, M, packed, scale, N, K, Y, s, e);
+  if (M <= 128) return launch_prefill_cfg<PrefillCfg<BITS, 128>>(dev, X, M, packed, scale, N, K, Y, s, e);
+  return launch_prefill_cfg<PrefillCfg<BITS, 256>>(dev, X, M, packed, scale, N, K, Y, s, e);
 }
 
 // ---------------------------------------------------------------- decode without allocation
@@ -519,6 +548,8 @@ glmq_status launch_decode_noalloc_cfg(const DeviceInfo& dev, const void* X, int 
   a.parts = pl.parts;
   a.tiles = pl.tiles;
   a.units = pl.units;
+  a.bias = nullptr;
+  a.geglu = 0;
   cudaError_t e;
   if (pl.parts > 1) {
     if ((st = noalloc_scratch(&a.ws)) != GLMQ_OK) return st;
@@ -548,7 +579,7 @@ glmq_status launch_decode_noalloc(const DeviceInfo& dev, const void* X, int M, c
 enum class Route { kAuto, kDecode, kPrefill };
 
 glmq_status gemm_entry(Route route, const void* X, int64_t M, const void* packed, const void* scale, int64_t N,
-                       int64_t K, int bits, void* Y, void* stream) {
+                       int64_t K, int bits, void* Y, void* stream, const Epi& e = Epi()) {
   glmq_status st = check_gemm(X, M, packed, scale, N, K, bits, Y);
   if (st != GLMQ_OK) return st;
   if (route == Route::kDecode && M > GLMQ_DECODE_MAX_M) return GLMQ_ERR_BAD_SHAPE;
@@ -559,11 +590,27 @@ glmq_status gemm_entry(Route route, const void* X, int64_t M, const void* packed
   const bool decode = route == Route::kDecode || (route == Route::kAuto && M <= GLMQ_DECODE_AUTO_MAX_M);
   const int m = static_cast<int>(M), n = static_cast<int>(N), k = static_cast<int>(K);
   if (decode) {
-    return bits == 4 ? launch_decode<4>(*dev, X, m, packed, scale, n, k, Y, s)
-                     : launch_decode<8>(*dev, X, m, packed, scale, n, k, Y, s);
+    return bits == 4 ? launch_decode<4>(*dev, X, m, packed, scale, n, k, Y, s, e)
+                     : launch_decode<8>(*dev, X, m, packed, scale, n, k, Y, s, e);
   }
-  return bits == 4 ? launch_prefill<4>(*dev, X, m, packed, scale, n, k, Y, s)
-                   : launch_prefill<8>(*dev, X, m, packed, scale, n, k, Y, s);
+  return bits == 4 ? launch_prefill<4>(*dev, X, m, packed, scale, n, k, Y, s, e)
+                   : launch_prefill<8>(*dev, X, m, packed, scale, n, k, Y, s, e);
+}
+
+glmq_status quantize_entry(const void* W, int64_t N, int64_t K, int bits, void* packed, void* scale, void* stream,
+                           bool geglu) {
+  glmq_status st = check_common(N, K, bits);
+  if (st != GLMQ_OK) return st;
+  if (geglu && (N % 16) != 0) return GLMQ_ERR_BAD_SHAPE;
+  if (N == 0) return GLMQ_OK;
+  if (!W || !packed || !scale) return GLMQ_ERR_NULL_POINTER;
+  if (!aligned16(W) || !aligned16(packed) || !aligned16(scale)) return GLMQ_ERR_MISALIGNED;
+  const DeviceInfo* dev = nullptr;
+  if ((st = current_device(&dev)) != GLMQ_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int half = geglu ? static_cast<int>(N / 2) : 0;
+  return bits == 4 ? launch_quantize<4>(W, N, K, packed, scale, half, s)
+                   : launch_quantize<8>(W, N, K, packed, scale, half, s);
 }
 
 }  // namespace
@@ -578,15 +625,12 @@ size_t glmq_packed_bytes(int64_t N, int64_t K, int bits) {
 }
 
 glmq_status glmq_quantize(const void* W, int64_t N, int64_t K, int bits, void* packed, void* scale, void* stream) {
-  glmq_status st = check_common(N, K, bits);
-  if (st != GLMQ_OK) return st;
-  if (N == 0) return GLMQ_OK;
-  if (!W || !packed || !scale) return GLMQ_ERR_NULL_POINTER;
-  if (!aligned16(W) || !aligned16(packed) || !aligned16(scale)) return GLMQ_ERR_MISALIGNED;
-  const DeviceInfo* dev = nullptr;
-  if ((st = current_device(&dev)) != GLMQ_OK) return st;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return bits == 4 ? launch_quantize<4>(W, N, K, packed, scale, s) : launch_quantize<8>(W, N, K, packed, scale, s);
+  return quantize_entry(W, N, K, bits, packed, scale, stream, false);
+}
+
+glmq_status glmq_quantize_geglu(const void* W, int64_t N, int64_t K, int bits, void* packed, void* scale,
+                                void* stream) {
+  return quantize_entry(W, N, K, bits, packed, scale, stream, true);
 }
 
 glmq_status glmq_gemm(const void* X, int64_t M, const void* packed, const void* scale, int64_t N, int64_t K, int bits,
@@ -602,6 +646,18 @@ glmq_status glmq_gemm_decode(const void* X, int64_t M, const void* packed, const
 glmq_status glmq_gemm_prefill(const void* X, int64_t M, const void* packed, const void* scale, int64_t N, int64_t K,
                               int bits, void* Y, void* stream) {
   return gemm_entry(Route::kPrefill, X, M, packed, scale, N, K, bits, Y, stream);
+}
+
+glmq_status glmq_gemm_fused(const void* X, int64_t M, const void* packed, const void* scale, const void* bias,
+                            int64_t N, int64_t K, int bits, int epilogue, void* Y, void* stream) {
+  if (epilogue != GLMQ_EPILOGUE_NONE && epilogue != GLMQ_EPILOGUE_GEGLU) return GLMQ_ERR_BAD_SHAPE;
+  const bool geglu = epilogue == GLMQ_EPILOGUE_GEGLU;
+  if (geglu && (N % 16) != 0) return GLMQ_ERR_BAD_SHAPE;
+  if (bias && (reinterpret_cast<uintptr_t>(bias) & 1u) != 0) return GLMQ_ERR_MISALIGNED;
+  Epi e;
+  e.bias = static_cast<const __half*>(bias);
+  e.geglu = geglu ? 1 : 0;
+  return gemm_entry(Route::kAuto, X, M, packed, scale, N, K, bits, Y, stream, e);
 }
 
 glmq_status glmq_gemm_decode_noalloc(const void* X, int64_t M, const void* packed, const void* scale, int64_t N,

@@ -41,6 +41,7 @@
 
 #include <cuda.h>
 
+#include "epilogue.cuh"
 #include "glmq_ptx.cuh"
 
 namespace glmq {
@@ -83,6 +84,8 @@ struct PrefillArgs {
   __half* Y;
   float* ws;      // fp32 [M, N] scratch, zero on entry (used when parts > 1)
   const uint8_t* xs;  // skinny kernel only: activation tiles pre-swizzled by skinny_pack_x_kernel
+  const __half* bias; // fp16 [N] in the natural row order of W, or NULL (epilogue.cuh)
+  int geglu;          // 1: packed rows in the GeGLU layout, Y is [M, N / 2]
   int M;
   int N;
   int K;
@@ -92,6 +95,33 @@ struct PrefillArgs {
   int kbp;        // K blocks per part
   int units;      // tiles * parts
 };
+
+// Epilogue of one TMEM lane (packed weight row n) for tokens m0 .. m0 + mend - 1,
+// called by all 32 lanes of an epilogue warp (the GeGLU pair of row n, n % 16 < 8,
+// is row n + 8, 8 lanes up in the same warp). Lanes with n >= N pass s = 0.
+template <int kChunk>
+__device__ __forceinline__ void tmem_lane_epilogue(const PrefillArgs& a, int n, float s, const uint32_t (&v)[32],
+                                                   int m0, int mend) {
+  const bool live = n < a.N;
+  const float b = live ? epilogue_bias(a.bias, a.geglu, n, a.N) : 0.0f;
+  if (!a.geglu) {
+    if (!live) return;
+    __half* yp = a.Y + static_cast<long long>(m0) * a.N + n;
+#pragma unroll
+    for (int j = 0; j < kChunk; ++j)
+      if (j < mend) yp[static_cast<long long>(j) * a.N] = __float2half_rn(s * __uint_as_float(v[j]) + b);
+    return;
+  }
+  const int F = a.N >> 1;
+  const bool first_half = live && (n & 15) < 8;
+  __half* yp = a.Y + static_cast<long long>(m0) * F + geglu_column(n);
+#pragma unroll
+  for (int j = 0; j < kChunk; ++j) {
+    const float u = s * __uint_as_float(v[j]) + b;
+    const float ub = __shfl_down_sync(0xffffffffu, u, 8);
+    if (first_half && j < mend) yp[static_cast<long long>(j) * F] = __float2half_rn(gelu_exact(u) * ub);
+  }
+}
 
 // ---------------------------------------------------------------- tcgen05 / TMA wrappers
 __device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t smem_addr) {
@@ -402,19 +432,16 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         uint32_t v[32];
         if constexpr (kChunk == 16) tmem_ld16(t_row + cb * kChunk, v);
         else tmem_ld32(t_row + cb * kChunk, v);
-        if (n < a.N) {
-          const int mend = min(kChunk, a.M - m0);
-          if (split) {
+        const int mend = min(kChunk, a.M - m0);
+        if (split) {
+          if (n < a.N) {
             float* wp = a.ws + static_cast<long long>(m0) * a.N + n;
 #pragma unroll
             for (int j = 0; j < kChunk; ++j)
               if (j < mend) atomicAdd(wp + static_cast<long long>(j) * a.N, __uint_as_float(v[j]));
-          } else {
-            __half* yp = a.Y + static_cast<long long>(m0) * a.N + n;
-#pragma unroll
-            for (int j = 0; j < kChunk; ++j)
-              if (j < mend) yp[static_cast<long long>(j) * a.N] = __float2half_rn(s * __uint_as_float(v[j]));
           }
+        } else {
+          tmem_lane_epilogue<kChunk>(a, n, s, v, m0, mend);
         }
       }
       tc_fence_before();

@@ -28,6 +28,7 @@
 // and are exact in fp32.
 #pragma once
 
+#include "epilogue.cuh"
 #include "glmq_ptx.cuh"
 
 namespace glmq {
@@ -83,13 +84,17 @@ __device__ __forceinline__ void chunk_codes(const uint4 v, float sf, float r, bo
 }
 
 // One CTA of T threads per row; each thread holds CPT 16-byte chunks of the row.
+// geglu_half = F > 0 writes the GeGLU row layout (output row 16g + r from input row
+// 8g + r, r < 8, or F + 8g + r - 8); 0 keeps the natural order.
 template <int BITS, int CPT, int T>
 __global__ void __launch_bounds__(T) quantize_kernel(const __half* __restrict__ W, int K,
-                                                     uint8_t* __restrict__ packed, __half* __restrict__ scale) {
+                                                     uint8_t* __restrict__ packed, __half* __restrict__ scale,
+                                                     int geglu_half) {
   constexpr int D = (1 << (BITS - 1)) - 1;
   const long long row = blockIdx.x;
+  const long long src_row = geglu_half > 0 ? geglu_natural_row(static_cast<int>(row), geglu_half) : row;
   const int nchunks = K >> 3;
-  const uint4* src = reinterpret_cast<const uint4*>(W + row * static_cast<long long>(K));
+  const uint4* src = reinterpret_cast<const uint4*>(W + src_row * static_cast<long long>(K));
 
   uint4 v[CPT];
   uint32_t m = 0;

@@ -341,19 +341,16 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
         uint32_t v[32];
         if constexpr (kChunk == 16) tmem_ld16(t_row + cb * kChunk, v);
         else tmem_ld32(t_row + cb * kChunk, v);
-        if (n < a.N) {
-          const int mend = min(kChunk, a.M - m0);
-          if (split) {
+        const int mend = min(kChunk, a.M - m0);
+        if (split) {
+          if (n < a.N) {
             float* wp = a.ws + static_cast<long long>(m0) * a.N + n;
 #pragma unroll
             for (int jj = 0; jj < kChunk; ++jj)
               if (jj < mend) atomicAdd(wp + static_cast<long long>(jj) * a.N, __uint_as_float(v[jj]));
-          } else {
-            __half* yp = a.Y + static_cast<long long>(m0) * a.N + n;
-#pragma unroll
-            for (int jj = 0; jj < kChunk; ++jj)
-              if (jj < mend) yp[static_cast<long long>(jj) * a.N] = __float2half_rn(s * __uint_as_float(v[jj]));
           }
+        } else {
+          tmem_lane_epilogue<kChunk>(a, n, s, v, m0, mend);
         }
       }
       tc_fence_before();

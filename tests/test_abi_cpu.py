@@ -112,3 +112,16 @@ def test_kernel_launch_counter_ignores_rejected_calls():
     assert B.raw_gemm(ALIGNED, 4, ALIGNED, ALIGNED, 8, 64, 3, ALIGNED, 0, "auto") == B.ERR_BAD_BITS
     assert B.raw_gemm(0, 0, ALIGNED, ALIGNED, 8, 64, 4, 0, 0, "auto") == B.OK     # empty: nothing enqueued
     assert glmq.kernel_launches() == n0
+
+
+def test_fused_entry_points_validate_before_device_work():
+    g = lambda **kw: B.raw_gemm_fused(kw.get("X", ALIGNED), kw.get("M", 4), ALIGNED, ALIGNED, kw.get("bias", 0),
+                                      kw.get("N", 32), 64, 4, kw.get("epi", B.EPILOGUE_NONE), ALIGNED, 0)
+    assert g(epi=7) == B.ERR_BAD_SHAPE
+    assert g(epi=B.EPILOGUE_GEGLU, N=24) == B.ERR_BAD_SHAPE       # GeGLU needs N % 16 == 0
+    assert g(bias=ALIGNED + 1) == B.ERR_MISALIGNED
+    assert g(X=0) == B.ERR_NULL_POINTER
+    assert g(M=0, X=0) == B.OK
+    assert B.raw_quantize_geglu(ALIGNED, 40, 64, 4, ALIGNED, ALIGNED) == B.ERR_BAD_SHAPE
+    assert B.raw_quantize_geglu(ALIGNED, 48, 64, 3, ALIGNED, ALIGNED) == B.ERR_BAD_BITS
+    assert B.raw_quantize_geglu(0, 0, 64, 4, 0, 0) == B.OK

@@ -17,4 +17,5 @@ from .synthetic import (  # noqa: F401
     decode_activations,
     prefill_activations,
     outlier_positions,
+    outlier_activations,
 )

@@ -21,3 +21,14 @@ from .glmq_epilogue import (  # noqa: F401,E402
     geglu_row_order,
     quantize_linear_geglu,
 )
+from .glmq_zeropoint import (  # noqa: F401,E402
+    zp_range,
+    zp_scale,
+    zp_zero,
+    zp_codes,
+    pack_u4,
+    unpack_u4,
+    quantize_linear_zp,
+    dequantize_zp,
+    linear_forward_zp,
+)

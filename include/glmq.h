@@ -156,6 +156,31 @@ GLMQ_API glmq_status glmq_gemm_fused(const void* X, int64_t M, const void* packe
                                      void* stream);
 
 /*
+ * Zero-point (asymmetric) INT4 quantization (GLM-130B paper card, "Pitfalls": a
+ * zero-point INT4 quantizer scored better on LAMBADA than the absmax one, which the
+ * authors kept as cheaper; the card gives no formula). Per output row:
+ *   lo = min(0, min_k W), hi = max(0, max_k W)          (fp16 values)
+ *   s  = fp16_rn( fl32( fl32(hi - lo) / 15 ) )
+ *   z  = clamp( rint( fl32(-lo / s) ), 0, 15 )           (0 where s == 0)
+ *   q  = clamp( rint( fl32(w / s) ) + z, 0, 15 )         (0 where s == 0), unsigned
+ *   W   in : fp16 [N, K]
+ *   packed out: uint8 [N, K/2], two unsigned codes per byte, low nibble = even k
+ *   scale  out: fp16 [N];  zero out: uint8 [N]
+ * Limits and errors as glmq_quantize (bits is 4). Results are bit-for-bit reproducible.
+ */
+GLMQ_API glmq_status glmq_quantize_zp(const void* W, int64_t N, int64_t K, void* packed, void* scale, void* zero,
+                                      void* stream);
+
+/*
+ * Dequantizing linear layer for zero-point codes from glmq_quantize_zp:
+ *   Y[m,n] = fp16_rn( s[n] * sum_k X[m,k] * (q[n,k] - z[n]) ), fp32 accumulation.
+ * Arguments, dispatch, scratch and errors as glmq_gemm with bits = 4; zero must not be
+ * NULL (GLMQ_ERR_NULL_POINTER).
+ */
+GLMQ_API glmq_status glmq_gemm_zp(const void* X, int64_t M, const void* packed, const void* scale, const void* zero,
+                                  int64_t N, int64_t K, void* Y, void* stream);
+
+/*
  * glmq_gemm_decode without any device allocation (the paper has no counterpart:
  * this is a deployment variant of the decode kernel).
  *

@@ -12,6 +12,7 @@ from ._binding import (  # noqa: F401
     abi_version,
     gemm,
     gemm_fused,
+    gemm_zp,
     gemm_decode,
     gemm_prefill,
     kernel_launches,
@@ -19,6 +20,7 @@ from ._binding import (  # noqa: F401
     lib,
     packed_bytes,
     quantize,
+    quantize_zp,
     raw_gemm,
     raw_quantize,
     status_string,

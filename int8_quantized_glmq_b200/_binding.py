@@ -39,6 +39,8 @@ SIGNATURES = {
     "glmq_packed_bytes": (ctypes.c_size_t, [_c_int64, _c_int64, ctypes.c_int]),
     "glmq_quantize": (ctypes.c_int, [_vp, _c_int64, _c_int64, ctypes.c_int, _vp, _vp, _vp]),
     "glmq_quantize_geglu": (ctypes.c_int, [_vp, _c_int64, _c_int64, ctypes.c_int, _vp, _vp, _vp]),
+    "glmq_quantize_zp": (ctypes.c_int, [_vp, _c_int64, _c_int64, _vp, _vp, _vp, _vp]),
+    "glmq_gemm_zp": (ctypes.c_int, [_vp, _c_int64, _vp, _vp, _vp, _c_int64, _c_int64, _vp, _vp]),
     "glmq_gemm_fused": (ctypes.c_int, [_vp, _c_int64, _vp, _vp, _vp, _c_int64, _c_int64, ctypes.c_int, ctypes.c_int,
                                        _vp, _vp]),
     "glmq_gemm": (ctypes.c_int, [_vp, _c_int64, _vp, _vp, _c_int64, _c_int64, ctypes.c_int, _vp, _vp]),
@@ -109,6 +111,14 @@ def raw_quantize(W: int, N: int, K: int, bits: int, packed: int, scale: int, str
 
 def raw_quantize_geglu(W: int, N: int, K: int, bits: int, packed: int, scale: int, stream: int = 0) -> int:
     return lib().glmq_quantize_geglu(W, N, K, bits, packed, scale, stream)
+
+
+def raw_quantize_zp(W: int, N: int, K: int, packed: int, scale: int, zero: int, stream: int = 0) -> int:
+    return lib().glmq_quantize_zp(W, N, K, packed, scale, zero, stream)
+
+
+def raw_gemm_zp(X: int, M: int, packed: int, scale: int, zero: int, N: int, K: int, Y: int, stream: int = 0) -> int:
+    return lib().glmq_gemm_zp(X, M, packed, scale, zero, N, K, Y, stream)
 
 
 def raw_gemm_fused(X: int, M: int, packed: int, scale: int, bias: int, N: int, K: int, bits: int, epilogue: int,
@@ -237,6 +247,43 @@ def gemm_fused(X, packed, scale, bits: int = 4, bias=None, epilogue: str = "none
         st = raw_gemm_fused(X.data_ptr(), M, packed.data_ptr(), scale.data_ptr(),
                             0 if bias is None else bias.data_ptr(), N, K, bits, epi, Y.data_ptr(), _stream_ptr(stream))
     _check(st, "glmq_gemm_fused")
+    return Y
+
+
+def quantize_zp(W, stream=None, out=None):
+    """Zero-point INT4 quantization of fp16 W[N, K] -> (packed uint8 [N, K/2], scale fp16 [N], zero uint8 [N])."""
+    torch = _torch()
+    _require(W, torch.float16, 2, "W")
+    N, K = W.shape
+    if out is None:
+        packed = torch.empty((N, K // 2), dtype=torch.uint8, device=W.device)
+        scale = torch.empty((N,), dtype=torch.float16, device=W.device)
+        zero = torch.empty((N,), dtype=torch.uint8, device=W.device)
+    else:
+        packed, scale, zero = out
+    with _on_device(W):
+        st = raw_quantize_zp(W.data_ptr(), N, K, packed.data_ptr(), scale.data_ptr(), zero.data_ptr(),
+                             _stream_ptr(stream))
+    _check(st, "glmq_quantize_zp")
+    return packed, scale, zero
+
+
+def gemm_zp(X, packed, scale, zero, stream=None, out=None):
+    """Y[M, N] = fp16(s[n] * sum_k X (q - z[n])) for codes from :func:`quantize_zp`."""
+    torch = _torch()
+    _require(X, torch.float16, 2, "X")
+    _require(packed, torch.uint8, 2, "packed")
+    _require(scale, torch.float16, 1, "scale")
+    _require(zero, torch.uint8, 1, "zero")
+    M, K = X.shape
+    N = packed.shape[0]
+    if packed.shape[1] * 2 != K or scale.shape[0] != N or zero.shape[0] != N:
+        raise ValueError("packed/scale/zero shapes do not match X")
+    Y = torch.empty((M, N), dtype=torch.float16, device=X.device) if out is None else out
+    with _on_device(X):
+        st = raw_gemm_zp(X.data_ptr(), M, packed.data_ptr(), scale.data_ptr(), zero.data_ptr(), N, K, Y.data_ptr(),
+                         _stream_ptr(stream))
+    _check(st, "glmq_gemm_zp")
     return Y
 
 

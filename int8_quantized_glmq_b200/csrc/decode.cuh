@@ -53,9 +53,17 @@ constexpr int kDecodeStageBytes = kDecodeRows * kDecodeSegB;          // 32 KB: 
 // ring + barriers; the activation slice follows
 constexpr int kDecodeFixedSmem = kDecodeStages * kDecodeStageBytes + 256;
 
-template <int BITS, int MP, int CHAINS = 2>
+template <int BITS, int MP, int CHAINS = 2, int ZP = 0>
 struct DecodeCfg {
   static_assert(CHAINS == 2 || CHAINS == 4, "accumulator chains");
+  static_assert(ZP == 0 || BITS == 4, "zero-point codes are INT4");
+  static constexpr int kZP = ZP;   // 1: zero-point INT4 codes (unsigned, per-row zero point)
+  // biased dequantization: low nibbles give the fp16 integer kLowBase + (value), high
+  // nibbles kHighBase + 16 (value); symmetric codes carry their own +8 offset in the XOR
+  static constexpr uint32_t kXorLo = ZP ? 0x64006400u : 0x64086408u;
+  static constexpr uint32_t kXorHi = ZP ? 0x64006400u : 0x64806480u;
+  static constexpr float kLowBias = ZP ? 1024.0f : 1032.0f;    // per unit of x in a low-nibble slot
+  static constexpr float kHighBias = ZP ? 1024.0f : 1152.0f;   // per unit of x / 16 in a high-nibble slot
   static constexpr int kBits = BITS;
   static constexpr int kMP = MP;                    // token capacity of the activation layout (M <= MP)
   static constexpr int kNB = (MP + 7) / 8;          // n8 token blocks of the MMA
@@ -74,6 +82,7 @@ struct DecodeArgs {
   const __half* scale;
   __half* Y;
   float* ws;          // fp32 [M, N] scratch, zero on entry (used when parts > 1)
+  const uint8_t* zero;  // zero-point codes: uint8 [N] per-row zero point, else NULL
   const __half* bias; // fp16 [N] in the natural row order of W, or NULL (epilogue.cuh)
   int geglu;          // 1: packed rows in the GeGLU layout, Y is [M, N / 2]
   int M;
@@ -112,12 +121,13 @@ __device__ __forceinline__ void dequant_int4_word(uint32_t w, uint32_t (&p)[4]) 
 // for low-nibble slots and x / 16 for high-nibble slots, so every product is
 // q * x + (a bias depending only on x), and the accumulated bias is removed per
 // segment (see decode_segment). Four LOP3 and one shift per 8 codes.
+template <uint32_t XLO, uint32_t XHI>
 __device__ __forceinline__ void dequant_int4_word_biased(uint32_t w, uint32_t (&p)[4]) {
   const uint32_t w8 = w >> 8;
-  p[0] = lop3_and_xor(w, 0x000F000Fu, 0x64086408u);
-  p[1] = lop3_and_xor(w, 0x00F000F0u, 0x64806480u);
-  p[2] = lop3_and_xor(w8, 0x000F000Fu, 0x64086408u);
-  p[3] = lop3_and_xor(w8, 0x00F000F0u, 0x64806480u);
+  p[0] = lop3_and_xor(w, 0x000F000Fu, XLO);
+  p[1] = lop3_and_xor(w, 0x00F000F0u, XHI);
+  p[2] = lop3_and_xor(w8, 0x000F000Fu, XLO);
+  p[3] = lop3_and_xor(w8, 0x00F000F0u, XHI);
 }
 
 // INT8: one word (4 codes, k = 0..3) -> half2 pairs (0,1), (2,3).
@@ -180,8 +190,8 @@ __device__ __forceinline__ void decode_segment(uint32_t box, uint32_t xseg, uint
         if (!kTail || valid) bf[nb] = lds_v4(xseg + (nb ? xlane1 : xlane0) + j * kJStride);
       }
       uint32_t pa[4], pb[4];
-      dequant_int4_word_biased(wa[j], pa);
-      dequant_int4_word_biased(wb[j], pb);
+      dequant_int4_word_biased<C::kXorLo, C::kXorHi>(wa[j], pa);
+      dequant_int4_word_biased<C::kXorLo, C::kXorHi>(wb[j], pb);
       const int h0 = (C::kChains == 4) ? 2 * (j & 1) : 0;
 #pragma unroll
       for (int nb = 0; nb < C::kNB; ++nb) {
@@ -282,8 +292,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kDecodeStages * kDecodeStageBytes);
   uint64_t* empty = full + kDecodeStages;
   uint8_t* xbuf = smem + kDecodeFixedSmem;
-  // INT4 only: per (segment, token) bias of the biased dequantization, after the activation slice
+  // INT4 only: per (segment, token) bias of the biased dequantization, after the activation slice;
+  // zero-point codes: then per-token sums of x over the part
   float* bias_s = reinterpret_cast<float*>(xbuf + 2 * C::kMP * a.KPP);
+  float* sx_s = bias_s + (a.KPP / C::SEGK) * 16;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -388,11 +400,35 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
             const float2 fy = __half22float2(*reinterpret_cast<const __half2*>(&o.y));
             const float2 fz = __half22float2(*reinterpret_cast<const __half2*>(&o.z));
             const float2 fw = __half22float2(*reinterpret_cast<const __half2*>(&o.w));
-            bias = 1032.0f * ((fx.x + fx.y) + (fz.x + fz.y)) + 1152.0f * ((fy.x + fy.y) + (fw.x + fw.y));
+            bias = C::kLowBias * ((fx.x + fx.y) + (fz.x + fz.y)) + C::kHighBias * ((fy.x + fy.y) + (fw.x + fw.y));
           }
 #pragma unroll
           for (int off = 16; off > 0; off >>= 1) bias += __shfl_xor_sync(0xffffffffu, bias, off);
           if (lane == 0) bias_s[sg * 16 + n] = bias;
+        }
+        if constexpr (C::kZP) {
+          // per-token sum of x over the part, for the zero-point term z[n] * sum_k x[m,k]
+          // (high-nibble slots hold x / 16)
+          const int units = pseg * C::XU * 4;
+          for (int n = warp; n < M; n += kDecodeConsumerWarps) {
+            float sx = 0.0f;
+            for (int i = lane; i < units; i += 32) {
+              const int sg = i / (C::XU * 4);
+              const int rem = i - sg * (C::XU * 4);
+              const int jj = rem >> 2, cc = rem & 3;
+              if (sg * C::SEGK + cc * C::TK + jj * 8 < plen) {
+                const uint4 o = *reinterpret_cast<const uint4*>(xbuf + 16u * x_unit<C>(sg, jj, n, cc));
+                const float2 fx = __half22float2(*reinterpret_cast<const __half2*>(&o.x));
+                const float2 fy = __half22float2(*reinterpret_cast<const __half2*>(&o.y));
+                const float2 fz = __half22float2(*reinterpret_cast<const __half2*>(&o.z));
+                const float2 fw = __half22float2(*reinterpret_cast<const __half2*>(&o.w));
+                sx += ((fx.x + fx.y) + (fz.x + fz.y)) + 16.0f * ((fy.x + fy.y) + (fw.x + fw.y));
+              }
+            }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) sx += __shfl_xor_sync(0xffffffffu, sx, off);
+            if (lane == 0) sx_s[n] = sx;
+          }
         }
       }
       cur_part = p;
@@ -434,6 +470,11 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     const float sa = (!split && live_a) ? __half2float(a.scale[row_a]) : 0.0f;
     const float sb = (!split && live_b) ? __half2float(a.scale[row_b]) : 0.0f;
     const float ba = (!split && live_a) ? epilogue_bias(a.bias, a.geglu, row_a, N) : 0.0f;
+    float za = 0.0f, zb = 0.0f;
+    if constexpr (C::kZP) {
+      za = live_a ? static_cast<float>(a.zero[row_a]) : 0.0f;
+      zb = live_b ? static_cast<float>(a.zero[row_b]) : 0.0f;
+    }
     const float bb = (!split && live_b) ? epilogue_bias(a.bias, a.geglu, row_b, N) : 0.0f;
 #pragma unroll
     for (int nb = 0; nb < C::kNB; ++nb) {
@@ -441,6 +482,14 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       for (int h = 1; h < C::kChains; ++h)
 #pragma unroll
         for (int i = 0; i < 4; ++i) acc[0][nb][i] += acc[h][nb][i];
+      if constexpr (C::kZP) {
+        // the MMAs saw the unsigned codes: remove z[row] * sum_k x[m,k] (this part's k)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int m = 8 * nb + 2 * c + (i & 1);
+          if (m < M) acc[0][nb][i] -= ((i < 2) ? za : zb) * sx_s[m];
+        }
+      }
       if (!split && a.geglu) {
         // rows row_a (first GeGLU half) and row_b (second half) of the same output column
 #pragma unroll

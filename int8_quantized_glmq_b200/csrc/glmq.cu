@@ -175,6 +175,30 @@ glmq_status launch_quantize(const void* W, int64_t N, int64_t K, void* packed, v
   return launch_quantize_cpt<BITS, 8, 1024>(W, N, K, packed, scale, geglu_half, s);
 }
 
+template <int CPT, int T>
+glmq_status launch_quantize_zp_cpt(const void* W, int64_t N, int64_t K, void* packed, void* scale, void* zero,
+                                   cudaStream_t s) {
+  quantize_zp_kernel<CPT, T><<<static_cast<unsigned>(N), T, 0, s>>>(
+      static_cast<const __half*>(W), static_cast<int>(K), static_cast<uint8_t*>(packed), static_cast<__half*>(scale),
+      static_cast<uint8_t*>(zero));
+  return launched();
+}
+
+// Same block-size choice as launch_quantize.
+glmq_status launch_quantize_zp(const void* W, int64_t N, int64_t K, void* packed, void* scale, void* zero,
+                               cudaStream_t s) {
+  const int64_t chunks = K / 8;
+  if (chunks <= 256) return launch_quantize_zp_cpt<1, 256>(W, N, K, packed, scale, zero, s);
+  if (chunks <= 512) return launch_quantize_zp_cpt<2, 256>(W, N, K, packed, scale, zero, s);
+  if (chunks <= 1024) return launch_quantize_zp_cpt<4, 256>(W, N, K, packed, scale, zero, s);
+  if (chunks <= 1536) return launch_quantize_zp_cpt<6, 256>(W, N, K, packed, scale, zero, s);
+  if (chunks <= 2048) return launch_quantize_zp_cpt<4, 512>(W, N, K, packed, scale, zero, s);
+  if (chunks <= 3072) return launch_quantize_zp_cpt<6, 512>(W, N, K, packed, scale, zero, s);
+  if (chunks <= 4096) return launch_quantize_zp_cpt<8, 512>(W, N, K, packed, scale, zero, s);
+  if (chunks <= 6144) return launch_quantize_zp_cpt<6, 1024>(W, N, K, packed, scale, zero, s);
+  return launch_quantize_zp_cpt<8, 1024>(W, N, K, packed, scale, zero, s);
+}
+
 // ---------------------------------------------------------------- TMA descriptors
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -241,6 +265,7 @@ glmq_status decode_scratch(size_t ws_elems, float** out) {
 struct Epi {
   const __half* bias = nullptr;
   int geglu = 0;
+  const uint8_t* zero = nullptr;   // zero-point INT4 codes: per-row zero points
 };
 
 // Launches finalize_epilogue_kernel: one thread per output column of every token row.
@@ -293,7 +318,7 @@ struct DecodePlan {
 // sums through the scratch buffer and a finalize launch).
 template <class C>
 bool plan_decode(const DeviceInfo& dev, int N, int K, DecodePlan* pl) {
-  const int x_budget = dev.smem_optin - kDecodeFixedSmem - 1024;
+  const int x_budget = dev.smem_optin - kDecodeFixedSmem - 1024 - 64;   // 64: per-token sums (zero point)
   const int stages = (K + C::SK - 1) / C::SK;
   const int per_stage = 2 * C::kMP * C::SK + ((C::kBits == 4) ? 16 * 4 : 0);
   const int max_spp = x_budget / per_stage;
@@ -321,7 +346,7 @@ bool plan_decode(const DeviceInfo& dev, int N, int K, DecodePlan* pl) {
   pl->tiles = static_cast<int>(tiles);
   pl->units = pl->parts * pl->tiles;
   pl->grid = pl->units < dev.sms ? pl->units : dev.sms;
-  pl->smem = kDecodeFixedSmem + 1024 + spp * per_stage;
+  pl->smem = kDecodeFixedSmem + 1024 + spp * per_stage + 64;
   return pl->smem <= dev.smem_optin;
 }
 
@@ -340,6 +365,7 @@ glmq_status launch_decode_cfg(const DeviceInfo& dev, const void* X, int M, const
   a.scale = static_cast<const __half*>(scale);
   a.Y = static_cast<__half*>(Y);
   a.ws = nullptr;
+  a.zero = e.zero;
   a.bias = e.bias;
   a.geglu = e.geglu;
   a.M = M;
@@ -361,14 +387,14 @@ glmq_status launch_decode_cfg(const DeviceInfo& dev, const void* X, int M, const
   return GLMQ_OK;
 }
 
-template <int BITS>
+template <int BITS, int ZP = 0>
 glmq_status launch_decode(const DeviceInfo& dev, const void* X, int M, const void* packed, const void* scale, int N,
                           int K, void* Y, cudaStream_t s, const Epi& e = Epi()) {
-  if (M <= 1) return launch_decode_cfg<DecodeCfg<BITS, 1>>(dev, X, M, packed, scale, N, K, Y, s, e);
-  if (M <= 2) return launch_decode_cfg<DecodeCfg<BITS, 2>>(dev, X, M, packed, scale, N, K, Y, s, e);
-  if (M <= 4) return launch_decode_cfg<DecodeCfg<BITS, 4>>(dev, X, M, packed, scale, N, K, Y, s, e);
-  if (M <= 8) return launch_decode_cfg<DecodeCfg<BITS, 8>>(dev, X, M, packed, scale, N, K, Y, s, e);
-  return launch_decode_cfg<DecodeCfg<BITS, 16>>(dev, X, M, packed, scale, N, K, Y, s, e);
+  if (M <= 1) return launch_decode_cfg<DecodeCfg<BITS, 1, 2, ZP>>(dev, X, M, packed, scale, N, K, Y, s, e);
+  if (M <= 2) return launch_decode_cfg<DecodeCfg<BITS, 2, 2, ZP>>(dev, X, M, packed, scale, N, K, Y, s, e);
+  if (M <= 4) return launch_decode_cfg<DecodeCfg<BITS, 4, 2, ZP>>(dev, X, M, packed, scale, N, K, Y, s, e);
+  if (M <= 8) return launch_decode_cfg<DecodeCfg<BITS, 8, 2, ZP>>(dev, X, M, packed, scale, N, K, Y, s, e);
+  return launch_decode_cfg<DecodeCfg<BITS, 16, 2, ZP>>(dev, X, M, packed, scale, N, K, Y, s, e);
 }
 
 // ---------------------------------------------------------------- prefill
@@ -412,6 +438,7 @@ glmq_status launch_prefill_cfg(const DeviceInfo& dev, const void* X, int M, cons
   a.xs = nullptr;
   a.bias = e.bias;
   a.geglu = e.geglu;
+  a.zero = e.zero;
   a.M = M;
   a.N = N;
   a.K = K;
@@ -456,6 +483,7 @@ glmq_status launch_skinny_cfg(const DeviceInfo& dev, const void* X, int M, const
   a.xs = xs;
   a.bias = e.bias;
   a.geglu = e.geglu;
+  a.zero = e.zero;
   a.M = M;
   a.N = N;
   a.K = K;
@@ -488,15 +516,15 @@ glmq_status launch_skinny_cfg(const DeviceInfo& dev, const void* X, int M, const
   return GLMQ_OK;
 }
 
-template <int BITS>
+template <int BITS, int ZP = 0>
 glmq_status launch_prefill(const DeviceInfo& dev, const void* X, int M, const void* packed, const void* scale, int N,
                            int K, void* Y, cudaStream_t s, const Epi& e = Epi()) {
   // up to 64 tokens: the skinny kernel (wide weight stream, A operand in tensor memory)
-  if (M <= 16) return launch_skinny_cfg<SkinnyCfg<BITS, 16>>(dev, X, M, packed, scale, N, K, Y, s, e);
-  if (M <= 32) return launch_skinny_cfg<SkinnyCfg<BITS, 32>>(dev, X, M, packed, scale, N, K, Y, s, e);
-  if (M <= 64) return launch_skinny_cfg<SkinnyCfg<BITS, 64>>(dev, X, M, packed, scale, N, K, Y, s, e);
-  if (M <= 128) return launch_prefill_cfg<PrefillCfg<BITS, 128>>(dev, X, M, packed, scale, N, K, Y, s, e);
-  return launch_prefill_cfg<PrefillCfg<BITS, 256>>(dev, X, M, packed, scale, N, K, Y, s, e);
+  if (M <= 16) return launch_skinny_cfg<SkinnyCfg<BITS, 16, ZP>>(dev, X, M, packed, scale, N, K, Y, s, e);
+  if (M <= 32) return launch_skinny_cfg<SkinnyCfg<BITS, 32, ZP>>(dev, X, M, packed, scale, N, K, Y, s, e);
+  if (M <= 64) return launch_skinny_cfg<SkinnyCfg<BITS, 64, ZP>>(dev, X, M, packed, scale, N, K, Y, s, e);
+  if (M <= 128) return launch_prefill_cfg<PrefillCfg<BITS, 128, ZP>>(dev, X, M, packed, scale, N, K, Y, s, e);
+  return launch_prefill_cfg<PrefillCfg<BITS, 256, ZP>>(dev, X, M, packed, scale, N, K, Y, s, e);
 }
 
 // ---------------------------------------------------------------- decode without allocation
@@ -550,6 +578,7 @@ glmq_status launch_decode_noalloc_cfg(const DeviceInfo& dev, const void* X, int 
   a.units = pl.units;
   a.bias = nullptr;
   a.geglu = 0;
+  a.zero = nullptr;
   cudaError_t e;
   if (pl.parts > 1) {
     if ((st = noalloc_scratch(&a.ws)) != GLMQ_OK) return st;
@@ -590,9 +619,11 @@ glmq_status gemm_entry(Route route, const void* X, int64_t M, const void* packed
   const bool decode = route == Route::kDecode || (route == Route::kAuto && M <= GLMQ_DECODE_AUTO_MAX_M);
   const int m = static_cast<int>(M), n = static_cast<int>(N), k = static_cast<int>(K);
   if (decode) {
+    if (e.zero) return launch_decode<4, 1>(*dev, X, m, packed, scale, n, k, Y, s, e);
     return bits == 4 ? launch_decode<4>(*dev, X, m, packed, scale, n, k, Y, s, e)
                      : launch_decode<8>(*dev, X, m, packed, scale, n, k, Y, s, e);
   }
+  if (e.zero) return launch_prefill<4, 1>(*dev, X, m, packed, scale, n, k, Y, s, e);
   return bits == 4 ? launch_prefill<4>(*dev, X, m, packed, scale, n, k, Y, s, e)
                    : launch_prefill<8>(*dev, X, m, packed, scale, n, k, Y, s, e);
 }
@@ -658,6 +689,26 @@ glmq_status glmq_gemm_fused(const void* X, int64_t M, const void* packed, const 
   e.bias = static_cast<const __half*>(bias);
   e.geglu = geglu ? 1 : 0;
   return gemm_entry(Route::kAuto, X, M, packed, scale, N, K, bits, Y, stream, e);
+}
+
+glmq_status glmq_quantize_zp(const void* W, int64_t N, int64_t K, void* packed, void* scale, void* zero,
+                             void* stream) {
+  glmq_status st = check_common(N, K, 4);
+  if (st != GLMQ_OK) return st;
+  if (N == 0) return GLMQ_OK;
+  if (!W || !packed || !scale || !zero) return GLMQ_ERR_NULL_POINTER;
+  if (!aligned16(W) || !aligned16(packed) || !aligned16(scale)) return GLMQ_ERR_MISALIGNED;
+  const DeviceInfo* dev = nullptr;
+  if ((st = current_device(&dev)) != GLMQ_OK) return st;
+  return launch_quantize_zp(W, N, K, packed, scale, zero, static_cast<cudaStream_t>(stream));
+}
+
+glmq_status glmq_gemm_zp(const void* X, int64_t M, const void* packed, const void* scale, const void* zero,
+                         int64_t N, int64_t K, void* Y, void* stream) {
+  if (!zero && M > 0 && N > 0) return GLMQ_ERR_NULL_POINTER;
+  Epi e;
+  e.zero = static_cast<const uint8_t*>(zero);
+  return gemm_entry(Route::kAuto, X, M, packed, scale, N, K, 4, Y, stream, e);
 }
 
 glmq_status glmq_gemm_decode_noalloc(const void* X, int64_t M, const void* packed, const void* scale, int64_t N,

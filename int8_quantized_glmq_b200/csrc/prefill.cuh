@@ -55,8 +55,9 @@ constexpr int kPrefillThreads = 22 * 32;
 constexpr int kPrefillMaxStages = 8;
 constexpr int kPrefillSmemBudget = 232448 - 1024 /*alignment*/ - 512 /*barriers*/;
 
-template <int BITS, int BN>
+template <int BITS, int BN, int ZP = 0>
 struct PrefillCfg {
+  static constexpr int kZP = ZP;   // 1: zero-point INT4 codes (unsigned, per-row zero point)
   static constexpr int kBits = BITS;
   static constexpr int kBN = BN;
   static constexpr int BM = 128;
@@ -86,6 +87,7 @@ struct PrefillArgs {
   const uint8_t* xs;  // skinny kernel only: activation tiles pre-swizzled by skinny_pack_x_kernel
   const __half* bias; // fp16 [N] in the natural row order of W, or NULL (epilogue.cuh)
   int geglu;          // 1: packed rows in the GeGLU layout, Y is [M, N / 2]
+  const uint8_t* zero;  // zero-point codes: uint8 [N] per-row zero point, else NULL
   int M;
   int N;
   int K;
@@ -192,43 +194,60 @@ __device__ __forceinline__ uint32_t sw128_off(int row, int c) {
 }
 
 // INT4 packed word (8 codes, k = 0..7) -> 4 words of fp16 pairs in natural k order.
-__device__ __forceinline__ uint4 dequant_int4_natural(uint32_t w) {
-  const __half2 kBias0 = __halves2half2(__ushort_as_half(0xE408), __ushort_as_half(0xE408));  // -1032
+// INT4 word (8 codes) -> fp16 values. A code nibble c OR-ed into the mantissa of 1024
+// (low nibbles: XOR constant xlo) or of 1024 at 16x weight (high nibbles: xhi) gives
+// an exact fp16 integer; adding b0 (low) or scaling by 1/16 and adding b1 (high)
+// leaves the code's value. Symmetric codes: xlo = 0x6408 (1024 + (c ^ 8) = 1032 + q),
+// xhi = 0x6480, b0 = -1032, b1 = -72. Zero-point codes: xlo = xhi = 0x6400,
+// b0 = -(1024 + z), b1 = -(64 + z), giving c - z.
+__device__ __forceinline__ void dequant_int4_pairs(uint32_t w, uint32_t xlo, uint32_t xhi, __half2 b0, __half2 b1,
+                                                   __half2 (&r)[4]) {
   const __half2 kOne16 = __halves2half2(__ushort_as_half(0x2C00), __ushort_as_half(0x2C00));  // 1/16
-  const __half2 kBias1 = __halves2half2(__ushort_as_half(0xD480), __ushort_as_half(0xD480));  // -72
   const uint32_t w8 = w >> 8;
-  uint32_t h0 = lop3_and_xor(w, 0x000F000Fu, 0x64086408u);   // (0, 4)
-  uint32_t h1 = lop3_and_xor(w, 0x00F000F0u, 0x64806480u);   // (1, 5) * 16
-  uint32_t h2 = lop3_and_xor(w8, 0x000F000Fu, 0x64086408u);  // (2, 6)
-  uint32_t h3 = lop3_and_xor(w8, 0x00F000F0u, 0x64806480u);  // (3, 7) * 16
-  __half2 r0 = __hadd2(*reinterpret_cast<__half2*>(&h0), kBias0);
-  __half2 r1 = __hfma2(*reinterpret_cast<__half2*>(&h1), kOne16, kBias1);
-  __half2 r2 = __hadd2(*reinterpret_cast<__half2*>(&h2), kBias0);
-  __half2 r3 = __hfma2(*reinterpret_cast<__half2*>(&h3), kOne16, kBias1);
-  const uint32_t p0 = *reinterpret_cast<uint32_t*>(&r0), p1 = *reinterpret_cast<uint32_t*>(&r1);
-  const uint32_t p2 = *reinterpret_cast<uint32_t*>(&r2), p3 = *reinterpret_cast<uint32_t*>(&r3);
+  uint32_t h0 = lop3_and_xor(w, 0x000F000Fu, xlo);   // (0, 4)
+  uint32_t h1 = lop3_and_xor(w, 0x00F000F0u, xhi);   // (1, 5) * 16
+  uint32_t h2 = lop3_and_xor(w8, 0x000F000Fu, xlo);  // (2, 6)
+  uint32_t h3 = lop3_and_xor(w8, 0x00F000F0u, xhi);  // (3, 7) * 16
+  r[0] = __hadd2(*reinterpret_cast<__half2*>(&h0), b0);
+  r[1] = __hfma2(*reinterpret_cast<__half2*>(&h1), kOne16, b1);
+  r[2] = __hadd2(*reinterpret_cast<__half2*>(&h2), b0);
+  r[3] = __hfma2(*reinterpret_cast<__half2*>(&h3), kOne16, b1);
+}
+
+struct Int4Dequant {
+  uint32_t xlo, xhi;
+  __half2 b0, b1;
+};
+
+__device__ __forceinline__ Int4Dequant int4_dequant_symmetric() {
+  return {0x64086408u, 0x64806480u, __halves2half2(__ushort_as_half(0xE408), __ushort_as_half(0xE408)),   // -1032
+          __halves2half2(__ushort_as_half(0xD480), __ushort_as_half(0xD480))};                             // -72
+}
+
+__device__ __forceinline__ Int4Dequant int4_dequant_zero_point(int z) {
+  return {0x64006400u, 0x64006400u, __float2half2_rn(-(1024.0f + static_cast<float>(z))),
+          __float2half2_rn(-(64.0f + static_cast<float>(z)))};
+}
+
+// k order 0..7 of the word
+__device__ __forceinline__ uint4 dequant_int4_natural(uint32_t w, const Int4Dequant& d) {
+  __half2 r[4];
+  dequant_int4_pairs(w, d.xlo, d.xhi, d.b0, d.b1, r);
+  const uint32_t p0 = *reinterpret_cast<uint32_t*>(&r[0]), p1 = *reinterpret_cast<uint32_t*>(&r[1]);
+  const uint32_t p2 = *reinterpret_cast<uint32_t*>(&r[2]), p3 = *reinterpret_cast<uint32_t*>(&r[3]);
   return make_uint4(prmt(p0, p1, 0x5410u), prmt(p2, p3, 0x5410u), prmt(p0, p1, 0x7632u), prmt(p2, p3, 0x7632u));
 }
-
-// INT4 packed word -> 4 words of fp16 pairs (0,4), (1,5), (2,6), (3,7): the k order
-// (0,4,1,5,2,6,3,7) within the 8-code group, matched by a permuted activation tile.
-__device__ __forceinline__ uint4 dequant_int4_paired(uint32_t w) {
-  const __half2 kBias0 = __halves2half2(__ushort_as_half(0xE408), __ushort_as_half(0xE408));  // -1032
-  const __half2 kOne16 = __halves2half2(__ushort_as_half(0x2C00), __ushort_as_half(0x2C00));  // 1/16
-  const __half2 kBias1 = __halves2half2(__ushort_as_half(0xD480), __ushort_as_half(0xD480));  // -72
-  const uint32_t w8 = w >> 8;
-  uint32_t h0 = lop3_and_xor(w, 0x000F000Fu, 0x64086408u);
-  uint32_t h1 = lop3_and_xor(w, 0x00F000F0u, 0x64806480u);
-  uint32_t h2 = lop3_and_xor(w8, 0x000F000Fu, 0x64086408u);
-  uint32_t h3 = lop3_and_xor(w8, 0x00F000F0u, 0x64806480u);
-  __half2 r0 = __hadd2(*reinterpret_cast<__half2*>(&h0), kBias0);
-  __half2 r1 = __hfma2(*reinterpret_cast<__half2*>(&h1), kOne16, kBias1);
-  __half2 r2 = __hadd2(*reinterpret_cast<__half2*>(&h2), kBias0);
-  __half2 r3 = __hfma2(*reinterpret_cast<__half2*>(&h3), kOne16, kBias1);
-  return make_uint4(*reinterpret_cast<uint32_t*>(&r0), *reinterpret_cast<uint32_t*>(&r1),
-                    *reinterpret_cast<uint32_t*>(&r2), *reinterpret_cast<uint32_t*>(&r3));
+__device__ __forceinline__ uint4 dequant_int4_natural(uint32_t w) {
+  return dequant_int4_natural(w, int4_dequant_symmetric());
 }
-
+// k order (0,4,1,5,2,6,3,7): no byte shuffle
+__device__ __forceinline__ uint4 dequant_int4_paired(uint32_t w, const Int4Dequant& d) {
+  __half2 r[4];
+  dequant_int4_pairs(w, d.xlo, d.xhi, d.b0, d.b1, r);
+  return make_uint4(*reinterpret_cast<uint32_t*>(&r[0]), *reinterpret_cast<uint32_t*>(&r[1]),
+                    *reinterpret_cast<uint32_t*>(&r[2]), *reinterpret_cast<uint32_t*>(&r[3]));
+}
+__device__ __forceinline__ uint4 dequant_int4_paired(uint32_t w) { return dequant_int4_paired(w, int4_dequant_symmetric()); }
 __device__ __forceinline__ uint2 dequant_int8_natural(uint32_t w) {
   const __half2 kBias = __halves2half2(__ushort_as_half(0xE480), __ushort_as_half(0xE480));  // -1152
   const uint32_t x = w ^ 0x80808080u;
@@ -322,6 +341,11 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     for (int u = blockIdx.x; u < a.units && ok; u += G) {
       const int p = u / a.tiles;
       const int kb1 = min(num_kb, (p + 1) * a.kbp);
+      Int4Dequant dq = int4_dequant_symmetric();
+      if constexpr (C::kZP) {
+        const int wrow = ((u - p * a.tiles) / a.tiles_m) * C::BM + row;
+        dq = int4_dequant_zero_point(wrow < a.N ? a.zero[wrow] : 0);
+      }
       for (int kb = p * a.kbp; kb < kb1; ++kb, ++seq) {
         if ((seq & (kPrefillDequantGroups - 1)) == grp) {
           if (!mbar_wait_warp(&full[stage], phase)) { ok = false; break; }
@@ -345,7 +369,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
               const uint32_t words[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
               for (int j = 0; j < 4; ++j) {
-                const uint4 o = C::kPermX ? dequant_int4_paired(words[j]) : dequant_int4_natural(words[j]);
+                const uint4 o = C::kPermX ? dequant_int4_paired(words[j], dq) : dequant_int4_natural(words[j], dq);
                 st_shared_v4(a_tile + sw128_off(row, 4 * h + j), o.x, o.y, o.z, o.w);
               }
             }

@@ -34,9 +34,10 @@
 namespace glmq {
 
 
-template <int BITS>
-__device__ __forceinline__ int exact_code(float w, float sf, float kf) {
-  constexpr int D = (1 << (BITS - 1)) - 1;
+// RNE(w / s) from a candidate kf within one of it, clamped to magnitude D, by exact
+// comparisons of 2|w| with (2k +- 1) s.
+template <int D>
+__device__ __forceinline__ int exact_code_d(float w, float sf, float kf) {
   const float aw = fabsf(w);
   const int k0 = static_cast<int>(fabsf(kf));
   const float aw2 = aw + aw;                                   // exact
@@ -50,6 +51,11 @@ __device__ __forceinline__ int exact_code(float w, float sf, float kf) {
   }
   k = min(k, D);
   return (w < 0.0f) ? -k : k;
+}
+
+template <int BITS>
+__device__ __forceinline__ int exact_code(float w, float sf, float kf) {
+  return exact_code_d<(1 << (BITS - 1)) - 1>(w, sf, kf);
 }
 
 // Codes for the 8 halves of one 16-byte chunk, as 32-bit words whose low bits hold
@@ -154,6 +160,109 @@ __global__ void __launch_bounds__(T) quantize_kernel(const __half* __restrict__ 
       out.y = (u[4] & 0xFFu) | ((u[5] & 0xFFu) << 8) | ((u[6] & 0xFFu) << 16) | ((u[7] & 0xFFu) << 24);
       reinterpret_cast<uint2*>(packed + row * static_cast<long long>(K))[c] = out;
     }
+  }
+}
+
+// ---------------------------------------------------------------- zero-point INT4
+// Asymmetric variant (GLM-130B paper card, "Pitfalls": a zero-point INT4 quantizer
+// scored better on LAMBADA but was not adopted; the card gives no formula). Per row:
+//   lo = min(0, min W), hi = max(0, max W), s = fp16_rn(fl32(fl32(hi - lo) / 15)),
+//   z = clamp(rint(fl32(-lo / s)), 0, 15), q = clamp(RNE(w / s) + z, 0, 15) unsigned,
+// q = 0 and z = 0 where s == 0. Codes are packed like the symmetric ones (low nibble =
+// even k). RNE(w / s) is exact, by the same fma candidate and comparison fix-up as
+// quantize_kernel (|w / s| <= 16 here).
+__device__ __forceinline__ void zp_chunk_codes(const uint4 v, float sf, float r, bool exact_all, int z,
+                                               uint32_t (&q)[8]) {
+  const uint32_t words[4] = {v.x, v.y, v.z, v.w};
+  float w[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&words[i]));
+    w[2 * i] = f.x;
+    w[2 * i + 1] = f.y;
+  }
+  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+  constexpr float kMargin = 0.5f - 0x1p-15f;
+  float kf[8];
+  bool near = exact_all;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    kf[i] = fmaf(w[i], r, kMagic) - kMagic;
+    near |= fabsf(fmaf(w[i], r, -kf[i])) >= kMargin;
+  }
+  if (near) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) kf[i] = static_cast<float>(exact_code_d<16>(w[i], sf, kf[i]));
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) q[i] = static_cast<uint32_t>(min(max(static_cast<int>(kf[i]) + z, 0), 15));
+}
+
+template <int CPT, int T>
+__global__ void __launch_bounds__(T) quantize_zp_kernel(const __half* __restrict__ W, int K,
+                                                        uint8_t* __restrict__ packed, __half* __restrict__ scale,
+                                                        uint8_t* __restrict__ zero) {
+  const long long row = blockIdx.x;
+  const int nchunks = K >> 3;
+  const uint4* src = reinterpret_cast<const uint4*>(W + row * static_cast<long long>(K));
+  uint4 v[CPT];
+  __half2 mn = __float2half2_rn(0.0f), mx = mn;      // the range includes zero
+#pragma unroll
+  for (int i = 0; i < CPT; ++i) {
+    const int c = threadIdx.x + i * T;
+    v[i] = make_uint4(0, 0, 0, 0);
+    if (c < nchunks) {
+      v[i] = ld_stream_v4(src + c);
+      const uint32_t words[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const __half2 h = *reinterpret_cast<const __half2*>(&words[j]);
+        mn = __hmin2(mn, h);
+        mx = __hmax2(mx, h);
+      }
+    }
+  }
+  float lo = fminf(__low2float(mn), __high2float(mn));
+  float hi = fmaxf(__low2float(mx), __high2float(mx));
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, off));
+    hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, off));
+  }
+  __shared__ float warp_lo[T / 32], warp_hi[T / 32];
+  const int warp = threadIdx.x >> 5;
+  if ((threadIdx.x & 31) == 0) {
+    warp_lo[warp] = lo;
+    warp_hi[warp] = hi;
+  }
+  __syncthreads();
+  lo = warp_lo[0];
+  hi = warp_hi[0];
+#pragma unroll
+  for (int i = 1; i < T / 32; ++i) {
+    lo = fminf(lo, warp_lo[i]);
+    hi = fmaxf(hi, warp_hi[i]);
+  }
+  const __half s = __float2half_rn(__fdiv_rn(hi - lo, 15.0f));
+  const float sf = __half2float(s);
+  const bool zero_row = (sf == 0.0f);
+  const int z = zero_row ? 0 : min(max(static_cast<int>(rintf(__fdiv_rn(-lo, sf))), 0), 15);
+  if (threadIdx.x == 0) {
+    scale[row] = s;
+    zero[row] = static_cast<uint8_t>(z);
+  }
+  const bool exact_all = sf < 0x1p-14f;  // subnormal scale
+  const float r = zero_row ? 0.0f : __frcp_rn(sf);
+#pragma unroll
+  for (int i = 0; i < CPT; ++i) {
+    const int c = threadIdx.x + i * T;
+    if (c >= nchunks) continue;
+    uint32_t q[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    if (!zero_row) zp_chunk_codes(v[i], sf, r, exact_all, z, q);
+    uint32_t word = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) word |= q[j] << (4 * j);
+    reinterpret_cast<uint32_t*>(packed + row * static_cast<long long>(K / 2))[c] = word;
   }
 }
 

@@ -48,8 +48,9 @@ constexpr int kSkinnyMmaWarp = 21;
 constexpr int kSkinnyThreads = 22 * 32;
 constexpr int kSkinnyASlots = 8;           // A operand slots in TMEM (one 64-wide K block each)
 
-template <int BITS, int BN>
+template <int BITS, int BN, int ZP = 0>
 struct SkinnyCfg {
+  static constexpr int kZP = ZP;   // 1: zero-point INT4 codes (unsigned, per-row zero point)
   static constexpr int kBits = BITS;
   static constexpr int kBN = BN;
   static constexpr int BM = 128;
@@ -216,6 +217,11 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
     for (int u = blockIdx.x; u < a.units && ok; u += G) {
       const int p = u / a.tiles;
       const int st1 = min(num_st, (p + 1) * a.kbp);
+      Int4Dequant dq = int4_dequant_symmetric();
+      if constexpr (C::kZP) {
+        const int wrow = ((u - p * a.tiles) / a.tiles_m) * C::BM + row;
+        dq = int4_dequant_zero_point(wrow < a.N ? a.zero[wrow] : 0);
+      }
       for (int ks = p * a.kbp; ks < st1 && ok; ++ks) {
         const int nkb = skinny_stage_kblocks(ks * C::SK, K, C::KB);
         bool waited = false;
@@ -240,7 +246,7 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
               const uint32_t words[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
               for (int wv = 0; wv < 4; ++wv) {
-                const uint4 o = dequant_int4_paired(words[wv]);
+                const uint4 o = dequant_int4_paired(words[wv], dq);
                 h[16 * q + 4 * wv + 0] = o.x;
                 h[16 * q + 4 * wv + 1] = o.y;
                 h[16 * q + 4 * wv + 2] = o.z;

@@ -125,3 +125,13 @@ def test_fused_entry_points_validate_before_device_work():
     assert B.raw_quantize_geglu(ALIGNED, 40, 64, 4, ALIGNED, ALIGNED) == B.ERR_BAD_SHAPE
     assert B.raw_quantize_geglu(ALIGNED, 48, 64, 3, ALIGNED, ALIGNED) == B.ERR_BAD_BITS
     assert B.raw_quantize_geglu(0, 0, 64, 4, 0, 0) == B.OK
+
+
+def test_zero_point_entry_points_validate_before_device_work():
+    assert B.raw_quantize_zp(ALIGNED, 4, 100, ALIGNED, ALIGNED, ALIGNED) == B.ERR_BAD_SHAPE
+    assert B.raw_quantize_zp(ALIGNED, 4, 64, ALIGNED, ALIGNED, 0) == B.ERR_NULL_POINTER
+    assert B.raw_quantize_zp(ALIGNED + 2, 4, 64, ALIGNED, ALIGNED, ALIGNED) == B.ERR_MISALIGNED
+    assert B.raw_quantize_zp(0, 0, 64, 0, 0, 0) == B.OK
+    assert B.raw_gemm_zp(ALIGNED, 4, ALIGNED, ALIGNED, 0, 8, 64, ALIGNED) == B.ERR_NULL_POINTER
+    assert B.raw_gemm_zp(ALIGNED, 4, ALIGNED, ALIGNED, ALIGNED, 8, 96, ALIGNED) == B.ERR_BAD_SHAPE
+    assert B.raw_gemm_zp(0, 0, ALIGNED, ALIGNED, 0, 8, 64, 0) == B.OK

@@ -415,6 +415,23 @@ def run_extras(torch, glmq, W16, quant, peaks):
                                                "fused_weight_gbs": round(pg.numel() / tg / 1e9, 1)}
         del X, Yg, Yp
     del pg, sg
+    # zero-point INT4 on QKV against the symmetric codes
+    N, K = GLM_PROJECTIONS["qkv"]
+    pz = torch.empty((N, K // 2), dtype=torch.uint8, device="cuda")
+    sz = torch.empty((N,), dtype=torch.float16, device="cuda")
+    zz = torch.empty((N,), dtype=torch.uint8, device="cuda")
+    tq = time_launches(torch, lambda: glmq.quantize_zp(W16["qkv"], out=(pz, sz, zz)), 3)
+    out["zero_point_int4_qkv"] = {"quantize_us": round(tq * 1e6, 1),
+                                  "quantize_gbs": round((N * K * 2 + N * K // 2 + N * 3) / tq / 1e9, 1)}
+    for M in (1, 16, 2048):
+        g = torch.Generator(device="cuda").manual_seed(7000 + M)
+        X = torch.randn((M, K), generator=g, device="cuda", dtype=torch.float32).half()
+        Y = torch.empty((M, N), dtype=torch.float16, device="cuda")
+        t = time_launches(torch, lambda: glmq.gemm_zp(X, pz, sz, zz, out=Y), 5)
+        out["zero_point_int4_qkv"][f"M={M}"] = {"us": round(t * 1e6, 1), "weight_gbs": round(pz.numel() / t / 1e9, 1),
+                                                "tflops": round(2.0 * M * N * K / t / 1e12, 1)}
+        del X, Y
+    del pz, sz, zz
     for name in PROJECTION_ORDER:
         N, K = GLM_PROJECTIONS[name]
         p8 = torch.empty((N, K), dtype=torch.uint8, device="cuda")

@@ -94,33 +94,14 @@ struct DecodeArgs {
   int units;          // parts * tiles
 };
 
-// ---------------------------------------------------------------- dequantization
-// INT4: one packed word (8 codes, k = 0..7 of the word) -> 4 half2 registers
-// holding the pairs (0,4), (1,5), (2,6), (3,7).
-__device__ __forceinline__ void dequant_int4_word(uint32_t w, uint32_t (&p)[4]) {
-  const __half2 kBias0 = __halves2half2(__ushort_as_half(0xE408), __ushort_as_half(0xE408));  // -1032
-  const __half2 kOne16 = __halves2half2(__ushort_as_half(0x2C00), __ushort_as_half(0x2C00));  // 1/16
-  const __half2 kBias1 = __halves2half2(__ushort_as_half(0xD480), __ushort_as_half(0xD480));  // -72
-  const uint32_t w8 = w >> 8;
-  uint32_t h0 = lop3_and_xor(w, 0x000F000Fu, 0x64086408u);
-  uint32_t h1 = lop3_and_xor(w, 0x00F000F0u, 0x64806480u);
-  uint32_t h2 = lop3_and_xor(w8, 0x000F000Fu, 0x64086408u);
-  uint32_t h3 = lop3_and_xor(w8, 0x00F000F0u, 0x64806480u);
-  __half2 r0 = __hadd2(*reinterpret_cast<__half2*>(&h0), kBias0);
-  __half2 r1 = __hfma2(*reinterpret_cast<__half2*>(&h1), kOne16, kBias1);
-  __half2 r2 = __hadd2(*reinterpret_cast<__half2*>(&h2), kBias0);
-  __half2 r3 = __hfma2(*reinterpret_cast<__half2*>(&h3), kOne16, kBias1);
-  p[0] = *reinterpret_cast<uint32_t*>(&r0);
-  p[1] = *reinterpret_cast<uint32_t*>(&r1);
-  p[2] = *reinterpret_cast<uint32_t*>(&r2);
-  p[3] = *reinterpret_cast<uint32_t*>(&r3);
-}
-
-// INT4, biased form: the same pairs without the final subtraction. Low nibbles give
-// the fp16 integers 1032 + q, high nibbles 1152 + 16 q; the MMA's B operand holds x
-// for low-nibble slots and x / 16 for high-nibble slots, so every product is
-// q * x + (a bias depending only on x), and the accumulated bias is removed per
-// segment (see decode_segment). Four LOP3 and one shift per 8 codes.
+// INT4, biased form: one packed word (8 codes, k = 0..7 of the word) -> 4 half2
+// registers holding the pairs (0,4), (1,5), (2,6), (3,7). A code nibble OR-ed into
+// the mantissa of 1024 gives an exact fp16 integer: for symmetric codes (XOR 0x6408 /
+// 0x6480) low nibbles give 1032 + q and high nibbles 1152 + 16 q; for zero-point codes
+// (XOR 0x6400) 1024 + c and 1024 + 16 c. The MMA's B operand holds x for low-nibble
+// slots and x / 16 for high-nibble slots, so every product is (code value) * x plus a
+// bias depending only on x, and the accumulated bias is removed per segment (see
+// decode_segment). Four LOP3 and one shift per 8 codes.
 template <uint32_t XLO, uint32_t XHI>
 __device__ __forceinline__ void dequant_int4_word_biased(uint32_t w, uint32_t (&p)[4]) {
   const uint32_t w8 = w >> 8;

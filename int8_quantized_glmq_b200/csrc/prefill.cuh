@@ -31,11 +31,6 @@
 // there are fewer tiles than SMs (small M), tiles are split over K parts so every
 // SM has work, each unit adds its fp32 partial tile into a scratch buffer with
 // red.global.add and a stream-ordered finalize kernel scales, rounds and stores Y.
-// For small token tiles (INT4, BN <= 32) the dequantizers write each 8-code group
-// in the order the register dequantization produces it, (0,4,1,5,2,6,3,7), and
-// permute the activation tile identically in place after it lands, which saves the
-// byte shuffles per packed word; the MMA's k order is immaterial when both
-// operands use the same one.
 // No TMA multicast is used anywhere.
 #pragma once
 
@@ -69,7 +64,6 @@ struct PrefillCfg {
   static constexpr int STAGE_BYTES = X_BYTES + A_BYTES + W_BYTES;
   static constexpr int kStages = (kPrefillSmemBudget / STAGE_BYTES) < kPrefillMaxStages
                                      ? (kPrefillSmemBudget / STAGE_BYTES) : kPrefillMaxStages;
-  static constexpr int kPermX = (BITS == 4 && BN <= 32) ? 1 : 0;   // permuted k order (see above)
   static constexpr int TMEM_COLS = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64 : (2 * BN <= 128) ? 128
                                  : (2 * BN <= 256) ? 256 : 512;
   static constexpr int SMEM_BYTES = kStages * STAGE_BYTES + 1024 /*align*/ + 512 /*barriers*/;
@@ -237,9 +231,6 @@ __device__ __forceinline__ uint4 dequant_int4_natural(uint32_t w, const Int4Dequ
   const uint32_t p2 = *reinterpret_cast<uint32_t*>(&r[2]), p3 = *reinterpret_cast<uint32_t*>(&r[3]);
   return make_uint4(prmt(p0, p1, 0x5410u), prmt(p2, p3, 0x5410u), prmt(p0, p1, 0x7632u), prmt(p2, p3, 0x7632u));
 }
-__device__ __forceinline__ uint4 dequant_int4_natural(uint32_t w) {
-  return dequant_int4_natural(w, int4_dequant_symmetric());
-}
 // k order (0,4,1,5,2,6,3,7): no byte shuffle
 __device__ __forceinline__ uint4 dequant_int4_paired(uint32_t w, const Int4Dequant& d) {
   __half2 r[4];
@@ -247,7 +238,6 @@ __device__ __forceinline__ uint4 dequant_int4_paired(uint32_t w, const Int4Dequa
   return make_uint4(*reinterpret_cast<uint32_t*>(&r[0]), *reinterpret_cast<uint32_t*>(&r[1]),
                     *reinterpret_cast<uint32_t*>(&r[2]), *reinterpret_cast<uint32_t*>(&r[3]));
 }
-__device__ __forceinline__ uint4 dequant_int4_paired(uint32_t w) { return dequant_int4_paired(w, int4_dequant_symmetric()); }
 __device__ __forceinline__ uint2 dequant_int8_natural(uint32_t w) {
   const __half2 kBias = __halves2half2(__ushort_as_half(0xE480), __ushort_as_half(0xE480));  // -1152
   const uint32_t x = w ^ 0x80808080u;
@@ -350,17 +340,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         if ((seq & (kPrefillDequantGroups - 1)) == grp) {
           if (!mbar_wait_warp(&full[stage], phase)) { ok = false; break; }
           uint8_t* st = smem + stage * C::STAGE_BYTES;
-          const uint32_t x_tile = smem_u32(st);
           const uint32_t a_tile = smem_u32(st + C::X_BYTES);
           const uint32_t w_tile = smem_u32(st + C::X_BYTES + C::A_BYTES);
-          if constexpr (C::kPermX) {
-            // permute each 16-byte unit of the activation tile to (0,4,1,5,2,6,3,7) in place
-            for (int i = row; i < C::kBN * 8; i += 128) {
-              const uint4 v = lds_v4(x_tile + 16 * i);
-              st_shared_v4(x_tile + 16 * i, prmt(v.x, v.z, 0x5410u), prmt(v.x, v.z, 0x7632u),
-                           prmt(v.y, v.w, 0x5410u), prmt(v.y, v.w, 0x7632u));
-            }
-          }
           if constexpr (C::kBits == 4) {
             // 32-byte rows, 32-byte swizzle: 16-byte unit u sits at u ^ ((row >> 2) & 1)
 #pragma unroll
@@ -369,7 +350,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
               const uint32_t words[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
               for (int j = 0; j < 4; ++j) {
-                const uint4 o = C::kPermX ? dequant_int4_paired(words[j], dq) : dequant_int4_natural(words[j], dq);
+                const uint4 o = dequant_int4_natural(words[j], dq);
                 st_shared_v4(a_tile + sw128_off(row, 4 * h + j), o.x, o.y, o.z, o.w);
               }
             }

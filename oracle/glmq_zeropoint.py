@@ -14,7 +14,8 @@ Readings (each also listed in the design notes):
   Z1 range: lo = min(0, min_k W[n,k]), hi = max(0, max_k W[n,k]) (exact fp16 values;
      zero is inside the range, so an all-zero row gives s = 0 and a constant row is
      still representable).
-  Z2 scale: s = fp16_rn( fp32(hi - lo) / 15 )  (hi - lo is exact in fp32).
+  Z2 scale: s = fp16_rn( fp32(hi - lo) / 15 ), the difference and the quotient each
+     rounded to nearest in IEEE fp32.
   Z3 zero point: z = clamp(rint(fp32(-lo) / fp32(s)), 0, 15), one uint8 per row;
      z = 0 where s == 0.
   Z4 codes: q = clamp(rint(fp32(w) / fp32(s)) + z, 0, 15), unsigned 4-bit, round half
@@ -38,7 +39,7 @@ def zp_range(W: np.ndarray):
 
 
 def zp_scale(lo: np.ndarray, hi: np.ndarray) -> np.ndarray:
-    """s = fp16_rn( fp32(hi - lo) / 15 ): reading Z2."""
+    """s = fp16_rn( fl32(fl32(hi - lo) / 15) ): reading Z2."""
     return ((np.asarray(hi, np.float32) - np.asarray(lo, np.float32)) / np.float32(15.0)).astype(np.float16)
 
 

@@ -209,6 +209,25 @@ def time_launches(torch, fn, iters: int, warmup: int = 2):
     return e0.elapsed_time(e1) / 1e3 / iters
 
 
+def time_launches_cold(torch, fn, iters: int, warmup: int = 2):
+    """Average device time of fn() per call with L2 flushed before each call (a
+    256 MB write between calls, outside the timed events)."""
+    flush = torch.empty((256 << 20,), dtype=torch.uint8, device="cuda")
+    for _ in range(warmup):
+        fn()
+    s = torch.cuda.current_stream()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(iters)]
+    torch.cuda.synchronize()
+    for e0, e1 in ev:
+        flush.zero_()
+        e0.record(s)
+        fn()
+        e1.record(s)
+    torch.cuda.synchronize()
+    del flush
+    return sum(e0.elapsed_time(e1) for e0, e1 in ev) / 1e3 / iters
+
+
 def run_decode(args, world, rank, local):
     import torch
     import int8_quantized_glmq_b200 as glmq
@@ -432,6 +451,30 @@ def run_extras(torch, glmq, W16, quant, peaks):
                                                 "tflops": round(2.0 * M * N * K / t / 1e12, 1)}
         del X, Y
     del pz, sz, zz
+    # one rank's local GEMM under 4-way tensor parallelism (column: QKV, FFN-up; row:
+    # attn-out, FFN-down); every rank's shard has the same shape, so rank 0's is timed.
+    # The shards fit in L2, so L2 is flushed before each timed call.
+    from int8_quantized_glmq_b200 import tensor_parallel as tpm
+    out["tp4_local_int4"] = {}
+    for name in PROJECTION_ORDER:
+        N, K = GLM_PROJECTIONS[name]
+        packed, scale = quant[name]
+        if name in ("qkv", "ffn_up"):
+            layer = tpm.ColumnParallelLinear(packed, scale, 4, 0, 4)
+            Kl, Nl = K, N // 4
+        else:
+            layer = tpm.RowParallelLinear(packed, scale, 4, 0, 4)
+            Kl, Nl = K // 4, N
+        res = {"shard": f"{Nl}x{Kl}"}
+        for M in (1, 16):
+            g = torch.Generator(device="cuda").manual_seed(8000 + M)
+            X = torch.randn((M, Kl), generator=g, device="cuda", dtype=torch.float32).half()
+            Y = torch.empty((M, Nl), dtype=torch.float16, device="cuda")
+            t = time_launches_cold(torch, lambda: glmq.gemm(X, layer.packed, layer.scale, 4, out=Y), 5)
+            res[f"M={M}"] = {"us": round(t * 1e6, 1), "weight_gbs": round(layer.packed.numel() / t / 1e9, 1)}
+            del X, Y
+        out["tp4_local_int4"][name] = res
+        del layer
     for name in PROJECTION_ORDER:
         N, K = GLM_PROJECTIONS[name]
         p8 = torch.empty((N, K), dtype=torch.uint8, device="cuda")

@@ -217,13 +217,16 @@ __device__ __forceinline__ void decode_segment(uint32_t box, uint32_t xseg, uint
 // the B fragments are read (x_unit), INT4 slots permuted and high-nibble slots
 // divided by 16 (see dequant_int4_word_biased). Units of tokens >= M and of k past
 // plen are not written (no fragment of a real token reads them).
+// With issued != 0 every thread adds 1 to that shared counter once its first batch of
+// global loads has been issued (or at once when it has none).
 template <class C>
 __device__ __forceinline__ void stage_activations(const __half* __restrict__ X, int K, int M, int pk0, int plen,
-                                                  uint8_t* xbuf, int ct) {
+                                                  uint8_t* xbuf, int ct, uint32_t issued = 0) {
   constexpr int kCT = kDecodeConsumerWarps * 32;
   constexpr int kBatch = 8;
   const int nseg = (plen + C::SEGK - 1) / C::SEGK;
   const int total = nseg * C::XU * C::kMP * 4;                  // 16-byte units of the slice
+  if (issued != 0 && ct >= total) shared_count_add(issued);
   for (int d0 = ct; d0 < total; d0 += kCT * kBatch) {
     uint4 v[kBatch];
     bool live[kBatch];
@@ -240,6 +243,7 @@ __device__ __forceinline__ void stage_activations(const __half* __restrict__ X, 
       v[b] = make_uint4(0, 0, 0, 0);
       if (live[b]) v[b] = __ldg(reinterpret_cast<const uint4*>(X + static_cast<long long>(n) * K + pk0 + kr));
     }
+    if (issued != 0 && d0 == ct) shared_count_add(issued);
 #pragma unroll
     for (int b = 0; b < kBatch; ++b) {
       if (!live[b]) continue;
@@ -272,6 +276,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   uint8_t* wring = smem;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kDecodeStages * kDecodeStageBytes);
   uint64_t* empty = full + kDecodeStages;
+  uint32_t* x_issued = reinterpret_cast<uint32_t*>(empty + kDecodeStages);   // inside the fixed 256 bytes
   uint8_t* xbuf = smem + kDecodeFixedSmem;
   // INT4 only: per (segment, token) bias of the biased dequantization, after the activation slice;
   // zero-point codes: then per-token sums of x over the part
@@ -290,6 +295,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], kDecodeConsumerWarps);
     }
+    *x_issued = 0;
     fence_barrier_init();
   }
   __syncthreads();
@@ -306,12 +312,28 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
+      // The consumers stage the first part's activations as soon as they start. Let
+      // their loads enter the memory system before the weight stream fills the ring
+      // (behind ~200 KB per SM of TMA traffic they would arrive microseconds later).
+      // Only an ordering hint: the wait is bounded and the stream starts either way.
+      const uint32_t issued_u32 = smem_u32(x_issued);
+      for (int i = 0; i < 4096 && shared_count_read(issued_u32) < static_cast<uint32_t>(kDecodeConsumerWarps * 32);
+           ++i)
+        __nanosleep(32);
+      int pref_part = u_begin < u_end ? u_begin / a.tiles : -1;
       for (int u = u_begin; u < u_end && ok; ++u) {
         const int p = u / a.tiles;
         const int t = u - p * a.tiles;
         const int pk0 = p * a.KPP;
         const int plen = min(a.KPP, K - pk0);
         const int nst = (plen + C::SK - 1) / C::SK;
+        if (p != pref_part) {
+          // a later part: bring its activation slice into L2 while the ring still holds
+          // the previous part's stages (rows of X are 128-byte aligned: K % 64 == 0)
+          for (int n = 0; n < M; ++n)
+            bulk_prefetch_l2(a.X + static_cast<long long>(n) * K + pk0, static_cast<uint32_t>(plen) * 2u);
+          pref_part = p;
+        }
         for (int ks = 0; ks < nst; ++ks) {
           if (!mbar_wait(&empty[stage], phase ^ 1)) { ok = false; break; }
           const int xb0 = (pk0 + ks * C::SK) / C::KPB;            // first packed byte of the stage
@@ -360,7 +382,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       // Thread i fills shared 16-byte unit i (conflict-free stores); each thread first
       // issues all its global loads of a batch through the read-only path, then stores.
       named_barrier_sync(1, kCT);
-      stage_activations<C>(a.X, K, M, pk0, plen, xbuf, ct);
+      stage_activations<C>(a.X, K, M, pk0, plen, xbuf, ct, cur_part < 0 ? smem_u32(x_issued) : 0u);
       if constexpr (C::kBits == 4) {
         // per (segment, token) bias sum_k (1032 or 1152) * B[k], one warp per real pair
         // (lane = 8-value chunk of the 256-k segment), read back from the staged slice

@@ -19,6 +19,10 @@ namespace glmq {
 template <int VEC>
 __global__ void __launch_bounds__(256) decode_finalize_kernel(float* __restrict__ ws, const __half* __restrict__ scale,
                                                               __half* __restrict__ Y, int M, int N) {
+  // Let the next kernel in the stream launch now: its CTAs take their SM slots and run
+  // their shared-memory prologue while this pass waits; every kernel launched with a
+  // grid dependency here waits (griddep_wait) for this one before touching memory.
+  griddep_launch_dependents();
   griddep_wait();   // the partial sums come from the kernel before this one
   const int n = (blockIdx.x * 256 + threadIdx.x) * VEC;
   if (n >= N) return;
@@ -56,6 +60,7 @@ __global__ void __launch_bounds__(256) finalize_epilogue_kernel(float* __restric
                                                                 const __half* __restrict__ scale,
                                                                 const __half* __restrict__ bias, int geglu,
                                                                 __half* __restrict__ Y, int M, int N) {
+  griddep_launch_dependents();   // as in decode_finalize_kernel
   griddep_wait();   // the partial sums come from the kernel before this one
   const int width = geglu ? (N >> 1) : N;
   const int j = blockIdx.x * 256 + threadIdx.x;

@@ -131,9 +131,10 @@ __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity) {
 // previous kernel in the stream is still running. griddep_wait() blocks until that
 // kernel has completed and its memory operations are visible; every thread calls it
 // before its first global-memory access. griddep_launch_dependents() lets the next
-// such kernel start launching once every CTA of this grid has called it or exited;
-// only single-wave grids call it (all their CTAs are resident before any dependent
-// CTA can take an SM). Both are no-ops for a kernel launched without the attribute.
+// such kernel start launching once every CTA of this grid has called it or exited, so
+// every CTA of this grid holds its SM (or is done) before a dependent CTA can take
+// one: a dependent waiting in griddep_wait never keeps this grid from finishing.
+// Both are no-ops for a kernel launched without the attribute.
 __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" :::); }
 
@@ -152,6 +153,23 @@ __device__ __forceinline__ uint64_t policy_evict_first() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
   return p;
+}
+
+// L2 prefetch of a contiguous global range (a hint: nothing waits for it). Address
+// 16-byte aligned, size a multiple of 16.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* gmem, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(gmem), "r"(bytes) : "memory");
+}
+
+// ---------------------------------------------------------------- shared-memory counter
+__device__ __forceinline__ void shared_count_add(uint32_t addr) {
+  asm volatile("red.relaxed.cta.shared::cta.add.u32 [%0], 1;" ::"r"(addr) : "memory");
+}
+
+__device__ __forceinline__ uint32_t shared_count_read(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.volatile.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
 }
 
 // ---------------------------------------------------------------- named barrier for a warp subset

@@ -268,18 +268,31 @@ def run_decode(args, world, rank, local):
     alg_bytes = sum(quant[n][0].numel() + quant[n][1].numel() * 2 + xs[(M, n)].numel() * 2 + ys[(M, n)].numel() * 2
                     for (M, n) in launches)
 
+    # Each call names the next call of the step (the last one the next step's first) in
+    # glmq_gemm_decode_prefetch, which prefetches that call's first weight tiles into L2
+    # while its own pipeline drains; the outputs are computed exactly as by the plain call.
+    def call(j, hint=True, X=None, Y=None):
+        M, n = launches[j]
+        Mn, nn = launches[(j + 1) % len(launches)]
+        X = xs[(M, n)] if X is None else X
+        Y = ys[(M, n)] if Y is None else Y
+        if not hint:
+            return glmq.gemm(X, quant[n][0], quant[n][1], bits, out=Y)
+        return glmq.gemm_decode_prefetch(X, quant[n][0], quant[n][1], bits, next_packed=quant[nn][0], next_M=Mn,
+                                         out=Y)
+
     # The timed steps are captured into one CUDA graph: K steps of the 12 public calls.
     # Every EVENT_EVERY-th step carries timing-event record nodes (external events)
     # around each call; those give the per-launch device times of the roofline. The
     # other steps run as a plain chain of kernels (event nodes between kernels add
     # gaps and cut the programmatic-launch edges, so they are kept to a sample).
     # The eager calls before capture size the library's scratch and set attributes.
-    for (M, n) in launches:
-        glmq.gemm(xs[(M, n)], quant[n][0], quant[n][1], bits, out=ys[(M, n)])
+    for j in range(len(launches)):
+        call(j)
     torch.cuda.synchronize()
     cap_stream = torch.cuda.Stream()
 
-    def capture(n_steps, with_events):
+    def capture(n_steps, with_events, hint=True):
         g = torch.cuda.CUDAGraph()
         sampled = [it for it in range(n_steps) if with_events and it % EVENT_EVERY == 0]
         evs = {it: [(torch.cuda.Event(enable_timing=True, external=True),
@@ -294,7 +307,7 @@ def run_decode(args, world, rank, local):
                 for j, (M, n) in enumerate(launches):
                     if it in evs:
                         evs[it][j][0].record()
-                    glmq.gemm(xs[(M, n)], quant[n][0], quant[n][1], bits, out=ys[(M, n)])
+                    call(j, hint)
                     if it in evs:
                         evs[it][j][1].record()
             if with_events:
@@ -322,6 +335,19 @@ def run_decode(args, world, rank, local):
     value, elapsed_max = whole_job_rate(weight_bytes / 1e9, args.steps, elapsed, world)
     del warm_graph, timed_graph
 
+    # the same step with plain decode calls (no next-call hint), for comparison
+    # (the returned events stay referenced until the graph is gone: its event nodes use them)
+    plain_graph, plain_ev, (p0, p1), _ = capture(args.steps, True, hint=False)
+    plain_graph.replay()
+    torch.cuda.synchronize()
+    barrier(world)
+    plain_graph.replay()
+    torch.cuda.synchronize()
+    barrier(world)
+    plain_value, _ = whole_job_rate(weight_bytes / 1e9, args.steps, p0.elapsed_time(p1) / 1e3, world)
+    del plain_graph, plain_ev
+    extras["decode_step_without_prefetch_hint_gbs"] = round(plain_value, 2)
+
     # e2e through the public API: pinned host X in, pinned host Y out, every step
     hx = {k: v.cpu().pin_memory() for k, v in xs.items()}
     hy = {k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in ys.items()}
@@ -348,7 +374,7 @@ def run_decode(args, world, rank, local):
                 xbuf[k].copy_(hx[k], non_blocking=True)
             ev_x[k].record(h2d_stream)
             cap_stream.wait_event(ev_x[k])
-            glmq.gemm(xbuf[k], quant[n][0], quant[n][1], bits, out=ybuf[k])
+            call(launches.index(k), X=xbuf[k], Y=ybuf[k])
             ev_y[k].record(cap_stream)
             d2h_stream.wait_event(ev_y[k])
             with torch.cuda.stream(d2h_stream):

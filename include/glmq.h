@@ -119,6 +119,28 @@ GLMQ_API glmq_status glmq_gemm(const void* X, int64_t M, const void* packed, con
 GLMQ_API glmq_status glmq_gemm_decode(const void* X, int64_t M, const void* packed, const void* scale,
                              int64_t N, int64_t K, int bits, void* Y, void* stream);
 
+/*
+ * glmq_gemm_decode with a prefetch hint for the NEXT decode call on the same stream
+ * (a decode step runs the layers' projections back to back, and a layer's weights do
+ * not depend on the previous layer's output). Y is computed exactly as by
+ * glmq_gemm_decode (same kernel and plan; the hint only adds L2 prefetches).
+ *   next_packed in : codes of the next call's weight, uint8 [next_N, next_K*bits/8], same
+ *                    bits as this call, 16-byte aligned; NULL = no hint (plain
+ *                    glmq_gemm_decode)
+ *   next_M         : the next call's token count, 1..GLMQ_DECODE_MAX_M
+ *   next_N, next_K : the next call's shape (limits as glmq_gemm)
+ * While this call's pipeline drains, its kernel prefetches into L2 the weight tiles the
+ * next call's kernel loads first (the first ring fill of each of its CTAs). Only reads
+ * of next_packed are issued, and only as L2 prefetches; nothing is written. The hint
+ * pays when the next call follows directly (no other large traffic in between).
+ * Errors: as glmq_gemm_decode; GLMQ_ERR_BAD_SHAPE for next_M outside 1..16, next_N < 1
+ * or a bad next_K; GLMQ_ERR_BAD_BITS never (bits is shared); GLMQ_ERR_MISALIGNED for an
+ * unaligned next_packed.
+ */
+GLMQ_API glmq_status glmq_gemm_decode_prefetch(const void* X, int64_t M, const void* packed, const void* scale,
+                                               int64_t N, int64_t K, int bits, void* Y, const void* next_packed,
+                                               int64_t next_M, int64_t next_N, int64_t next_K, void* stream);
+
 /* glmq_gemm forced onto the tensor-core prefill kernel (any M >= 0). */
 GLMQ_API glmq_status glmq_gemm_prefill(const void* X, int64_t M, const void* packed, const void* scale,
                               int64_t N, int64_t K, int bits, void* Y, void* stream);

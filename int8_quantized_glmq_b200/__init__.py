@@ -14,6 +14,7 @@ from ._binding import (  # noqa: F401
     gemm_fused,
     gemm_zp,
     gemm_decode,
+    gemm_decode_prefetch,
     gemm_prefill,
     kernel_launches,
     last_device_error,

@@ -46,6 +46,8 @@ SIGNATURES = {
     "glmq_gemm": (ctypes.c_int, [_vp, _c_int64, _vp, _vp, _c_int64, _c_int64, ctypes.c_int, _vp, _vp]),
     "glmq_gemm_decode": (ctypes.c_int, [_vp, _c_int64, _vp, _vp, _c_int64, _c_int64, ctypes.c_int, _vp, _vp]),
     "glmq_gemm_prefill": (ctypes.c_int, [_vp, _c_int64, _vp, _vp, _c_int64, _c_int64, ctypes.c_int, _vp, _vp]),
+    "glmq_gemm_decode_prefetch": (ctypes.c_int, [_vp, _c_int64, _vp, _vp, _c_int64, _c_int64, ctypes.c_int, _vp,
+                                                 _vp, _c_int64, _c_int64, _c_int64, _vp]),
     "glmq_gemm_decode_noalloc": (ctypes.c_int, [_vp, _c_int64, _vp, _vp, _c_int64, _c_int64, ctypes.c_int, _vp,
                                                 _vp]),
     "glmq_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -131,6 +133,12 @@ def raw_gemm(X: int, M: int, packed: int, scale: int, N: int, K: int, bits: int,
     fn = {"auto": lib().glmq_gemm, "decode": lib().glmq_gemm_decode, "prefill": lib().glmq_gemm_prefill,
           "decode_noalloc": lib().glmq_gemm_decode_noalloc}[route]
     return fn(X, M, packed, scale, N, K, bits, Y, stream)
+
+
+def raw_gemm_decode_prefetch(X: int, M: int, packed: int, scale: int, N: int, K: int, bits: int, Y: int,
+                             next_packed: int, next_M: int, next_N: int, next_K: int, stream: int = 0) -> int:
+    return lib().glmq_gemm_decode_prefetch(X, M, packed, scale, N, K, bits, Y, next_packed, next_M, next_N, next_K,
+                                           stream)
 
 
 def kernel_launches() -> int:
@@ -289,6 +297,30 @@ def gemm_zp(X, packed, scale, zero, stream=None, out=None):
 
 def gemm_decode(X, packed, scale, bits: int = 4, stream=None, out=None):
     return gemm(X, packed, scale, bits, stream, out, route="decode")
+
+
+def gemm_decode_prefetch(X, packed, scale, bits: int = 4, next_packed=None, next_M: int = 1, stream=None, out=None):
+    """glmq_gemm_decode_prefetch: the decode GEMM (M <= 16), which also prefetches into L2
+    the first weight tiles of the next decode call (``next_packed``, same bits, called
+    with ``next_M`` tokens). Y is computed exactly as by :func:`gemm_decode`."""
+    torch = _torch()
+    _require(X, torch.float16, 2, "X")
+    _require(packed, torch.uint8, 2, "packed")
+    _require(scale, torch.float16, 1, "scale")
+    M, K = X.shape
+    N = packed.shape[0]
+    if packed.shape[1] * 8 != K * bits or scale.shape[0] != N:
+        raise ValueError("packed/scale shapes do not match X and bits")
+    nptr, nN, nK = 0, 0, 0
+    if next_packed is not None:
+        _require(next_packed, torch.uint8, 2, "next_packed")
+        nptr, nN, nK = next_packed.data_ptr(), next_packed.shape[0], next_packed.shape[1] * 8 // bits
+    Y = torch.empty((M, N), dtype=torch.float16, device=X.device) if out is None else out
+    with _on_device(X):
+        st = raw_gemm_decode_prefetch(X.data_ptr(), M, packed.data_ptr(), scale.data_ptr(), N, K, bits, Y.data_ptr(),
+                                      nptr, next_M, nN, nK, _stream_ptr(stream))
+    _check(st, "glmq_gemm_decode_prefetch")
+    return Y
 
 
 def gemm_prefill(X, packed, scale, bits: int = 4, stream=None, out=None):

@@ -92,6 +92,14 @@ struct DecodeArgs {
   int parts;
   int tiles;
   int units;          // parts * tiles
+  // The next decode call on the stream (glmq_gemm_decode_prefetch), planned the same
+  // way: while this call's ring drains, its producer prefetches into L2 the stages the
+  // next call's CTAs load first. nxt_grid == 0: no next call.
+  int nxt_grid;
+  int nxt_units;
+  int nxt_tiles;
+  int nxt_KPP;
+  int nxt_K;
 };
 
 // INT4, biased form: one packed word (8 codes, k = 0..7 of the word) -> 4 half2
@@ -130,6 +138,14 @@ __device__ __forceinline__ void tma_load_2d_hint(void* smem_dst, const CUtensorM
       "[%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_u32(smem_dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar)), "l"(policy)
       : "memory");
+}
+
+// L2 prefetch of one TMA box (a hint: no shared memory is written, nothing waits).
+__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* map, int x, int y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(x), "r"(y)
+               : "memory");
 }
 
 // Index (in 16-byte units) of the activation unit read by lane (n, c) for unit jj of
@@ -270,7 +286,8 @@ __device__ __forceinline__ void stage_activations(const __half* __restrict__ X, 
 // ---------------------------------------------------------------- the kernel
 template <class C>
 __global__ void __launch_bounds__(kDecodeThreads, 1)
-    decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const DecodeArgs a) {
+    decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_next,
+                  const DecodeArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* wring = smem;
@@ -341,6 +358,26 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
           armed[stage] = phase + 1;
           tma_load_2d_hint(wring + stage * kDecodeStageBytes, &tmap_w, xb0, t * kDecodeRows, &full[stage], pol);
           if (++stage == kDecodeStages) { stage = 0; phase ^= 1; }
+        }
+      }
+      if (ok && a.nxt_grid > 0) {
+        // Every load of this CTA is issued; its consumers still work through up to a
+        // full ring. Meanwhile bring the next call's first ring fill into L2: next CTA b
+        // (b = this CTA, this CTA + G, ...) starts with the first kDecodeStages stages
+        // of its units. The next call's weights do not depend on this call's output.
+        for (int b = blockIdx.x; b < a.nxt_grid; b += G) {
+          const int ub = static_cast<int>((static_cast<long long>(b) * a.nxt_units) / a.nxt_grid);
+          const int ue = static_cast<int>((static_cast<long long>(b + 1) * a.nxt_units) / a.nxt_grid);
+          int left = kDecodeStages;
+          for (int u = ub; u < ue && left > 0; ++u) {
+            const int p = u / a.nxt_tiles;
+            const int t = u - p * a.nxt_tiles;
+            const int pk0 = p * a.nxt_KPP;
+            const int plen = min(a.nxt_KPP, a.nxt_K - pk0);
+            const int nst = (plen + C::SK - 1) / C::SK;
+            for (int ks = 0; ks < nst && left > 0; ++ks, --left)
+              tma_prefetch_2d(&tmap_next, (pk0 + ks * C::SK) / C::KPB, t * kDecodeRows);
+          }
         }
       }
       // never leave while TMA writes into this CTA's shared memory may be in flight

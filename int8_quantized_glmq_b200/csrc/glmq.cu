@@ -261,11 +261,14 @@ glmq_status decode_scratch(size_t ws_elems, float** out) {
   return GLMQ_OK;
 }
 
-// Fused epilogue of a GEMM call (epilogue.cuh): optional bias, optional GeGLU.
+// Per-call options of a GEMM call: the fused epilogue (epilogue.cuh: optional bias,
+// optional GeGLU), zero-point codes, and the decode kernel's next-call prefetch hint.
 struct Epi {
   const __half* bias = nullptr;
   int geglu = 0;
   const uint8_t* zero = nullptr;   // zero-point INT4 codes: per-row zero points
+  const void* next_packed = nullptr;   // glmq_gemm_decode_prefetch: the next call's weights
+  int next_M = 0, next_N = 0, next_K = 0;
 };
 
 // Launches finalize_epilogue_kernel: one thread per output column of every token row.
@@ -350,6 +353,16 @@ bool plan_decode(const DeviceInfo& dev, int N, int K, DecodePlan* pl) {
   return pl->smem <= dev.smem_optin;
 }
 
+// The decode plan of a call with M tokens (the kernel configuration launch_decode picks).
+template <int BITS>
+bool plan_decode_for(const DeviceInfo& dev, int M, int N, int K, DecodePlan* pl) {
+  if (M <= 1) return plan_decode<DecodeCfg<BITS, 1>>(dev, N, K, pl);
+  if (M <= 2) return plan_decode<DecodeCfg<BITS, 2>>(dev, N, K, pl);
+  if (M <= 4) return plan_decode<DecodeCfg<BITS, 4>>(dev, N, K, pl);
+  if (M <= 8) return plan_decode<DecodeCfg<BITS, 8>>(dev, N, K, pl);
+  return plan_decode<DecodeCfg<BITS, 16>>(dev, N, K, pl);
+}
+
 template <class C>
 glmq_status launch_decode_cfg(const DeviceInfo& dev, const void* X, int M, const void* packed, const void* scale,
                               int N, int K, void* Y, cudaStream_t s, const Epi& e = Epi()) {
@@ -360,6 +373,16 @@ glmq_status launch_decode_cfg(const DeviceInfo& dev, const void* X, int M, const
   glmq_status st = make_map_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, packed, row_bytes, N, row_bytes, kDecodeSegB,
                                kDecodeRows, CU_TENSOR_MAP_SWIZZLE_128B);
   if (st != GLMQ_OK) return st;
+  // next-call hint: the same map and plan the next decode call will use
+  CUtensorMap tn = tw;
+  DecodePlan npl = {};
+  if (e.next_packed) {
+    if (!plan_decode_for<C::kBits>(dev, e.next_M, e.next_N, e.next_K, &npl)) return GLMQ_ERR_BAD_SHAPE;
+    const uint64_t nrow = uint64_t(e.next_K) / C::KPB;
+    st = make_map_2d(&tn, CU_TENSOR_MAP_DATA_TYPE_UINT8, e.next_packed, nrow, e.next_N, nrow, kDecodeSegB, kDecodeRows,
+                     CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st != GLMQ_OK) return st;
+  }
   DecodeArgs a;
   a.X = static_cast<const __half*>(X);
   a.scale = static_cast<const __half*>(scale);
@@ -375,9 +398,14 @@ glmq_status launch_decode_cfg(const DeviceInfo& dev, const void* X, int M, const
   a.parts = pl.parts;
   a.tiles = pl.tiles;
   a.units = pl.units;
+  a.nxt_grid = e.next_packed ? npl.grid : 0;
+  a.nxt_units = npl.units;
+  a.nxt_tiles = npl.tiles;
+  a.nxt_KPP = npl.KPP;
+  a.nxt_K = e.next_K;
   if (pl.parts > 1 && (st = decode_scratch(static_cast<size_t>(M) * N, &a.ws)) != GLMQ_OK) return st;
   if ((st = allow_smem(decode_kernel<C>, pl.smem)) != GLMQ_OK) return st;
-  if ((st = launch_pdl(decode_kernel<C>, dim3(pl.grid), dim3(kDecodeThreads), pl.smem, s, tw, a)) != GLMQ_OK)
+  if ((st = launch_pdl(decode_kernel<C>, dim3(pl.grid), dim3(kDecodeThreads), pl.smem, s, tw, tn, a)) != GLMQ_OK)
     return st;
   if (pl.parts > 1) {
     st = (e.bias || e.geglu) ? launch_finalize_epi(a.ws, a.scale, e, a.Y, M, N, s)
@@ -579,6 +607,7 @@ glmq_status launch_decode_noalloc_cfg(const DeviceInfo& dev, const void* X, int 
   a.bias = nullptr;
   a.geglu = 0;
   a.zero = nullptr;
+  a.nxt_grid = a.nxt_units = a.nxt_tiles = a.nxt_KPP = a.nxt_K = 0;
   cudaError_t e;
   if (pl.parts > 1) {
     if ((st = noalloc_scratch(&a.ws)) != GLMQ_OK) return st;
@@ -587,7 +616,7 @@ glmq_status launch_decode_noalloc_cfg(const DeviceInfo& dev, const void* X, int 
       return cuda_fail(e);
   }
   if ((st = allow_smem(decode_kernel<C>, pl.smem)) != GLMQ_OK) return st;
-  if ((st = launch_pdl(decode_kernel<C>, dim3(pl.grid), dim3(kDecodeThreads), pl.smem, s, tw, a)) != GLMQ_OK)
+  if ((st = launch_pdl(decode_kernel<C>, dim3(pl.grid), dim3(kDecodeThreads), pl.smem, s, tw, tw, a)) != GLMQ_OK)
     return st;
   if (pl.parts > 1) {
     if ((st = launch_finalize(a.ws, a.scale, a.Y, M, N, s)) != GLMQ_OK) return st;
@@ -672,6 +701,23 @@ glmq_status glmq_gemm(const void* X, int64_t M, const void* packed, const void* 
 glmq_status glmq_gemm_decode(const void* X, int64_t M, const void* packed, const void* scale, int64_t N, int64_t K,
                              int bits, void* Y, void* stream) {
   return gemm_entry(Route::kDecode, X, M, packed, scale, N, K, bits, Y, stream);
+}
+
+glmq_status glmq_gemm_decode_prefetch(const void* X, int64_t M, const void* packed, const void* scale, int64_t N,
+                                      int64_t K, int bits, void* Y, const void* next_packed, int64_t next_M,
+                                      int64_t next_N, int64_t next_K, void* stream) {
+  Epi e;
+  if (next_packed) {
+    if (next_M < 1 || next_M > GLMQ_DECODE_MAX_M || next_N < 1) return GLMQ_ERR_BAD_SHAPE;
+    glmq_status st = check_common(next_N, next_K, bits);
+    if (st != GLMQ_OK) return st;
+    if (!aligned16(next_packed)) return GLMQ_ERR_MISALIGNED;
+    e.next_packed = next_packed;
+    e.next_M = static_cast<int>(next_M);
+    e.next_N = static_cast<int>(next_N);
+    e.next_K = static_cast<int>(next_K);
+  }
+  return gemm_entry(Route::kDecode, X, M, packed, scale, N, K, bits, Y, stream, e);
 }
 
 glmq_status glmq_gemm_prefill(const void* X, int64_t M, const void* packed, const void* scale, int64_t N, int64_t K,

@@ -135,3 +135,19 @@ def test_zero_point_entry_points_validate_before_device_work():
     assert B.raw_gemm_zp(ALIGNED, 4, ALIGNED, ALIGNED, 0, 8, 64, ALIGNED) == B.ERR_NULL_POINTER
     assert B.raw_gemm_zp(ALIGNED, 4, ALIGNED, ALIGNED, ALIGNED, 8, 96, ALIGNED) == B.ERR_BAD_SHAPE
     assert B.raw_gemm_zp(0, 0, ALIGNED, ALIGNED, 0, 8, 64, 0) == B.OK
+
+
+def test_decode_prefetch_entry_validates_before_device_work():
+    g = lambda **kw: B.raw_gemm_decode_prefetch(
+        kw.get("X", ALIGNED), kw.get("M", 4), ALIGNED, ALIGNED, kw.get("N", 8), kw.get("K", 64), kw.get("bits", 4),
+        kw.get("Y", ALIGNED), kw.get("NP", ALIGNED), kw.get("NM", 1), kw.get("NN", 8), kw.get("NK", 64), 0)
+    assert g(NM=0) == B.ERR_BAD_SHAPE
+    assert g(NM=17) == B.ERR_BAD_SHAPE                 # the next call must be a decode call too
+    assert g(NN=0) == B.ERR_BAD_SHAPE
+    assert g(NK=96) == B.ERR_BAD_SHAPE
+    assert g(NP=ALIGNED + 8) == B.ERR_MISALIGNED
+    assert g(bits=3) == B.ERR_BAD_BITS
+    assert g(M=17) == B.ERR_BAD_SHAPE                  # this call is a decode call
+    assert g(X=0) == B.ERR_NULL_POINTER
+    assert g(M=0, X=0, Y=0) == B.OK                    # empty problem: nothing enqueued
+    assert g(NP=0, NM=0, NN=0, NK=0, M=0, X=0, Y=0) == B.OK   # no hint: the hint fields are ignored

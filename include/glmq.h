@@ -39,8 +39,13 @@
  *     M == 0 is an empty problem: GLMQ_OK, nothing is enqueued, pointers may
  *     be NULL.
  *   - Inputs are finite fp16 values; NaN or Inf inputs are outside the contract.
- *   - Calls that overlap on the GPU and write the same output race; distinct
- *     calls share no library-owned state except the device status word.
+ *   - Calls that overlap on the GPU and write the same output race.
+ *   - Library-owned device state, one instance per device: the fp32 scratch of
+ *     GEMM calls whose tiles are split over K parts (see glmq_gemm), the skinny
+ *     kernel's activation image (16 < M <= 64), the fixed array of
+ *     glmq_gemm_decode_noalloc, and the device status word. GEMM calls that use
+ *     one of these buffers must not overlap on the GPU: issue them on one stream,
+ *     or order the streams. Quantize calls use none of them.
  */
 #ifndef GLMQ_H
 #define GLMQ_H

@@ -4,7 +4,7 @@ The GLM-130B paper card ("Paper vs code") runs the INT4 model 4-way model-parall
 These tests check the host side of that split with the oracle standing in for the
 local GEMM (the library's GEMM needs a GPU; its own parity is covered by the GPU
 tests): shard slicing, bias placement, the GeGLU-packed column split, and the
-all-gather / all-reduce run by two gloo ranks on 127.0.0.1.
+all-gather / all-reduce run by two and by four gloo ranks on 127.0.0.1.
 """
 import os
 import socket
@@ -154,15 +154,16 @@ def _rank_main(rank, world, port, out_q):
         dist.destroy_process_group()
 
 
-def test_two_gloo_ranks_gather_and_reduce():
+@pytest.mark.parametrize("world", [2, 4])           # 4: the INT4 model's 4-way split
+def test_gloo_ranks_gather_and_reduce(world):
     import torch.multiprocessing as mp
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, q)) for r in range(2)]
+    procs = [ctx.Process(target=_rank_main, args=(r, world, port, q)) for r in range(world)]
     for pr in procs:
         pr.start()
-    got = sorted((q.get(timeout=120) for _ in range(2)), key=lambda t: t[0])
+    got = sorted((q.get(timeout=120) for _ in range(world)), key=lambda t: t[0])
     for pr in procs:
         pr.join(timeout=60)
         if pr.is_alive():
@@ -176,11 +177,13 @@ def test_two_gloo_ranks_gather_and_reduce():
     b = gaussian_fp16((1, N), 0.5, 62)[0]
     X = gaussian_fp16((3, K), 1.0, 63)
     ref = oracle.linear_bias_forward(X, pn, sn, 4, b)
-    # the reduced result, computed here from the two ranks' partials
-    half = K // 2
-    part0 = oracle.linear_bias_forward(X[:, :half], pn[:, :half // 2], sn, 4, b).astype(np.float32)
-    part1 = oracle.linear_forward(X[:, half:], pn[:, half // 2:], sn, 4).astype(np.float32)
-    expect_row = (part0 + part1).astype(np.float16)
+    # the reduced result, computed here from the ranks' fp16 partials (rank 0 adds the bias)
+    kl = K // world
+    acc = oracle.linear_bias_forward(X[:, :kl], pn[:, :kl // 2], sn, 4, b).astype(np.float32)
+    for r in range(1, world):
+        acc += oracle.linear_forward(X[:, r * kl:(r + 1) * kl], pn[:, r * kl // 2:(r + 1) * kl // 2], sn,
+                                     4).astype(np.float32)
+    expect_row = acc.astype(np.float16)
     for _, Yc, Yr in got:
         assert np.array_equal(Yc.view(np.uint16), ref.view(np.uint16))        # column: identical
         assert np.array_equal(Yr.view(np.uint16), expect_row.view(np.uint16))  # row: fp32 sum of partials

@@ -37,7 +37,7 @@ sys.path.insert(0, ROOT)
 METRIC = "W4A16 GEMM weight GB/s (decode) and TFLOP/s (prefill) vs B200 roofline"
 HIDDEN = 12288
 DECODE_MS = (1, 4, 16)
-EVENT_EVERY = 4          # timed steps that carry per-launch timing events: 0, 4, 8, ...
+EVENT_STEPS = 4          # steps of the separate event-carrying graph (per-launch shares)
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 
@@ -281,71 +281,78 @@ def run_decode(args, world, rank, local):
         return glmq.gemm_decode_prefetch(X, quant[n][0], quant[n][1], bits, next_packed=quant[nn][0], next_M=Mn,
                                          out=Y)
 
-    # The timed steps are captured into one CUDA graph: K steps of the 12 public calls.
-    # Every EVENT_EVERY-th step carries timing-event record nodes (external events)
-    # around each call; those give the per-launch device times of the roofline. The
-    # other steps run as a plain chain of kernels (event nodes between kernels add
-    # gaps and cut the programmatic-launch edges, so they are kept to a sample).
+    # The timed steps are captured into one CUDA graph: K steps of the 12 public calls,
+    # nothing else between the kernels (so the programmatic-launch edges between them
+    # stay intact). The per-launch split of the step comes from a separate graph of
+    # EVENT_STEPS steps with timing-event record nodes (external events) around every
+    # call; event nodes add gaps and cut the programmatic-launch edges, so those
+    # durations are used only as shares of the step, scaled to the event-free step time.
     # The eager calls before capture size the library's scratch and set attributes.
     for j in range(len(launches)):
         call(j)
     torch.cuda.synchronize()
     cap_stream = torch.cuda.Stream()
 
-    def capture(n_steps, with_events, hint=True):
+    def capture(n_steps, with_events=False, hint=True):
         g = torch.cuda.CUDAGraph()
-        sampled = [it for it in range(n_steps) if with_events and it % EVENT_EVERY == 0]
-        evs = {it: [(torch.cuda.Event(enable_timing=True, external=True),
-                     torch.cuda.Event(enable_timing=True, external=True)) for _ in launches] for it in sampled}
-        edge = (torch.cuda.Event(enable_timing=True, external=True),
-                torch.cuda.Event(enable_timing=True, external=True)) if with_events else None
+        evs = [[(torch.cuda.Event(enable_timing=True, external=True),
+                 torch.cuda.Event(enable_timing=True, external=True)) for _ in launches]
+               for _ in range(n_steps)] if with_events else None
         n0 = glmq.kernel_launches()
         with torch.cuda.graph(g, stream=cap_stream):
-            if with_events:
-                edge[0].record()
             for it in range(n_steps):
-                for j, (M, n) in enumerate(launches):
-                    if it in evs:
+                for j in range(len(launches)):
+                    if with_events:
                         evs[it][j][0].record()
                     call(j, hint)
-                    if it in evs:
+                    if with_events:
                         evs[it][j][1].record()
-            if with_events:
-                edge[1].record()
-        return g, evs, edge, glmq.kernel_launches() - n0
+        return g, evs, glmq.kernel_launches() - n0
 
-    warm_graph, _, _, _ = capture(args.warmup, False)
-    timed_graph, ev, (t0, t1), kernels_timed = capture(args.steps, True)
+    def timed_replay(graph):
+        """Device seconds of one replay, CUDA events on the launching stream around it."""
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(world)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        graph.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        return e0.elapsed_time(e1) / 1e3
+
     stream = torch.cuda.current_stream()
+    warm_graph, _, _ = capture(args.warmup)
+    timed_graph, _, kernels_timed = capture(args.steps)
     warm_graph.replay()
     torch.cuda.synchronize()
 
     clocks = ClockSampler(local)
     clocks.start()
-    barrier(world)
-    torch.cuda.synchronize()
-    timed_graph.replay()
-    torch.cuda.synchronize()
-    barrier(world)
+    elapsed = timed_replay(timed_graph)
     clk = clocks.stop()
     gpu_launches = kernels_timed
-    elapsed = t0.elapsed_time(t1) / 1e3
-    per_launch_s = [sum(ev[it][j][0].elapsed_time(ev[it][j][1]) for it in ev) / 1e3 / len(ev)
-                    for j in range(len(launches))]
     value, elapsed_max = whole_job_rate(weight_bytes / 1e9, args.steps, elapsed, world)
+    step_s = elapsed_max / args.steps
     del warm_graph, timed_graph
 
+    # per-launch shares of the step (event-timed, separate graph)
+    ev_graph, ev, _ = capture(EVENT_STEPS, with_events=True)
+    ev_graph.replay()
+    torch.cuda.synchronize()
+    ev_graph.replay()
+    torch.cuda.synchronize()
+    ev_s = [sum(ev[it][j][0].elapsed_time(ev[it][j][1]) for it in range(EVENT_STEPS)) / 1e3 / EVENT_STEPS
+            for j in range(len(launches))]
+    per_launch_s = [t / sum(ev_s) * step_s for t in ev_s]
+    del ev_graph, ev
+
     # the same step with plain decode calls (no next-call hint), for comparison
-    # (the returned events stay referenced until the graph is gone: its event nodes use them)
-    plain_graph, plain_ev, (p0, p1), _ = capture(args.steps, True, hint=False)
+    plain_graph, _, _ = capture(args.steps, hint=False)
     plain_graph.replay()
     torch.cuda.synchronize()
-    barrier(world)
-    plain_graph.replay()
-    torch.cuda.synchronize()
-    barrier(world)
-    plain_value, _ = whole_job_rate(weight_bytes / 1e9, args.steps, p0.elapsed_time(p1) / 1e3, world)
-    del plain_graph, plain_ev
+    plain_value, _ = whole_job_rate(weight_bytes / 1e9, args.steps, timed_replay(plain_graph), world)
+    del plain_graph
     extras["decode_step_without_prefetch_hint_gbs"] = round(plain_value, 2)
 
     # e2e through the public API: pinned host X in, pinned host Y out, every step
@@ -396,21 +403,30 @@ def run_decode(args, world, rank, local):
     e2e_value, _ = whole_job_rate(weight_bytes / 1e9, args.steps, a0.elapsed_time(a1) / 1e3, world)
     del e2e_graph
 
-    kern_time = sum(per_launch_s)
-    achieved = alg_bytes / kern_time / 1e9
+    # Dominant kernel: decode_kernel, with the finalize pass of the calls whose tiles are
+    # split over K parts (one "launch" = one public call). Its time is the event-free
+    # step time, so achieved is algorithmic bytes per step / step time: a lower bound on
+    # the decode kernel's own rate (the step also holds the launches' gaps).
+    achieved = alg_bytes / step_s / 1e9
     ratio = profile_traffic_ratio("decode_int4_glm_shapes")
-    roofline = {"kernel": "decode_kernel (INT4, M in {1,4,16})", "bound": "hbm", "achieved": round(achieved, 1),
+    roofline = {"kernel": "decode_kernel (+ decode_finalize_kernel on split tiles), INT4, M in {1,4,16}",
+                "bound": "hbm", "achieved": round(achieved, 1),
                 "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
                 "peak_source": peaks["source"],
                 "traffic": (round(ratio * alg_bytes / len(launches)) if ratio else None),
-                "algorithmic_bytes_per_launch": round(alg_bytes / len(launches))}
+                "algorithmic_bytes_per_launch": round(alg_bytes / len(launches)),
+                "launch_time": "event-free step time / 12 calls"}
     per_launch = {f"{n}/M={M}": {"us": round(per_launch_s[j] * 1e6, 2),
                                  "gbs": round((quant[n][0].numel() + quant[n][1].numel() * 2 + xs[(M, n)].numel() * 2
                                                + ys[(M, n)].numel() * 2) / per_launch_s[j] / 1e9, 1)}
                   for j, (M, n) in enumerate(launches)}
     extras["decode_per_launch"] = per_launch
-    extras["quantize_int4"] = {k: {"us": round(v["us"], 1), "gbs": round(v["gbs"], 1)} for k, v in qstats.items()}
-    return {
+    extras["quantize_int4"] = {k: {"us": round(v["us"], 1), "gbs": round(v["gbs"], 1),
+                                   "frac_hbm": round(v["gbs"] / peaks["hbm_gbs"], 4)} for k, v in qstats.items()}
+    if not args.no_extras and world == 1:
+        del xs, ys, hx, hy, xbuf, ybuf
+        extras["sweep_70_layers_int4"] = sweep_summary(torch, glmq, peaks)
+    result = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(elapsed_max / args.steps * 1e3, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "fp16", "weight_dtype": "int4", "data": "synthetic",
@@ -426,6 +442,35 @@ def run_decode(args, world, rank, local):
         "clocks": clk,
         "extras": extras,
     }
+    result["highlights"] = highlights(result, peaks)
+    return result
+
+
+def highlights(res, peaks):
+    """The headline figures of the extras, repeated compactly at the end of the line."""
+    ex = res.get("extras", {})
+    h = {"decode_step_gbs": res["value"], "decode_frac_hbm": res["roofline"]["frac"]}
+    pre = ex.get("prefill_int4_m2048")
+    if pre:
+        h["prefill_int4_m2048_tflops"] = {k: v["tflops"] for k, v in pre.items()}
+        h["prefill_frac_burst_min"] = min(v["frac_burst"] for v in pre.values())
+    m64 = ex.get("int4_m64")
+    if m64:
+        h["int4_m64_frac_binding_roof"] = {k: v["frac_binding_roof"] for k, v in m64.items()}
+    i8 = ex.get("int8")
+    if i8:
+        h["int8_m64_frac_hbm"] = {k: v["M=64"].get("frac_hbm") for k, v in i8.items()}
+    q = ex.get("quantize_int4")
+    if q:
+        h["quantize_int4_frac_hbm"] = {k: v["frac_hbm"] for k, v in q.items()}
+    sw = ex.get("sweep_70_layers_int4")
+    if sw and "tokens_per_s" in sw:
+        h["sweep_70_layers"] = {"tokens_per_s": sw["tokens_per_s"], "frac_hbm": sw["frac_hbm"],
+                                "quantize_all_ms": sw["quantize_all_ms"]}
+    per = ex.get("decode_per_launch")
+    if per:
+        h["decode_min_call_frac_hbm"] = round(min(v["gbs"] for v in per.values()) / peaks["hbm_gbs"], 4)
+    return h
 
 
 def run_extras(torch, glmq, W16, quant, peaks):
@@ -442,6 +487,27 @@ def run_extras(torch, glmq, W16, quant, peaks):
         tf = 2.0 * 2048 * N * K / t / 1e12
         out["prefill_int4_m2048"][name] = {"us": round(t * 1e6, 1), "tflops": round(tf, 1),
                                            "frac_burst": round(tf / peaks["bf16_tflops"], 4)}
+        del X, Y
+    # INT4 at M=64 (the skinny tensor-core kernel): arithmetic intensity ~249 flop/B, at the
+    # ridge of the roofline, so both roofs are reported with the one that binds. L2 is
+    # flushed before each timed call (attn-out's 75 MB of codes would otherwise stay in L2).
+    out["int4_m64"] = {}
+    for name in PROJECTION_ORDER:
+        N, K = GLM_PROJECTIONS[name]
+        packed, scale = quant[name]
+        g = torch.Generator(device="cuda").manual_seed(3100)
+        X = torch.randn((64, K), generator=g, device="cuda", dtype=torch.float32).half()
+        Y = torch.empty((64, N), dtype=torch.float16, device="cuda")
+        t = time_launches_cold(torch, lambda: glmq.gemm(X, packed, scale, 4, out=Y), 5)
+        nbytes = packed.numel() + scale.numel() * 2 + X.numel() * 2 + Y.numel() * 2
+        flops = 2.0 * 64 * N * K
+        t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
+        t_tc = flops / (peaks["bf16_tflops"] * 1e12)
+        out["int4_m64"][name] = {"us": round(t * 1e6, 1), "weight_gbs": round(packed.numel() / t / 1e9, 1),
+                                 "tflops": round(flops / t / 1e12, 1), "t_hbm_us": round(t_hbm * 1e6, 1),
+                                 "t_tensor_us": round(t_tc * 1e6, 1),
+                                 "binding": "hbm" if t_hbm >= t_tc else "tensor",
+                                 "frac_binding_roof": round(max(t_hbm, t_tc) / t, 4)}
         del X, Y
     # FFN-up with the fused GeGLU epilogue (plus an fp16 bias) against the plain call
     N, K = GLM_PROJECTIONS["ffn_up"]
@@ -511,9 +577,12 @@ def run_extras(torch, glmq, W16, quant, peaks):
             g = torch.Generator(device="cuda").manual_seed(4000 + M)
             X = torch.randn((M, K), generator=g, device="cuda", dtype=torch.float32).half()
             Y = torch.empty((M, N), dtype=torch.float16, device="cuda")
-            t = time_launches(torch, lambda: glmq.gemm(X, p8, s8, 8, out=Y), 5)
+            timer = time_launches if M == 2048 else time_launches_cold
+            t = timer(torch, lambda: glmq.gemm(X, p8, s8, 8, out=Y), 5)
             res[f"M={M}"] = {"us": round(t * 1e6, 1), "weight_gbs": round(N * K / t / 1e9, 1),
                              "tflops": round(2.0 * M * N * K / t / 1e12, 1)}
+            if M == 64:
+                res["M=64"]["frac_hbm"] = round(N * K / t / 1e9 / peaks["hbm_gbs"], 4)
         out["int8"][name] = res
         del p8, s8
     return out
@@ -590,85 +659,136 @@ def cpu_baseline(budget_s: float = 12.0):
 
 
 # ----------------------------------------------------------------------------- sweep
+SWEEP_LAYERS = 70
+
+
+def sweep_weight(torch, layer: int, proj_index: int, out):
+    """Fills out with the fp16 weights of one projection of the layer sweep, N(0, 0.02),
+    seeded by (layer, projection): seed 10000 + 4 * layer + proj_index."""
+    g = torch.Generator(device="cuda").manual_seed(10000 + 4 * layer + proj_index)
+    return out.normal_(0.0, 0.02, generator=g)
+
+
+class Sweep:
+    """The INT4 layer sweep: every projection of every layer quantized once (one-shot,
+    layer by layer, each call timed) and resident in HBM, plus one CUDA graph that runs
+    the M=1 decode GEMM through all of them in layer order. Each projection p reads the
+    same seeded activation row xs[p]; the outputs of the layers in ``keep`` go to their
+    own buffers (kept[(layer, name)]) so they can be checked after a replay."""
+
+    def __init__(self, torch, glmq, layers: int, keep=()):
+        from inputs import GLM_PROJECTIONS, PROJECTION_ORDER
+        self.layers = layers
+        self.quant = []
+        self.qtime = 0.0
+        self.qbytes = 0
+        wbuf = {n: torch.empty(GLM_PROJECTIONS[n], dtype=torch.float16, device="cuda") for n in PROJECTION_ORDER}
+        s = torch.cuda.current_stream()
+        for layer in range(layers):
+            row = []
+            for p, n in enumerate(PROJECTION_ORDER):
+                N, K = GLM_PROJECTIONS[n]
+                sweep_weight(torch, layer, p, wbuf[n])
+                packed = torch.empty((N, K // 2), dtype=torch.uint8, device="cuda")
+                scale = torch.empty((N,), dtype=torch.float16, device="cuda")
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(s)
+                glmq.quantize(wbuf[n], 4, out=(packed, scale))
+                e1.record(s)
+                torch.cuda.synchronize()
+                self.qtime += e0.elapsed_time(e1) / 1e3
+                self.qbytes += N * K * 2 + N * K // 2 + N * 2
+                row.append((packed, scale))
+            self.quant.append(row)
+        del wbuf
+        torch.cuda.empty_cache()
+        self.xs = {}
+        for p, n in enumerate(PROJECTION_ORDER):
+            g = torch.Generator(device="cuda").manual_seed(20000 + p)
+            self.xs[n] = torch.randn((1, GLM_PROJECTIONS[n][1]), generator=g, device="cuda").half()
+        self.ys = {n: torch.empty((1, GLM_PROJECTIONS[n][0]), dtype=torch.float16, device="cuda")
+                   for n in PROJECTION_ORDER}
+        self.kept = {(layer, n): torch.full((1, GLM_PROJECTIONS[n][0]), float("nan"), dtype=torch.float16,
+                                            device="cuda")
+                     for layer in keep for n in PROJECTION_ORDER}
+        self.order = [(layer, p, n) for layer in range(layers) for p, n in enumerate(PROJECTION_ORDER)]
+        self.wbytes = sum(q[0].numel() for row in self.quant for q in row)
+        cs = torch.cuda.Stream()
+        cs.wait_stream(s)
+        with torch.cuda.stream(cs):
+            for _ in range(2):
+                self._step(glmq)
+        torch.cuda.synchronize()
+        self.graph = torch.cuda.CUDAGraph()
+        n0 = glmq.kernel_launches()
+        with torch.cuda.graph(self.graph, stream=cs):
+            self._step(glmq)
+        self.kernels_per_replay = glmq.kernel_launches() - n0
+
+    def _step(self, glmq):
+        for layer, p, n in self.order:
+            out = self.kept.get((layer, n), self.ys[n])
+            glmq.gemm(self.xs[n], self.quant[layer][p][0], self.quant[layer][p][1], 4, out=out)
+
+    def time_replays(self, torch, steps: int, warmup: int, world: int = 1):
+        """Device seconds of `steps` replays (CUDA events on the current stream)."""
+        for _ in range(warmup):
+            self.graph.replay()
+        torch.cuda.synchronize()
+        barrier(world)
+        s = torch.cuda.current_stream()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(s)
+        for _ in range(steps):
+            self.graph.replay()
+        e1.record(s)
+        torch.cuda.synchronize()
+        barrier(world)
+        return e0.elapsed_time(e1) / 1e3
+
+
 def run_sweep(args, world, rank, local):
     """70 layers x 4 projections resident as INT4; M=1 decode through all 280 in one CUDA graph."""
     import torch
     import int8_quantized_glmq_b200 as glmq
-    from inputs import GLM_PROJECTIONS, PROJECTION_ORDER
 
-    layers = args.layers
-    bits = 4
-    quant = []
-    qtime = 0.0
-    qbytes = 0
-    wbuf = {n: torch.empty(GLM_PROJECTIONS[n], dtype=torch.float16, device="cuda") for n in PROJECTION_ORDER}
-    s = torch.cuda.current_stream()
-    for layer in range(layers):
-        row = []
-        for p, n in enumerate(PROJECTION_ORDER):
-            N, K = GLM_PROJECTIONS[n]
-            g = torch.Generator(device="cuda").manual_seed(10000 + 4 * layer + p)
-            wbuf[n].normal_(0.0, 0.02, generator=g)
-            packed = torch.empty((N, K // 2), dtype=torch.uint8, device="cuda")
-            scale = torch.empty((N,), dtype=torch.float16, device="cuda")
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(s)
-            glmq.quantize(wbuf[n], bits, out=(packed, scale))
-            e1.record(s)
-            torch.cuda.synchronize()
-            qtime += e0.elapsed_time(e1) / 1e3
-            qbytes += N * K * 2 + N * K // 2 + N * 2
-            row.append((packed, scale))
-        quant.append(row)
-    del wbuf
-    torch.cuda.empty_cache()
-    xs = {n: torch.randn((1, GLM_PROJECTIONS[n][1]), device="cuda").half() for n in PROJECTION_ORDER}
-    ys = {n: torch.empty((1, GLM_PROJECTIONS[n][0]), dtype=torch.float16, device="cuda") for n in PROJECTION_ORDER}
-    cs = torch.cuda.Stream()
-    cs.wait_stream(s)
-    with torch.cuda.stream(cs):
-        for _ in range(2):
-            for layer in range(layers):
-                for p, n in enumerate(PROJECTION_ORDER):
-                    glmq.gemm(xs[n], quant[layer][p][0], quant[layer][p][1], bits, out=ys[n])
-    torch.cuda.synchronize()
-    graph = torch.cuda.CUDAGraph()
-    n_capture0 = glmq.kernel_launches()
-    with torch.cuda.graph(graph, stream=cs):
-        for layer in range(layers):
-            for p, n in enumerate(PROJECTION_ORDER):
-                glmq.gemm(xs[n], quant[layer][p][0], quant[layer][p][1], bits, out=ys[n])
-    kernels_per_replay = glmq.kernel_launches() - n_capture0
-    for _ in range(args.warmup):
-        graph.replay()
-    torch.cuda.synchronize()
+    sw = Sweep(torch, glmq, args.layers)
     clocks = ClockSampler(local)
     clocks.start()
-    barrier(world)
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(s)
-    for _ in range(args.steps):
-        graph.replay()
-    e1.record(s)
-    torch.cuda.synchronize()
-    barrier(world)
+    el_local = sw.time_replays(torch, args.steps, args.warmup, world)
     clk = clocks.stop()
-    tok_s, el = whole_job_rate(1.0, args.steps, e0.elapsed_time(e1) / 1e3, world)
-    wbytes = sum(q[0].numel() for row in quant for q in row)
+    tok_s, el = whole_job_rate(1.0, args.steps, el_local, world)
     peaks = measured_peaks()
-    gbs = wbytes * args.steps / (el) / 1e9
-    del graph
-    return {"metric": "GLM-130B 70-layer INT4 decode sweep (M=1, 280 projections), tokens/s", "value": round(tok_s, 2),
-            "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": round(el / args.steps * 1e3, 4), "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "fp16", "weight_dtype": "int4", "data": "synthetic",
-            "config": {"workload": f"{layers}-layer GLM-130B projection sweep, M=1, CUDA graph of {4 * layers} launches",
-                       "packed_weight_bytes": wbytes, "l2": "63 GB working set >> L2"},
-            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": None},
-            "quantize_all_layers": {"ms": round(qtime * 1e3, 2), "gbs": round(qbytes / qtime / 1e9, 1)},
-            "gpu_launches": kernels_per_replay * args.steps, "clocks": clk}
+    gbs = sw.wbytes * args.steps / el / 1e9
+    res = {"metric": "GLM-130B 70-layer INT4 decode sweep (M=1, 280 projections), tokens/s",
+           "value": round(tok_s, 2), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": round(el / args.steps * 1e3, 4), "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "fp16", "weight_dtype": "int4", "data": "synthetic",
+           "config": {"workload": f"{args.layers}-layer GLM-130B projection sweep, M=1, "
+                                  f"CUDA graph of {4 * args.layers} calls",
+                      "packed_weight_bytes": sw.wbytes, "l2": "63 GB working set >> L2"},
+           "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                        "frac": round(gbs / peaks["hbm_gbs"], 4), "peak_source": peaks["source"], "traffic": None},
+           "quantize_all_layers": {"ms": round(sw.qtime * 1e3, 2), "gbs": round(sw.qbytes / sw.qtime / 1e9, 1)},
+           "gpu_launches": sw.kernels_per_replay * args.steps, "clocks": clk}
+    del sw
+    return res
+
+
+def sweep_summary(torch, glmq, peaks, layers: int = SWEEP_LAYERS, steps: int = 10, warmup: int = 3):
+    """Compact result of the layer sweep for the default bench line's extras."""
+    free, _ = torch.cuda.mem_get_info()
+    if free < 72e9 * layers / SWEEP_LAYERS:
+        return {"skipped": f"needs about {72 * layers // SWEEP_LAYERS} GB free on the device"}
+    sw = Sweep(torch, glmq, layers)
+    el = sw.time_replays(torch, steps, warmup)
+    gbs = sw.wbytes * steps / el / 1e9
+    out = {"layers": layers, "tokens_per_s": round(steps / el, 2), "ms_per_token": round(el / steps * 1e3, 3),
+           "weight_gbs": round(gbs, 1), "frac_hbm": round(gbs / peaks["hbm_gbs"], 4),
+           "quantize_all_ms": round(sw.qtime * 1e3, 2), "quantize_gbs": round(sw.qbytes / sw.qtime / 1e9, 1)}
+    del sw
+    torch.cuda.empty_cache()
+    return out
 
 
 # ----------------------------------------------------------------------------- one launch (profiling)
@@ -737,6 +857,7 @@ def main():
         res = run_decode(args, world, rank, local)
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
             res["cpu_baseline"] = cpu_baseline()
+        res["highlights"] = res.pop("highlights")       # keep the compact summary last on the line
     if rank == 0:
         print(json.dumps(res), flush=True)
     if world > 1:

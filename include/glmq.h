@@ -211,25 +211,26 @@ GLMQ_API glmq_status glmq_gemm_zp(const void* X, int64_t M, const void* packed, 
  * glmq_gemm_decode without any device allocation (the paper has no counterpart:
  * this is a deployment variant of the decode kernel).
  *
- * Some callers cannot call cudaMalloc: code that runs while a stream is being
- * captured into a CUDA graph (allocation is not a capturable operation), code
- * embedded under an allocator that owns the whole device-memory budget (a
- * framework's caching pool, a fixed-size arena on a shared serving GPU), and
- * latency-critical paths that must not block in the driver after start-up.
- * glmq_gemm_decode may allocate its split-K scratch on first use; this entry
- * point never does. Its scratch is a fixed, statically allocated device array of
- * GLMQ_NOALLOC_SCRATCH_FLOATS fp32 values (4 MiB) that every GPU which loads the
- * library holds until the process exits.
+ * glmq_gemm_decode may allocate its split-K scratch with cudaMalloc on first use.
+ * Some callers cannot let a library do that: a host framework whose caching
+ * allocator or fixed-size arena owns the whole device-memory budget (an
+ * allocation behind its back can fail, or push the framework out of memory), and
+ * serving loops with a latency budget, where cudaMalloc can synchronize the device
+ * and block in the driver. This entry point never allocates. Its scratch is a
+ * fixed, statically allocated device array of GLMQ_NOALLOC_SCRATCH_FLOATS fp32
+ * values (4 MiB) that every GPU which loads the library holds until the process
+ * exits.
  *   - Same arguments, layout and results as glmq_gemm_decode (M <= 16).
  *   - Requires M * N <= GLMQ_NOALLOC_SCRATCH_FLOATS, else GLMQ_ERR_BAD_SHAPE and
  *     nothing is enqueued.
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress, no allocation); make that first call before any
  *     stream capture on that device.
- *   - All calls share the one array, and it keeps the last call's contents: the
- *     part a call needs zeroed is cleared on its stream before use. Calls that
- *     overlap on the GPU (different streams, no ordering between them) race on
- *     the array and may produce wrong results.
+ *   - All calls share the one array, and it keeps the last call's contents: a call
+ *     whose tiles are split over K parts clears the part it accumulates into, on its
+ *     stream, before its kernel runs. Calls that overlap on the GPU (different
+ *     streams, no ordering between them) race on the array and may produce wrong
+ *     results.
  */
 #define GLMQ_NOALLOC_SCRATCH_FLOATS (1u << 20)
 GLMQ_API glmq_status glmq_gemm_decode_noalloc(const void* X, int64_t M, const void* packed, const void* scale,
@@ -259,6 +260,22 @@ GLMQ_API uint64_t glmq_kernel_launches(void);
  * it blocks the calling thread.
  */
 GLMQ_API glmq_status glmq_last_device_error(void* stream, uint32_t* flags);
+
+/*
+ * Failure-detection hook (the paper has no counterpart). Every internal wait of
+ * the kernels on a pipeline barrier gives up after a wall-clock limit, 2 s by
+ * default, sets a bit in the device status word (see glmq_last_device_error) and
+ * lets the kernel finish without hanging; its outputs are then not valid. This sets
+ * that limit, in nanoseconds, for kernels launched afterwards on the current
+ * device; 0 restores the default. Tests lower it to make a normal call's waits run
+ * out and check that the failure is reported. The waits by which a block makes sure
+ * its own copies and tensor-core operations have finished before it exits always
+ * keep the default limit, so a lowered limit never ends a block with work in flight.
+ * Not for production use. Synchronous with respect to the host; must not be called
+ * while kernels of this library run on the device.
+ * Errors: GLMQ_ERR_UNSUPPORTED_DEVICE, GLMQ_ERR_CUDA.
+ */
+GLMQ_API glmq_status glmq_set_wait_limit_ns(uint64_t limit_ns);
 
 #ifdef __cplusplus
 }

@@ -24,5 +24,6 @@ from ._binding import (  # noqa: F401
     quantize_zp,
     raw_gemm,
     raw_quantize,
+    set_wait_limit_ns,
     status_string,
 )

@@ -54,6 +54,7 @@ SIGNATURES = {
     "glmq_last_cuda_error": (ctypes.c_int, []),
     "glmq_kernel_launches": (ctypes.c_uint64, []),
     "glmq_last_device_error": (ctypes.c_int, [_vp, ctypes.POINTER(ctypes.c_uint32)]),
+    "glmq_set_wait_limit_ns": (ctypes.c_int, [ctypes.c_uint64]),
 }
 
 _lib = None
@@ -151,6 +152,12 @@ def last_device_error(stream: int = 0):
     flags = ctypes.c_uint32(0)
     st = lib().glmq_last_device_error(stream, ctypes.byref(flags))
     return st, flags.value
+
+
+def set_wait_limit_ns(limit_ns: int) -> None:
+    """glmq_set_wait_limit_ns: the give-up limit of the kernels' pipeline waits on the current
+    device (0 = the default 2 s). A test hook for the failure path; not for production."""
+    _check(lib().glmq_set_wait_limit_ns(int(limit_ns)), "glmq_set_wait_limit_ns")
 
 
 # ----------------------------------------------------------------- torch-tensor calls

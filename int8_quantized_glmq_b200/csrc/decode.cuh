@@ -11,23 +11,29 @@
 // HBM stream. Design:
 //  * Work units are (row tile of 256 rows, K part) pairs, enumerated K-part major;
 //    each persistent CTA takes one contiguous range of units, so the load is
-//    balanced to within one unit and a CTA changes K part (and so restages its
-//    activation slice) at most a few times. The number of K parts is the smallest
-//    that both fits the activation slice in shared memory and spreads the units
-//    evenly over the SMs.
-//  * Warp 16 is the producer: one lane issues, per stage, one 2-D TMA tile load of
-//    256 rows x 128 bytes (128-byte swizzle, 32 KB) into a kDecodeStages-deep
-//    ring, with an L2 evict-first hint. Rows past N and bytes past K are
-//    zero-filled by the TMA unit.
+//    balanced to within one unit. K parts exist only to spread the units evenly
+//    over the SMs (tiles split over parts cost a round trip of fp32 partial sums).
+//  * A stage is one 256-k segment of one tile: 256 weight rows x 128 packed bytes
+//    (32 KB), the matching activations of the MP token rows (in the order the
+//    MMA fragments read them) and a per-token bias for the biased dequantization.
+//    The ring has kStages stages (5 or 6, whatever fits in shared memory).
+//  * Warp 16 is the weight producer: one lane issues, per stage, one 2-D TMA tile
+//    load of the weight box (128-byte swizzle, L2 evict-first hint). Rows past N and
+//    bytes past K are zero-filled by the TMA unit.
+//  * Warps 17..19 are activation producers: warp 17 + i fills the activation slot of
+//    every third stage (sequence number i mod 3), reading X[:, k0 : k0 + 256] from
+//    global memory (it is small and L2-resident), permuting it into fragment order,
+//    dividing the high-nibble slots by 16 (see below) and summing the
+//    per-token bias. Three of them keep several stages in flight, so the L2 latency of
+//    one warp is hidden behind the others.
 //  * Warps 0..15 are consumers: warp w owns rows 16w .. 16w+15 of the tile and
 //    reads the whole stage's K segment for them. Codes are dequantized in
 //    registers with exponent-bias tricks (a code c becomes the fp16 number
 //    1024 + (c ^ 8) by OR-ing it into the mantissa) and feed mma.sync m16n8k16
 //    as the A operand straight from registers, X being the B operand. The K order
 //    inside each MMA is permuted identically on both operands so that each 32-bit
-//    packed word feeds two MMAs without a byte shuffle; the permutation is applied
-//    once, when the consumers stage the activation slice into shared memory in
-//    exactly the order the B fragments are read.
+//    packed word feeds two MMAs without a byte shuffle; the activation producers
+//    apply the permutation to X.
 //  * A warp's sums stay in registers for the whole unit, so a unit ends without
 //    any cross-warp reduction or barrier: the warp scales, rounds and stores its
 //    own 16 rows. When a tile is split over several K parts each warp instead adds
@@ -35,6 +41,10 @@
 //    red.global.add, and a small stream-ordered finalize kernel
 //    (decode_finalize_kernel) scales, rounds and stores Y and returns the scratch
 //    to zero for the next call.
+//  * Every wait is bounded. A warp whose wait gives up reports it and stops: it
+//    neither consumes nor releases further stages, so a stage is never refilled
+//    while a copy into it may still be in flight, and the weight producer still
+//    waits for each of its own copies to land before its CTA exits.
 #pragma once
 
 #include <cuda.h>
@@ -45,18 +55,21 @@
 namespace glmq {
 
 constexpr int kDecodeConsumerWarps = 16;
-constexpr int kDecodeThreads = (kDecodeConsumerWarps + 1) * 32;
-constexpr int kDecodeStages = 6;
+constexpr int kDecodeProducerWarp = 16;                               // weight TMA
+constexpr int kDecodeXWarp0 = 17;                                     // activation producers 17..19
+constexpr int kDecodeXWarps = 3;   // 20 warps in all: ptxas then allows 96 registers per thread
+constexpr int kDecodeThreads = (kDecodeConsumerWarps + 1 + kDecodeXWarps) * 32;
 constexpr int kDecodeRows = 16 * kDecodeConsumerWarps;                // rows per tile (256)
 constexpr int kDecodeSegB = 128;         // packed bytes per row per stage (one TMA box width)
 constexpr int kDecodeStageBytes = kDecodeRows * kDecodeSegB;          // 32 KB: one TMA box per stage
-// ring + barriers; the activation slice follows
-constexpr int kDecodeFixedSmem = kDecodeStages * kDecodeStageBytes + 256;
+constexpr int kDecodeSmemLimit = 232448;  // opt-in shared memory per block on sm_100
+constexpr int kDecodeMaxStages = 6;
 
 template <int BITS, int MP, int CHAINS = 2, int ZP = 0>
 struct DecodeCfg {
   static_assert(CHAINS == 2 || CHAINS == 4, "accumulator chains");
   static_assert(ZP == 0 || BITS == 4, "zero-point codes are INT4");
+  static_assert(MP == 1 || MP == 2 || MP == 4 || MP == 8 || MP == 16, "token capacity");
   static constexpr int kZP = ZP;   // 1: zero-point INT4 codes (unsigned, per-row zero point)
   // biased dequantization: low nibbles give the fp16 integer kLowBase + (value), high
   // nibbles kHighBase + 16 (value); symmetric codes carry their own +8 offset in the XOR
@@ -68,13 +81,23 @@ struct DecodeCfg {
   static constexpr int kMP = MP;                    // token capacity of the activation layout (M <= MP)
   static constexpr int kNB = (MP + 7) / 8;          // n8 token blocks of the MMA
   static constexpr int KPB = (BITS == 4) ? 2 : 1;   // codes per byte
-  static constexpr int SEGK = kDecodeSegB * KPB;    // k per segment
-  static constexpr int SK = SEGK;                   // k per stage (one segment)
-  static constexpr int TB = kDecodeSegB / 4;        // packed bytes per thread per row per segment (32)
-  static constexpr int TK = TB * KPB;               // k per thread per segment
-  static constexpr int TW = TB / 4;                 // 32-bit words per thread per row per segment (8)
-  static constexpr int XU = TK / 8;                 // 16-byte activation units per thread per segment
+  static constexpr int SK = kDecodeSegB * KPB;      // k per stage
+  static constexpr int TB = kDecodeSegB / 4;        // packed bytes per thread per row per stage (32)
+  static constexpr int TK = TB * KPB;               // k per thread per stage
+  static constexpr int TW = TB / 4;                 // 32-bit words per thread per row per stage (8)
+  static constexpr int XU = TK / 8;                 // 16-byte activation units per thread per stage
   static constexpr int kChains = CHAINS;            // independent MMA accumulator chains per token block
+  static constexpr int X_UNITS = XU * MP * 4;       // 16-byte units in a stage's activation slot
+  static constexpr int X_BYTES = X_UNITS * 16;
+  // per stage and token: the bias of the biased dequantization (INT4), then (zero point)
+  // the sum of x over the stage
+  static constexpr int B_FLOATS = ZP ? 32 : 16;
+  static constexpr int STAGE_TOTAL = kDecodeStageBytes + X_BYTES + B_FLOATS * 4 + 3 * 8;
+  static constexpr int kStages = (kDecodeSmemLimit - 1024) / STAGE_TOTAL < kDecodeMaxStages
+                                     ? (kDecodeSmemLimit - 1024) / STAGE_TOTAL : kDecodeMaxStages;
+  static constexpr int SMEM_BYTES = kStages * STAGE_TOTAL + 1024;   // + alignment slack
+  static_assert(kStages >= 4, "pipeline depth");
+  static_assert(SMEM_BYTES <= kDecodeSmemLimit, "shared memory");
 };
 
 struct DecodeArgs {
@@ -100,6 +123,7 @@ struct DecodeArgs {
   int nxt_tiles;
   int nxt_KPP;
   int nxt_K;
+  int nxt_stages;     // ring depth of the next call's kernel configuration
 };
 
 // INT4, biased form: one packed word (8 codes, k = 0..7 of the word) -> 4 half2
@@ -148,13 +172,14 @@ __device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* map, int x, i
                : "memory");
 }
 
-// Index (in 16-byte units) of the activation unit read by lane (n, c) for unit jj of
-// segment sg of the current K part. Consecutive lanes of a token read consecutive
+// Index (in 16-byte units) of activation unit (jj, n, c) in a stage's activation slot:
+// the 8 values of token n that lane c multiplies with its codes jj*8 .. jj*8+7 (k =
+// c*TK + jj*8 .. +7 of the stage). Consecutive lanes of a token read consecutive
 // units; the token stride is the compile-time capacity MP, so within a stage every
 // fragment address is a per-lane base plus an immediate.
 template <class C>
-__host__ __device__ constexpr uint32_t x_unit(int sg, int jj, int n, int c) {
-  return static_cast<uint32_t>(((sg * C::XU + jj) * C::kMP + n) * 4 + c);
+__host__ __device__ constexpr uint32_t x_unit(int jj, int n, int c) {
+  return static_cast<uint32_t>((jj * C::kMP + n) * 4 + c);
 }
 
 // One stage of one consumer warp: its segment (TK codes per lane) of rows ra and
@@ -229,56 +254,71 @@ __device__ __forceinline__ void decode_segment(uint32_t box, uint32_t xseg, uint
   }
 }
 
-// Copies the activation slice X[:, pk0 : pk0 + plen] into shared memory in the order
-// the B fragments are read (x_unit), INT4 slots permuted and high-nibble slots
-// divided by 16 (see dequant_int4_word_biased). Units of tokens >= M and of k past
-// plen are not written (no fragment of a real token reads them).
-// With issued != 0 every thread adds 1 to that shared counter once its first batch of
-// global loads has been issued (or at once when it has none).
+
+// Fills one stage's activation slot (and bias slot) for the k range [k0, k0 + SK) of
+// X, called by all 32 lanes of an activation-producer warp. Lane L serves token
+// n = L / (32 / MP); the 32 / MP lanes of a token split its units between them and
+// combine their bias sums with shuffles. Each unit: 8 consecutive values of X,
+// permuted to the MMA k order (0,4),(1,5),(2,6),(3,7) with the high-nibble slots (1,5)
+// and (3,7) divided by 16 (exact: a power of two); INT8 keeps the natural order.
+// Units of tokens >= M are not written (no fragment of a real token reads them);
+// values past K are written as zero.
 template <class C>
-__device__ __forceinline__ void stage_activations(const __half* __restrict__ X, int K, int M, int pk0, int plen,
-                                                  uint8_t* xbuf, int ct, uint32_t issued = 0) {
-  constexpr int kCT = kDecodeConsumerWarps * 32;
-  constexpr int kBatch = 8;
-  const int nseg = (plen + C::SEGK - 1) / C::SEGK;
-  const int total = nseg * C::XU * C::kMP * 4;                  // 16-byte units of the slice
-  if (issued != 0 && ct >= total) shared_count_add(issued);
-  for (int d0 = ct; d0 < total; d0 += kCT * kBatch) {
-    uint4 v[kBatch];
-    bool live[kBatch];
+__device__ __forceinline__ void fill_activation_stage(const __half* __restrict__ X, int K, int M, int k0,
+                                                      uint8_t* xslot, float* bslot, int lane) {
+  constexpr int LPT = 32 / C::kMP;          // lanes per token
+  constexpr int UPT = C::XU * 4;            // units per token
+  const int n = lane / LPT;
+  const int sub = lane - n * LPT;
+  float bias = 0.0f, sx = 0.0f;
+  if (n < M) {
+    const __half* xrow = X + static_cast<long long>(n) * K + k0;
+    uint4 v[(UPT + LPT - 1) / LPT];
 #pragma unroll
-    for (int b = 0; b < kBatch; ++b) {
-      const int d = d0 + b * kCT;
-      const int cc = d & 3;
-      const int n = (d >> 2) % C::kMP;
-      const int rest = (d >> 2) / C::kMP;
-      const int jj = rest % C::XU;
-      const int sg = rest / C::XU;
-      const int kr = sg * C::SEGK + cc * C::TK + jj * 8;        // part-relative k of the 8 values
-      live[b] = d < total && n < M && kr < plen;
-      v[b] = make_uint4(0, 0, 0, 0);
-      if (live[b]) v[b] = __ldg(reinterpret_cast<const uint4*>(X + static_cast<long long>(n) * K + pk0 + kr));
+    for (int i = 0; i < (UPT + LPT - 1) / LPT; ++i) {
+      const int r = sub + i * LPT;
+      const int kr = (r & 3) * C::TK + (r >> 2) * 8;
+      v[i] = make_uint4(0, 0, 0, 0);
+      if (r < UPT && k0 + kr < K) v[i] = __ldg(reinterpret_cast<const uint4*>(xrow + kr));
     }
-    if (issued != 0 && d0 == ct) shared_count_add(issued);
 #pragma unroll
-    for (int b = 0; b < kBatch; ++b) {
-      if (!live[b]) continue;
+    for (int i = 0; i < (UPT + LPT - 1) / LPT; ++i) {
+      const int r = sub + i * LPT;
+      if (r >= UPT) continue;
       uint4 o;
       if constexpr (C::kBits == 4) {
-        // low-nibble slots (x0,x4), (x2,x6) as is; high-nibble slots (x1,x5), (x3,x7) divided by 16
         const __half2 kSixteenth = __halves2half2(__ushort_as_half(0x2C00), __ushort_as_half(0x2C00));
-        o.x = prmt(v[b].x, v[b].z, 0x5410u);
-        uint32_t hy = prmt(v[b].x, v[b].z, 0x7632u);
-        o.z = prmt(v[b].y, v[b].w, 0x5410u);
-        uint32_t hw = prmt(v[b].y, v[b].w, 0x7632u);
+        o.x = prmt(v[i].x, v[i].z, 0x5410u);
+        uint32_t hy = prmt(v[i].x, v[i].z, 0x7632u);
+        o.z = prmt(v[i].y, v[i].w, 0x5410u);
+        uint32_t hw = prmt(v[i].y, v[i].w, 0x7632u);
         __half2 sy = __hmul2(*reinterpret_cast<__half2*>(&hy), kSixteenth);
         __half2 sw = __hmul2(*reinterpret_cast<__half2*>(&hw), kSixteenth);
         o.y = *reinterpret_cast<uint32_t*>(&sy);
         o.w = *reinterpret_cast<uint32_t*>(&sw);
+        const float2 fx = __half22float2(*reinterpret_cast<const __half2*>(&o.x));
+        const float2 fy = __half22float2(*reinterpret_cast<const __half2*>(&o.y));
+        const float2 fz = __half22float2(*reinterpret_cast<const __half2*>(&o.z));
+        const float2 fw = __half22float2(*reinterpret_cast<const __half2*>(&o.w));
+        const float lo = (fx.x + fx.y) + (fz.x + fz.y);
+        const float hi = (fy.x + fy.y) + (fw.x + fw.y);
+        bias += C::kLowBias * lo + C::kHighBias * hi;
+        if constexpr (C::kZP) sx += lo + 16.0f * hi;
       } else {
-        o = v[b];
+        o = v[i];
       }
-      *reinterpret_cast<uint4*>(xbuf + 16u * static_cast<uint32_t>(d0 + b * kCT)) = o;
+      *reinterpret_cast<uint4*>(xslot + 16u * x_unit<C>(r >> 2, n, r & 3)) = o;
+    }
+  }
+  if constexpr (C::kBits == 4) {
+#pragma unroll
+    for (int off = LPT / 2; off > 0; off >>= 1) {
+      bias += __shfl_xor_sync(0xffffffffu, bias, off);
+      if constexpr (C::kZP) sx += __shfl_xor_sync(0xffffffffu, sx, off);
+    }
+    if (sub == 0 && n < M) {
+      bslot[n] = bias;
+      if constexpr (C::kZP) bslot[16 + n] = sx;
     }
   }
 }
@@ -288,17 +328,15 @@ template <class C>
 __global__ void __launch_bounds__(kDecodeThreads, 1)
     decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_next,
                   const DecodeArgs a) {
+  constexpr int S = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* wring = smem;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kDecodeStages * kDecodeStageBytes);
-  uint64_t* empty = full + kDecodeStages;
-  uint32_t* x_issued = reinterpret_cast<uint32_t*>(empty + kDecodeStages);   // inside the fixed 256 bytes
-  uint8_t* xbuf = smem + kDecodeFixedSmem;
-  // INT4 only: per (segment, token) bias of the biased dequantization, after the activation slice;
-  // zero-point codes: then per-token sums of x over the part
-  float* bias_s = reinterpret_cast<float*>(xbuf + 2 * C::kMP * a.KPP);
-  float* sx_s = bias_s + (a.KPP / C::SEGK) * 16;
+  uint8_t* wring = smem;                                           // S x 32 KB weight boxes
+  uint8_t* xring = smem + S * kDecodeStageBytes;                   // S activation slots
+  float* bring = reinterpret_cast<float*>(xring + S * C::X_BYTES); // S bias slots
+  uint64_t* fullw = reinterpret_cast<uint64_t*>(bring + S * C::B_FLOATS);   // weight box landed (1 + tx)
+  uint64_t* fullx = fullw + S;                                     // activation slot written (1)
+  uint64_t* empty = fullx + S;                                     // stage released (16 consumer warps)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -308,67 +346,53 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   const int u_end = static_cast<int>((static_cast<long long>(blockIdx.x + 1) * a.units) / G);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kDecodeStages; ++s) {
-      mbar_init(&full[s], 1);
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&fullw[s], 1);
+      mbar_init(&fullx[s], 1);
       mbar_init(&empty[s], kDecodeConsumerWarps);
     }
-    *x_issued = 0;
     fence_barrier_init();
   }
+  // bias slots of tokens no activation producer writes (M <= token < 16) read as zero
+  for (int i = threadIdx.x; i < S * C::B_FLOATS; i += kDecodeThreads) bring[i] = 0.0f;
   __syncthreads();
   // everything above touches only shared memory; X, W, Y and the scratch may belong
   // to the previous kernel in the stream
   griddep_wait();
   if (threadIdx.x == 0) griddep_launch_dependents();
 
-  if (warp == kDecodeConsumerWarps) {
-    // ------------------------------------------------------------ producer warp
+  if (warp == kDecodeProducerWarp) {
+    // ------------------------------------------------------------ weight producer
     if (lane == 0) {
       const uint64_t pol = policy_evict_first();
-      uint32_t armed[kDecodeStages] = {};
+      uint32_t armed[S] = {};
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      // The consumers stage the first part's activations as soon as they start. Let
-      // their loads enter the memory system before the weight stream fills the ring
-      // (behind ~200 KB per SM of TMA traffic they would arrive microseconds later).
-      // Only an ordering hint: the wait is bounded and the stream starts either way.
-      const uint32_t issued_u32 = smem_u32(x_issued);
-      for (int i = 0; i < 4096 && shared_count_read(issued_u32) < static_cast<uint32_t>(kDecodeConsumerWarps * 32);
-           ++i)
-        __nanosleep(32);
-      int pref_part = u_begin < u_end ? u_begin / a.tiles : -1;
       for (int u = u_begin; u < u_end && ok; ++u) {
         const int p = u / a.tiles;
         const int t = u - p * a.tiles;
         const int pk0 = p * a.KPP;
         const int plen = min(a.KPP, K - pk0);
         const int nst = (plen + C::SK - 1) / C::SK;
-        if (p != pref_part) {
-          // a later part: bring its activation slice into L2 while the ring still holds
-          // the previous part's stages (rows of X are 128-byte aligned: K % 64 == 0)
-          for (int n = 0; n < M; ++n)
-            bulk_prefetch_l2(a.X + static_cast<long long>(n) * K + pk0, static_cast<uint32_t>(plen) * 2u);
-          pref_part = p;
-        }
         for (int ks = 0; ks < nst; ++ks) {
           if (!mbar_wait(&empty[stage], phase ^ 1)) { ok = false; break; }
           const int xb0 = (pk0 + ks * C::SK) / C::KPB;            // first packed byte of the stage
-          mbar_arrive_expect_tx(&full[stage], static_cast<uint32_t>(kDecodeStageBytes));
+          mbar_arrive_expect_tx(&fullw[stage], static_cast<uint32_t>(kDecodeStageBytes));
           armed[stage] = phase + 1;
-          tma_load_2d_hint(wring + stage * kDecodeStageBytes, &tmap_w, xb0, t * kDecodeRows, &full[stage], pol);
-          if (++stage == kDecodeStages) { stage = 0; phase ^= 1; }
+          tma_load_2d_hint(wring + stage * kDecodeStageBytes, &tmap_w, xb0, t * kDecodeRows, &fullw[stage], pol);
+          if (++stage == S) { stage = 0; phase ^= 1; }
         }
       }
       if (ok && a.nxt_grid > 0) {
         // Every load of this CTA is issued; its consumers still work through up to a
         // full ring. Meanwhile bring the next call's first ring fill into L2: next CTA b
-        // (b = this CTA, this CTA + G, ...) starts with the first kDecodeStages stages
+        // (b = this CTA, this CTA + G, ...) starts with the first nxt_stages stages
         // of its units. The next call's weights do not depend on this call's output.
         for (int b = blockIdx.x; b < a.nxt_grid; b += G) {
           const int ub = static_cast<int>((static_cast<long long>(b) * a.nxt_units) / a.nxt_grid);
           const int ue = static_cast<int>((static_cast<long long>(b + 1) * a.nxt_units) / a.nxt_grid);
-          int left = kDecodeStages;
+          int left = a.nxt_stages;
           for (int u = ub; u < ue && left > 0; ++u) {
             const int p = u / a.nxt_tiles;
             const int t = u - p * a.nxt_tiles;
@@ -382,98 +406,60 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       }
       // never leave while TMA writes into this CTA's shared memory may be in flight
       bool drained = true;
-      for (int s = 0; s < kDecodeStages; ++s)
-        if (armed[s] && !mbar_wait(&full[s], armed[s] - 1)) drained = false;
+      for (int s = 0; s < S; ++s)
+        if (armed[s] && !mbar_wait_drain(&fullw[s], armed[s] - 1)) drained = false;
       if (!ok || !drained) report_error(kErrDecodeProducerWait);
     }
+    return;
+  }
+
+  if (warp >= kDecodeXWarp0) {
+    // ------------------------------------------------------------ activation producers
+    const int xw = warp - kDecodeXWarp0;
+    int q = 0;                    // stage sequence number of this CTA
+    bool ok = true;
+    for (int u = u_begin; u < u_end && ok; ++u) {
+      const int p = u / a.tiles;
+      const int pk0 = p * a.KPP;
+      const int plen = min(a.KPP, K - pk0);
+      const int nst = (plen + C::SK - 1) / C::SK;
+      for (int ks = 0; ks < nst; ++ks, ++q) {
+        if (q % kDecodeXWarps != xw) continue;
+        const int stage = q % S;
+        const uint32_t phase = static_cast<uint32_t>(q / S) & 1u;
+        if (!mbar_wait_warp(&empty[stage], phase ^ 1)) { ok = false; break; }
+        fill_activation_stage<C>(a.X, K, M, pk0 + ks * C::SK, xring + stage * C::X_BYTES, bring + stage * C::B_FLOATS,
+                                 lane);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&fullx[stage]);
+      }
+    }
+    if (!ok && lane == 0) report_error(kErrDecodeProducerWait);
     return;
   }
 
   // -------------------------------------------------------------- consumer warps
   const int r = lane >> 2;
   const int c = lane & 3;
-  const int ct = threadIdx.x;                // 0 .. 511
-  constexpr int kCT = kDecodeConsumerWarps * 32;
   const uint32_t wring_u32 = smem_u32(wring);
-  const uint32_t xbuf_u32 = smem_u32(xbuf);
+  const uint32_t xring_u32 = smem_u32(xring);
   const int ra = 16 * warp + r;              // this lane's rows: ra and ra + 8 (same ra & 7)
   // per-lane byte offsets: packed row ra, 16-byte units 2c and 2c+1 under the 128-byte swizzle
   const uint32_t wlane = static_cast<uint32_t>(ra * kDecodeSegB + (((2 * c) ^ (ra & 7)) << 4)) |
                          (static_cast<uint32_t>(ra * kDecodeSegB + (((2 * c + 1) ^ (ra & 7)) << 4)) << 16);
   // activation units of this lane's tokens (clamped to a real token; results past M are discarded)
-  const uint32_t xlane0 = 16u * x_unit<C>(0, 0, min(r, M - 1), c);
-  const uint32_t xlane1 = 16u * x_unit<C>(0, 0, min(r + 8, M - 1), c);
+  const uint32_t xlane0 = 16u * x_unit<C>(0, min(r, M - 1), c);
+  const uint32_t xlane1 = 16u * x_unit<C>(0, min(r + 8, M - 1), c);
   const bool split = a.parts > 1;
   int stage = 0;
   uint32_t phase = 0;
-  int cur_part = -1;
   bool ok = true;
 
-  for (int u = u_begin; u < u_end; ++u) {
+  for (int u = u_begin; u < u_end && ok; ++u) {
     const int p = u / a.tiles;
     const int t = u - p * a.tiles;
     const int pk0 = p * a.KPP;
     const int plen = min(a.KPP, K - pk0);
-    if (p != cur_part) {
-      // stage this part's activations in fragment order (all consumers, then barrier).
-      // Thread i fills shared 16-byte unit i (conflict-free stores); each thread first
-      // issues all its global loads of a batch through the read-only path, then stores.
-      named_barrier_sync(1, kCT);
-      stage_activations<C>(a.X, K, M, pk0, plen, xbuf, ct, cur_part < 0 ? smem_u32(x_issued) : 0u);
-      if constexpr (C::kBits == 4) {
-        // per (segment, token) bias sum_k (1032 or 1152) * B[k], one warp per real pair
-        // (lane = 8-value chunk of the 256-k segment), read back from the staged slice
-        static_assert(C::SEGK == 256, "one lane per 8-value chunk of a segment");
-        named_barrier_sync(1, kCT);
-        const int nseg = a.KPP / C::SEGK;
-        const int pseg = (plen + C::SEGK - 1) / C::SEGK;
-        for (int i = ct; i < nseg * 16; i += kCT) {                // entries the pair loop never writes
-          if ((i & 15) >= M || (i >> 4) >= pseg) bias_s[i] = 0.0f;
-        }
-        for (int pair = warp; pair < pseg * M; pair += kDecodeConsumerWarps) {
-          const int sg = pair / M;
-          const int n = pair - sg * M;
-          float bias = 0.0f;
-          if (sg * C::SEGK + lane * 8 < plen) {
-            const uint4 o = *reinterpret_cast<const uint4*>(xbuf + 16u * x_unit<C>(sg, lane & 7, n, lane >> 3));
-            const float2 fx = __half22float2(*reinterpret_cast<const __half2*>(&o.x));
-            const float2 fy = __half22float2(*reinterpret_cast<const __half2*>(&o.y));
-            const float2 fz = __half22float2(*reinterpret_cast<const __half2*>(&o.z));
-            const float2 fw = __half22float2(*reinterpret_cast<const __half2*>(&o.w));
-            bias = C::kLowBias * ((fx.x + fx.y) + (fz.x + fz.y)) + C::kHighBias * ((fy.x + fy.y) + (fw.x + fw.y));
-          }
-#pragma unroll
-          for (int off = 16; off > 0; off >>= 1) bias += __shfl_xor_sync(0xffffffffu, bias, off);
-          if (lane == 0) bias_s[sg * 16 + n] = bias;
-        }
-        if constexpr (C::kZP) {
-          // per-token sum of x over the part, for the zero-point term z[n] * sum_k x[m,k]
-          // (high-nibble slots hold x / 16)
-          const int units = pseg * C::XU * 4;
-          for (int n = warp; n < M; n += kDecodeConsumerWarps) {
-            float sx = 0.0f;
-            for (int i = lane; i < units; i += 32) {
-              const int sg = i / (C::XU * 4);
-              const int rem = i - sg * (C::XU * 4);
-              const int jj = rem >> 2, cc = rem & 3;
-              if (sg * C::SEGK + cc * C::TK + jj * 8 < plen) {
-                const uint4 o = *reinterpret_cast<const uint4*>(xbuf + 16u * x_unit<C>(sg, jj, n, cc));
-                const float2 fx = __half22float2(*reinterpret_cast<const __half2*>(&o.x));
-                const float2 fy = __half22float2(*reinterpret_cast<const __half2*>(&o.y));
-                const float2 fz = __half22float2(*reinterpret_cast<const __half2*>(&o.z));
-                const float2 fw = __half22float2(*reinterpret_cast<const __half2*>(&o.w));
-                sx += ((fx.x + fx.y) + (fz.x + fz.y)) + 16.0f * ((fy.x + fy.y) + (fw.x + fw.y));
-              }
-            }
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) sx += __shfl_xor_sync(0xffffffffu, sx, off);
-            if (lane == 0) sx_s[n] = sx;
-          }
-        }
-      }
-      cur_part = p;
-      named_barrier_sync(1, kCT);
-    }
 
     float acc[C::kChains][C::kNB][4];
 #pragma unroll
@@ -482,26 +468,34 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       for (int nb = 0; nb < C::kNB; ++nb)
 #pragma unroll
         for (int i = 0; i < 4; ++i) acc[h][nb][i] = 0.0f;
+    float sxa[C::kNB][2] = {};   // zero point: sum of x over the unit for tokens 8 nb + 2 c (+1)
 
     const int nst = (plen + C::SK - 1) / C::SK;
     for (int ks = 0; ks < nst; ++ks) {
-      if (ok && !mbar_wait_warp(&full[stage], phase)) ok = false;
-      if (ok) {
-        const uint32_t box = wring_u32 + stage * kDecodeStageBytes;
-        const uint32_t xseg = xbuf_u32 + 16u * x_unit<C>(ks, 0, 0, 0);
-        const float* bias_seg = bias_s + ks * 16;
-        const int kseg = pk0 + ks * C::SK;                        // absolute k of this stage
-        if (kseg + C::SK <= K) {
-          decode_segment<C, false>(box, xseg, wlane, xlane0, xlane1, true, bias_seg, c, acc);
-        } else {
-          const bool valid = kseg + c * C::TK < K;
-          decode_segment<C, true>(box, xseg, wlane, xlane0, xlane1, valid, bias_seg, c, acc);
+      if (!mbar_wait_warp(&fullx[stage], phase) || !mbar_wait_warp(&fullw[stage], phase)) { ok = false; break; }
+      const uint32_t box = wring_u32 + stage * kDecodeStageBytes;
+      const uint32_t xseg = xring_u32 + stage * C::X_BYTES;
+      const float* bias_seg = bring + stage * C::B_FLOATS;
+      const int kseg = pk0 + ks * C::SK;                        // absolute k of this stage
+      if (kseg + C::SK <= K) {
+        decode_segment<C, false>(box, xseg, wlane, xlane0, xlane1, true, bias_seg, c, acc);
+      } else {
+        const bool valid = kseg + c * C::TK < K;
+        decode_segment<C, true>(box, xseg, wlane, xlane0, xlane1, valid, bias_seg, c, acc);
+      }
+      if constexpr (C::kZP) {
+#pragma unroll
+        for (int nb = 0; nb < C::kNB; ++nb) {
+          const float2 v = *reinterpret_cast<const float2*>(bias_seg + 16 + 8 * nb + 2 * c);
+          sxa[nb][0] += v.x;
+          sxa[nb][1] += v.y;
         }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[stage]);
-      if (++stage == kDecodeStages) { stage = 0; phase ^= 1; }
+      if (++stage == S) { stage = 0; phase ^= 1; }
     }
+    if (!ok) break;
 
     // ---- unit epilogue, per warp: rows ra and ra + 8, tokens 8 nb + 2 c (+1)
     const int row_a = t * kDecodeRows + ra;
@@ -523,12 +517,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
 #pragma unroll
         for (int i = 0; i < 4; ++i) acc[0][nb][i] += acc[h][nb][i];
       if constexpr (C::kZP) {
-        // the MMAs saw the unsigned codes: remove z[row] * sum_k x[m,k] (this part's k)
+        // the MMAs saw the unsigned codes: remove z[row] * sum_k x[m,k] (this unit's k)
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int m = 8 * nb + 2 * c + (i & 1);
-          if (m < M) acc[0][nb][i] -= ((i < 2) ? za : zb) * sx_s[m];
-        }
+        for (int i = 0; i < 4; ++i) acc[0][nb][i] -= ((i < 2) ? za : zb) * sxa[nb][i & 1];
       }
       if (!split && a.geglu) {
         // rows row_a (first GeGLU half) and row_b (second half) of the same output column

@@ -311,33 +311,47 @@ glmq_status skinny_x_scratch(size_t bytes, uint8_t** out) {
 
 // ---------------------------------------------------------------- decode
 struct DecodePlan {
-  int KPP, parts, tiles, units, smem, grid;
+  int KPP, parts, tiles, units, smem, grid, stages;
 };
 
-// Choose the K-part length. A part's activation slice (and, for INT4, its bias
-// table) must fit in shared memory beside the weight ring; among the part counts
-// that fit, take the one that spreads the (tile, part) units most evenly over the
-// SMs, preferring fewer parts (each split tile costs a round trip of fp32 partial
-// sums through the scratch buffer and a finalize launch).
+// Stages of the largest per-CTA share when `units` (tile, K part) units, enumerated
+// K-part major (part p holds units p*tiles .. p*tiles + tiles - 1), are split into G
+// contiguous ranges; every part has spp stages except the last, which has `last`.
+long long max_cta_stages(long long tiles, int parts, int spp, int last, int G) {
+  const long long units = tiles * parts;
+  const long long last0 = (parts - 1) * tiles;      // first unit of the last part
+  long long worst = 0;
+  for (int b = 0; b < G; ++b) {
+    const long long u0 = (b * units) / G, u1 = ((b + 1) * units) / G;
+    const long long in_last = std::max(0LL, u1 - std::max(u0, last0));
+    const long long w = (u1 - u0) * spp - in_last * (spp - last);
+    worst = std::max(worst, w);
+  }
+  return worst;
+}
+
+// Choose the K-part length. Activations stream through the stages, so any split fits;
+// parts only spread the (tile, part) units over the SMs. Among the part counts that
+// split the K stages into parts of equal length (the last may be shorter), take the
+// one whose most loaded CTA has the least work relative to a perfect spread,
+// preferring fewer parts (each split tile costs a round trip of fp32 partial sums
+// through the scratch buffer and a finalize launch).
 template <class C>
 bool plan_decode(const DeviceInfo& dev, int N, int K, DecodePlan* pl) {
-  const int x_budget = dev.smem_optin - kDecodeFixedSmem - 1024 - 64;   // 64: per-token sums (zero point)
+  if (C::SMEM_BYTES > dev.smem_optin) return false;
   const int stages = (K + C::SK - 1) / C::SK;
-  const int per_stage = 2 * C::kMP * C::SK + ((C::kBits == 4) ? 16 * 4 : 0);
-  const int max_spp = x_budget / per_stage;
-  if (max_spp < 1 || stages < 1) return false;
-  const int parts_min = (stages + max_spp - 1) / max_spp;
   const long long tiles = (static_cast<long long>(N) + kDecodeRows - 1) / kDecodeRows;
-  if (tiles * stages > 0x7fffffffLL) return false;
-  int parts = parts_min;
+  if (stages < 1 || tiles < 1 || tiles * stages > 0x7fffffffLL) return false;
+  int parts = 1;
   double best = -1.0;
-  for (int P = parts_min; P <= stages && P <= parts_min + 16; ++P) {
+  for (int P = 1; P <= stages && P <= 32; ++P) {
     const int spp = (stages + P - 1) / P;
-    if ((stages + spp - 1) / spp != P) continue;      // not a distinct split into equal-length parts
+    if ((stages + spp - 1) / spp != P) continue;      // not a distinct split
     const long long units = tiles * P;
-    const long long grid = units < dev.sms ? units : dev.sms;
-    const double eff = (static_cast<double>(units) / grid) / ((units + grid - 1) / grid) *
-                       (static_cast<double>(grid) / dev.sms);
+    const int G = static_cast<int>(units < dev.sms ? units : dev.sms);
+    const int last = stages - (P - 1) * spp;
+    const double eff = static_cast<double>(tiles * stages) /
+                       (static_cast<double>(dev.sms) * max_cta_stages(tiles, P, spp, last, G));
     if (eff > best + 0.02) {
       best = eff;
       parts = P;
@@ -349,8 +363,9 @@ bool plan_decode(const DeviceInfo& dev, int N, int K, DecodePlan* pl) {
   pl->tiles = static_cast<int>(tiles);
   pl->units = pl->parts * pl->tiles;
   pl->grid = pl->units < dev.sms ? pl->units : dev.sms;
-  pl->smem = kDecodeFixedSmem + 1024 + spp * per_stage + 64;
-  return pl->smem <= dev.smem_optin;
+  pl->smem = C::SMEM_BYTES;
+  pl->stages = C::kStages;
+  return true;
 }
 
 // The decode plan of a call with M tokens (the kernel configuration launch_decode picks).
@@ -403,6 +418,7 @@ glmq_status launch_decode_cfg(const DeviceInfo& dev, const void* X, int M, const
   a.nxt_tiles = npl.tiles;
   a.nxt_KPP = npl.KPP;
   a.nxt_K = e.next_K;
+  a.nxt_stages = npl.stages;
   if (pl.parts > 1 && (st = decode_scratch(static_cast<size_t>(M) * N, &a.ws)) != GLMQ_OK) return st;
   if ((st = allow_smem(decode_kernel<C>, pl.smem)) != GLMQ_OK) return st;
   if ((st = launch_pdl(decode_kernel<C>, dim3(pl.grid), dim3(kDecodeThreads), pl.smem, s, tw, tn, a)) != GLMQ_OK)
@@ -607,11 +623,14 @@ glmq_status launch_decode_noalloc_cfg(const DeviceInfo& dev, const void* X, int 
   a.bias = nullptr;
   a.geglu = 0;
   a.zero = nullptr;
-  a.nxt_grid = a.nxt_units = a.nxt_tiles = a.nxt_KPP = a.nxt_K = 0;
+  a.nxt_grid = a.nxt_units = a.nxt_tiles = a.nxt_KPP = a.nxt_K = a.nxt_stages = 0;
   cudaError_t e;
   if (pl.parts > 1) {
     if ((st = noalloc_scratch(&a.ws)) != GLMQ_OK) return st;
-    // the partial sums must start at zero; the array keeps whatever the last call left
+    // The partial sums must start at zero. Every call shares the array, and a call
+    // whose kernel gave up a bounded wait (glmq_last_device_error) can leave partial
+    // sums behind, so each call clears its own region on its stream instead of relying
+    // on the previous call's finalize pass having returned it to zero.
     if ((e = cudaMemsetAsync(a.ws, 0, static_cast<size_t>(M) * N * sizeof(float), s)) != cudaSuccess)
       return cuda_fail(e);
   }
@@ -770,6 +789,16 @@ glmq_status glmq_gemm_decode_noalloc(const void* X, int64_t M, const void* packe
   const int m = static_cast<int>(M), n = static_cast<int>(N), k = static_cast<int>(K);
   return bits == 4 ? launch_decode_noalloc<4>(*dev, X, m, packed, scale, n, k, Y, s)
                    : launch_decode_noalloc<8>(*dev, X, m, packed, scale, n, k, Y, s);
+}
+
+glmq_status glmq_set_wait_limit_ns(uint64_t limit_ns) {
+  const unsigned long long v = limit_ns == 0 ? glmq::kWaitLimitNs : static_cast<unsigned long long>(limit_ns);
+  const DeviceInfo* dev = nullptr;
+  glmq_status st = current_device(&dev);
+  if (st != GLMQ_OK) return st;
+  const cudaError_t e = cudaMemcpyToSymbol(glmq::g_wait_limit_ns, &v, sizeof(v));
+  if (e != cudaSuccess) return cuda_fail(e);
+  return GLMQ_OK;
 }
 
 const char* glmq_status_string(int status) {

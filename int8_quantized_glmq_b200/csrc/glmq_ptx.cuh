@@ -27,9 +27,15 @@ enum : unsigned {
 
 __device__ unsigned int g_device_status;
 
-// A single wait on an mbarrier phase gives up after this many nanoseconds of
-// wall-clock time (%globaltimer). No legitimate wait in these kernels comes close.
+// A single wait on an mbarrier phase gives up after g_wait_limit_ns nanoseconds of
+// wall-clock time (%globaltimer); no legitimate wait in these kernels comes close to
+// the default. glmq_set_wait_limit_ns() lowers it (in constant memory) so that tests
+// can make waits give up on purpose. The waits that let a CTA exit only after its own asynchronous copies and
+// MMAs have completed (the "drain" waits) always use kDrainLimitNs instead, so a lowered
+// limit never lets a CTA end with a copy into its shared memory or an MMA still in flight.
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
+constexpr unsigned long long kDrainLimitNs = 2000000000ull;  // 2 s
+__constant__ unsigned long long g_wait_limit_ns = kWaitLimitNs;
 
 __device__ __forceinline__ unsigned long long globaltimer_ns() {
   unsigned long long t;
@@ -80,15 +86,50 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking test of the phase with the given parity.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Wait for the phase with the given parity to complete. Returns false (and the
-// caller reports an error) if it does not complete within kWaitLimitNs.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+// caller reports an error) if it does not complete within the given limit. Each
+// try_wait may block in hardware for a while, so the limit is checked between tries.
+__device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity, unsigned long long limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer_ns();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+    if (globaltimer_ns() - t0 > limit_ns) return false;
   }
+}
+
+// The same wait under a lowered limit (glmq_set_wait_limit_ns): non-blocking tests, so
+// that the limit holds even for a wait the hardware would block through.
+__device__ __forceinline__ bool mbar_poll_for(uint64_t* bar, uint32_t parity, unsigned long long limit_ns) {
+  const unsigned long long t0 = globaltimer_ns();
+  while (!mbar_test_wait(bar, parity))
+    if (globaltimer_ns() - t0 > limit_ns) return false;
+  return true;
+}
+
+// A pipeline wait, limited by g_wait_limit_ns.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  const unsigned long long limit = g_wait_limit_ns;
+  if (limit < kWaitLimitNs) return mbar_poll_for(bar, parity, limit);
+  return mbar_wait_for(bar, parity, limit);
+}
+
+// A drain wait (the CTA's own copies or MMAs must complete before it exits): fixed limit.
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) {
+  return mbar_wait_for(bar, parity, kDrainLimitNs);
 }
 
 // Same wait, but each try_wait may suspend the thread in hardware (up to 20 us per
@@ -107,13 +148,23 @@ __device__ __forceinline__ bool mbar_try_wait_suspend(uint64_t* bar, uint32_t pa
   return ok != 0;
 }
 
-__device__ __forceinline__ bool mbar_wait_suspend(uint64_t* bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_wait_suspend_for(uint64_t* bar, uint32_t parity, unsigned long long limit_ns) {
   if (mbar_try_wait_suspend(bar, parity)) return true;
   const unsigned long long t0 = globaltimer_ns();
   while (true) {
     if (mbar_try_wait_suspend(bar, parity)) return true;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+    if (globaltimer_ns() - t0 > limit_ns) return false;
   }
+}
+
+__device__ __forceinline__ bool mbar_wait_suspend(uint64_t* bar, uint32_t parity) {
+  const unsigned long long limit = g_wait_limit_ns;
+  if (limit < kWaitLimitNs) return mbar_poll_for(bar, parity, limit);
+  return mbar_wait_suspend_for(bar, parity, limit);
+}
+
+__device__ __forceinline__ bool mbar_wait_drain_suspend(uint64_t* bar, uint32_t parity) {
+  return mbar_wait_suspend_for(bar, parity, kDrainLimitNs);
 }
 
 __device__ __forceinline__ bool mbar_wait_warp_suspend(uint64_t* bar, uint32_t parity) {

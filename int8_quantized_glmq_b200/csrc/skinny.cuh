@@ -141,7 +141,8 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
   uint64_t* aempty = afull + NA;          // A slot's MMAs done            (tcgen05.commit)
   uint64_t* accfull = aempty + NA;        // accumulator ready             (tcgen05.commit), x2
   uint64_t* accempty = accfull + 2;       // accumulator drained           (count 4 warps), x2
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accempty + 2);
+  uint64_t* final_bar = accempty + 2;     // all MMAs done, on the failure path (tcgen05.commit)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(final_bar + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -162,6 +163,7 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
       mbar_init(&accfull[b], 1);
       mbar_init(&accempty[b], 4);
     }
+    mbar_init(final_bar, 1);
     fence_barrier_init();
   }
   if (warp == kSkinnyMmaWarp) {
@@ -203,7 +205,7 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
       }
       bool drained = true;
       for (int s = 0; s < S; ++s)
-        if (armed[s] && !mbar_wait_suspend(&full[s], armed[s] - 1)) drained = false;
+        if (armed[s] && !mbar_wait_drain_suspend(&full[s], armed[s] - 1)) drained = false;
       if (!ok || !drained) report_error(kErrPrefillWait);
     }
   } else if (warp < kSkinnyDequantWarps) {
@@ -320,7 +322,12 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
       }
       bool drained = true;
       for (int b = 0; b < 2; ++b)
-        if (acc_armed[b] && !mbar_wait_suspend(&accfull[b], acc_armed[b] - 1)) drained = false;
+        if (acc_armed[b] && !mbar_wait_drain_suspend(&accfull[b], acc_armed[b] - 1)) drained = false;
+      if (!ok) {
+        // a wait gave up mid-unit: MMAs may have been issued after the last commit above
+        umma_commit(final_bar);
+        if (!mbar_wait_drain_suspend(final_bar, 0)) drained = false;
+      }
       if (!ok || !drained) report_error(kErrPrefillWait);
     }
   } else {

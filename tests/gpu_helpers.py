@@ -1,5 +1,15 @@
-"""Helpers for the GPU parity tests: host numpy <-> device tensors, edge-case weights."""
+"""Helpers for the GPU parity tests: host numpy <-> device tensors, edge-case weights,
+and a record of the observed GEMM errors."""
 import numpy as np
+
+#: (case, relative max error) of every GEMM parity check that records itself; written
+#: to the JSON file named by GLMQ_ERROR_REPORT at the end of the session (conftest.py)
+OBSERVED_ERRORS = []
+
+
+def record_error(case: str, err: float) -> float:
+    OBSERVED_ERRORS.append((case, float(err)))
+    return err
 
 
 def torch_cuda():

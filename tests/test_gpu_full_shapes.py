@@ -12,7 +12,7 @@ import numpy as np
 import pytest
 
 import oracle
-from gpu_helpers import to_dev, to_host, torch_cuda
+from gpu_helpers import record_error, to_dev, to_host, torch_cuda
 from inputs import GLM_PROJECTIONS, PROJECTION_ORDER, decode_activations, prefill_activations, projection_weight
 
 pytestmark = pytest.mark.gpu
@@ -69,13 +69,19 @@ def _check_gemm(projection, bits, M, seed):
     Ys = to_host(Y[:, to_dev(rows.astype(np.int64))])
     p_rows, s_rows = oracle.quantize_linear(projection["W_rows"], bits)
     Y_ref = oracle.linear_forward_rows(X, p_rows, s_rows, bits)
-    err = oracle.relative_max_error(Ys, Y_ref)
+    err = record_error(f"full/{projection['name']}/int{bits}/M={M}", oracle.relative_max_error(Ys, Y_ref))
     assert err <= TOL, err
 
 
 @pytest.mark.parametrize("M", [1, 4, 16])
 def test_decode_int4_full_projection(projection, M):
     _check_gemm(projection, 4, M, 2000 + M)
+
+
+@pytest.mark.parametrize("M", [17, 32, 64])
+def test_skinny_int4_full_projection(projection, M):
+    """16 < M <= 64: the tcgen05 skinny kernel (A operand in tensor memory)."""
+    _check_gemm(projection, 4, M, 5000 + M)
 
 
 def test_prefill_int4_full_projection(projection):

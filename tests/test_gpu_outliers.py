@@ -9,7 +9,7 @@ import numpy as np
 import pytest
 
 import oracle
-from gpu_helpers import to_dev, to_host, torch_cuda
+from gpu_helpers import record_error, to_dev, to_host, torch_cuda
 from inputs import gaussian_fp16
 from inputs.synthetic import outlier_activations
 
@@ -32,5 +32,5 @@ def test_gemm_with_outlier_activations(bits, M, N, K, route):
     Y = to_host(g.gemm(to_dev(X), to_dev(packed), to_dev(s), bits, route=route))
     ref = oracle.linear_forward(X, packed, s, bits)
     assert np.all(np.isfinite(Y))
-    err = oracle.relative_max_error(Y, ref)
+    err = record_error(f"outliers/{route}/int{bits}/M={M}/K={K}", oracle.relative_max_error(Y, ref))
     assert err <= TOL and err <= TIGHT, err

@@ -293,13 +293,22 @@ def run_decode(args, world, rank, local):
     torch.cuda.synchronize()
     cap_stream = torch.cuda.Stream()
 
-    def capture(n_steps, with_events=False, hint=True):
+    def capture(n_steps, with_events=False, hint=True, warmup=0):
+        """One CUDA graph: `warmup` untimed steps, then n_steps steps between two timing
+        events (so the graph's first-launch costs fall in the warm-up), optionally with
+        event nodes around every call of the timed steps."""
         g = torch.cuda.CUDAGraph()
         evs = [[(torch.cuda.Event(enable_timing=True, external=True),
                  torch.cuda.Event(enable_timing=True, external=True)) for _ in launches]
                for _ in range(n_steps)] if with_events else None
-        n0 = glmq.kernel_launches()
+        edge = (torch.cuda.Event(enable_timing=True, external=True),
+                torch.cuda.Event(enable_timing=True, external=True))
         with torch.cuda.graph(g, stream=cap_stream):
+            for _ in range(warmup):
+                for j in range(len(launches)):
+                    call(j, hint)
+            edge[0].record()
+            n0 = glmq.kernel_launches()
             for it in range(n_steps):
                 for j in range(len(launches)):
                     if with_events:
@@ -307,52 +316,45 @@ def run_decode(args, world, rank, local):
                     call(j, hint)
                     if with_events:
                         evs[it][j][1].record()
-        return g, evs, glmq.kernel_launches() - n0
+            n_timed = glmq.kernel_launches() - n0
+            edge[1].record()
+        return g, evs, edge, n_timed
 
-    def timed_replay(graph):
-        """Device seconds of one replay, CUDA events on the launching stream around it."""
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    def timed_replay(graph, edge):
+        """Device seconds between the graph's two timing events (one replay, bracketed by a
+        barrier and a device synchronize)."""
         barrier(world)
         torch.cuda.synchronize()
-        e0.record(stream)
         graph.replay()
-        e1.record(stream)
         torch.cuda.synchronize()
         barrier(world)
-        return e0.elapsed_time(e1) / 1e3
+        return edge[0].elapsed_time(edge[1]) / 1e3
 
     stream = torch.cuda.current_stream()
-    warm_graph, _, _ = capture(args.warmup)
-    timed_graph, _, kernels_timed = capture(args.steps)
-    warm_graph.replay()
-    torch.cuda.synchronize()
+    timed_graph, _, edge, kernels_timed = capture(args.steps, warmup=args.warmup)
 
     clocks = ClockSampler(local)
     clocks.start()
-    elapsed = timed_replay(timed_graph)
+    elapsed = timed_replay(timed_graph, edge)
     clk = clocks.stop()
     gpu_launches = kernels_timed
     value, elapsed_max = whole_job_rate(weight_bytes / 1e9, args.steps, elapsed, world)
     step_s = elapsed_max / args.steps
-    del warm_graph, timed_graph
+    del timed_graph
 
     # per-launch shares of the step (event-timed, separate graph)
-    ev_graph, ev, _ = capture(EVENT_STEPS, with_events=True)
-    ev_graph.replay()
-    torch.cuda.synchronize()
+    ev_graph, ev, ev_edge, _ = capture(EVENT_STEPS, with_events=True, warmup=args.warmup)
     ev_graph.replay()
     torch.cuda.synchronize()
     ev_s = [sum(ev[it][j][0].elapsed_time(ev[it][j][1]) for it in range(EVENT_STEPS)) / 1e3 / EVENT_STEPS
             for j in range(len(launches))]
     per_launch_s = [t / sum(ev_s) * step_s for t in ev_s]
-    del ev_graph, ev
+    del ev_graph, ev, ev_edge
 
     # the same step with plain decode calls (no next-call hint), for comparison
-    plain_graph, _, _ = capture(args.steps, hint=False)
-    plain_graph.replay()
-    torch.cuda.synchronize()
-    plain_value, _ = whole_job_rate(weight_bytes / 1e9, args.steps, timed_replay(plain_graph), world)
-    del plain_graph
+    plain_graph, _, plain_edge, _ = capture(args.steps, hint=False, warmup=args.warmup)
+    plain_value, _ = whole_job_rate(weight_bytes / 1e9, args.steps, timed_replay(plain_graph, plain_edge), world)
+    del plain_graph, plain_edge
     extras["decode_step_without_prefetch_hint_gbs"] = round(plain_value, 2)
 
     # e2e through the public API: pinned host X in, pinned host Y out, every step

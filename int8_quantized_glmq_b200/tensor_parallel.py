@@ -15,7 +15,7 @@ Quantize first, shard second: a layer is quantized once, whole, so every shard h
 exactly the codes and the per-row scales of the unsharded layer (a row-parallel
 shard keeps the full row's scale). Column-parallel results are therefore identical
 to the unsharded layer; row-parallel results differ only by the rounding of each
-rank's fp16 partial output (the partials are summed in fp32 and rounded once).
+rank's fp16 partial output and of the fp16 sums of the all-reduce.
 
 Biases (paper card, "Paper vs code": biases stay FP16) are fused into the local GEMM's
 epilogue: a column-parallel shard takes the bias entries of its own rows (for a
@@ -112,30 +112,62 @@ class ColumnParallelLinear:
         return torch.cat(parts, dim=1)
 
 
+def chunk_rows(N: int, chunks: int, align: int = 256):
+    """Row ranges [(n0, n1), ...] splitting N output rows into about `chunks` pieces whose
+    boundaries fall on multiples of `align` rows (the decode kernel's tile height)."""
+    if N <= 0:
+        return []
+    per = -(-N // max(1, chunks))
+    per = -(-per // align) * align
+    return [(n0, min(N, n0 + per)) for n0 in range(0, N, per)]
+
+
 class RowParallelLinear:
-    """Input columns [rank K/T, (rank+1) K/T) of a quantized linear layer."""
+    """Input columns [rank K/T, (rank+1) K/T) of a quantized linear layer.
+
+    forward() overlaps the reduction with the GEMM: the local GEMM runs in `chunks`
+    pieces of output rows, and each piece's all-reduce is issued (asynchronously) as
+    soon as its GEMM is enqueued, so the reduction of piece i runs while piece i+1 is
+    computed (with NCCL the collective waits only for the work already on the stream).
+    The pieces are reduced in fp16, the dtype the library writes: T - 1 fp16 roundings
+    of the partial sums, within the accuracy bar of the layer. By default decode-sized
+    inputs (M <= 16, where each piece would pay the GEMM's fixed cost) use one piece
+    and larger M four."""
 
     def __init__(self, packed, scale, bits: int, rank: int, world: int, group=None,
-                 bias=None, local: Optional[Callable] = None):
+                 bias=None, local: Optional[Callable] = None, chunks: Optional[int] = None):
         self.packed, self.scale = row_shard(packed, scale, bits, rank, world)
         self.K_local = self.packed.shape[1] * 8 // bits
         self.bias = bias if rank == 0 else None       # added once, by rank 0's epilogue
         self.bits, self.rank, self.world, self.group = bits, rank, world, group
         self.local = local or _default_local()
+        self.chunks = chunks
 
     def local_input(self, X):
         """This rank's slice of a full activation X [M, K]."""
         return X[:, self.rank * self.K_local:(self.rank + 1) * self.K_local].contiguous()
 
-    def partial(self, X_local):
-        """This rank's fp16 partial output [M, N] over its K range (rank 0 adds the bias)."""
-        return self.local(X_local, self.packed, self.scale, self.bits, self.bias, "none")
+    def partial(self, X_local, n0: int = 0, n1: Optional[int] = None):
+        """This rank's fp16 partial output [M, n1 - n0] over its K range for output rows
+        [n0, n1) (all rows by default); rank 0 adds the bias."""
+        n1 = self.packed.shape[0] if n1 is None else n1
+        bias = None if self.bias is None else self.bias[n0:n1]
+        return self.local(X_local, self.packed[n0:n1], self.scale[n0:n1], self.bits, bias, "none")
 
-    def forward(self, X_local):
-        """Y [M, N] on every rank: the fp16 partial outputs summed in fp32, rounded once."""
-        Y = self.partial(X_local)
+    def forward(self, X_local, chunks: Optional[int] = None):
+        """Y [M, N] on every rank: the fp16 partial outputs summed by the all-reduce."""
         if self.world == 1:
-            return Y
-        acc = Y.float()
-        _dist().all_reduce(acc, group=self.group)
-        return acc.half()
+            return self.partial(X_local)
+        M = X_local.shape[0]
+        n = chunks or self.chunks or (1 if M <= 16 else 4)
+        pieces, works = [], []
+        for n0, n1 in chunk_rows(self.packed.shape[0], n):
+            Y = self.partial(X_local, n0, n1)
+            works.append(_dist().all_reduce(Y, group=self.group, async_op=True))
+            pieces.append(Y)
+        for w in works:
+            w.wait()
+        if len(pieces) == 1:
+            return pieces[0]
+        import torch
+        return torch.cat(pieces, dim=1)

@@ -4,8 +4,9 @@ with the library's GEMM as the local step, through the C ABI.
 The GLM-130B paper card ("Paper vs code") runs the INT4 model 4-way model-parallel.
 With one GPU the four ranks are emulated one after another, each running its own
 shard: no collective runs and no kernel waits on another. The host concatenates the
-column-parallel outputs and sums the row-parallel partials in fp32, which is what the
-all-gather and the all-reduce compute (those two are covered by the gloo tests on CPU).
+column-parallel outputs and sums the row-parallel partials, which is what the
+all-gather and the all-reduce compute (the collectives themselves, and the fp16
+rounding of the reduction, are covered by the gloo tests on CPU).
 """
 import numpy as np
 import pytest
@@ -124,3 +125,22 @@ def test_glm_qkv_column_parallel_int4(M):
         pn, sn = oracle.quantize_linear(W[r * n + rows], 4)
         got = to_host(Y[:, to_dev(rows.astype(np.int64))])
         assert oracle.relative_max_error(got, oracle.linear_forward(X, pn, sn, 4)) <= TOL
+
+
+@pytest.mark.parametrize("M", [1, 20])
+def test_row_parallel_pieces_match_the_whole_partial(M):
+    """The overlapped forward runs the local GEMM in pieces of output rows (chunk_rows):
+    each piece, computed through the C ABI on its row slice of the shard, matches the
+    columns of the whole partial (up to the fp32 summation order of a different K split)."""
+    g, tp = modules()
+    N, K = 1536, 2048
+    W = gaussian_fp16((N, K), 0.02, 900 + M)
+    X = gaussian_fp16((M, K), 1.0, 910 + M)
+    p, s = g.quantize(to_dev(W), 4)
+    layer = tp.RowParallelLinear(p, s, 4, 1, T)
+    Xl = layer.local_input(to_dev(X))
+    whole = to_host(layer.partial(Xl))
+    pieces = tp.chunk_rows(N, 4)
+    assert len(pieces) > 1
+    for n0, n1 in pieces:
+        assert oracle.relative_max_error(to_host(layer.partial(Xl, n0, n1)), whole[:, n0:n1]) <= 1e-3

@@ -141,17 +141,26 @@ def _rank_main(rank, world, port, out_q):
     os.environ["MASTER_PORT"] = str(port)
     dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
     try:
-        N, K = 128, 512
-        p, s, _, _ = _layer(N, K, 4, 61)
-        b = torch.from_numpy(gaussian_fp16((1, N), 0.5, 62)[0])
-        X = torch.from_numpy(gaussian_fp16((3, K), 1.0, 63))
-        col = tp.ColumnParallelLinear(p, s, 4, rank, world, bias=b, local=oracle_local)
-        Yc = col.forward(X, gather=True)
-        row = tp.RowParallelLinear(p, s, 4, rank, world, bias=b, local=oracle_local)
-        Yr = row.forward(row.local_input(X))
-        out_q.put((rank, Yc.numpy(), Yr.numpy()))
+        out = {}
+        for N, M in ((128, 3), (768, 20)):        # 768 rows at M = 20: three overlapped row pieces
+            K = 512
+            p, s, _, _ = _layer(N, K, 4, 61 + N)
+            b = torch.from_numpy(gaussian_fp16((1, N), 0.5, 62 + N)[0])
+            X = torch.from_numpy(gaussian_fp16((M, K), 1.0, 63 + N))
+            col = tp.ColumnParallelLinear(p, s, 4, rank, world, bias=b, local=oracle_local)
+            row = tp.RowParallelLinear(p, s, 4, rank, world, bias=b, local=oracle_local)
+            out[N] = (col.forward(X, gather=True).numpy(), row.forward(row.local_input(X)).numpy())
+        out_q.put((rank, out))
     finally:
         dist.destroy_process_group()
+
+
+def test_chunk_rows():
+    assert tp.chunk_rows(768, 4) == [(0, 256), (256, 512), (512, 768)]
+    assert tp.chunk_rows(12288, 4) == [(0, 3072), (3072, 6144), (6144, 9216), (9216, 12288)]
+    assert tp.chunk_rows(300, 4) == [(0, 256), (256, 300)]
+    assert tp.chunk_rows(100, 1) == [(0, 100)]
+    assert tp.chunk_rows(0, 4) == []
 
 
 @pytest.mark.parametrize("world", [2, 4])           # 4: the INT4 model's 4-way split
@@ -171,20 +180,28 @@ def test_gloo_ranks_gather_and_reduce(world):
             pytest.fail("a rank did not finish")
         assert pr.exitcode == 0
 
-    N, K = 128, 512
-    W = gaussian_fp16((N, K), 0.02, 61)
-    pn, sn = oracle.quantize_linear(W, 4)
-    b = gaussian_fp16((1, N), 0.5, 62)[0]
-    X = gaussian_fp16((3, K), 1.0, 63)
-    ref = oracle.linear_bias_forward(X, pn, sn, 4, b)
-    # the reduced result, computed here from the ranks' fp16 partials (rank 0 adds the bias)
-    kl = K // world
-    acc = oracle.linear_bias_forward(X[:, :kl], pn[:, :kl // 2], sn, 4, b).astype(np.float32)
-    for r in range(1, world):
-        acc += oracle.linear_forward(X[:, r * kl:(r + 1) * kl], pn[:, r * kl // 2:(r + 1) * kl // 2], sn,
-                                     4).astype(np.float32)
-    expect_row = acc.astype(np.float16)
-    for _, Yc, Yr in got:
-        assert np.array_equal(Yc.view(np.uint16), ref.view(np.uint16))        # column: identical
-        assert np.array_equal(Yr.view(np.uint16), expect_row.view(np.uint16))  # row: fp32 sum of partials
-        assert oracle.relative_max_error(Yr, ref) <= 5e-3
+    for N, M in ((128, 3), (768, 20)):
+        K = 512
+        W = gaussian_fp16((N, K), 0.02, 61 + N)
+        pn, sn = oracle.quantize_linear(W, 4)
+        b = gaussian_fp16((1, N), 0.5, 62 + N)[0]
+        X = gaussian_fp16((M, K), 1.0, 63 + N)
+        ref = oracle.linear_bias_forward(X, pn, sn, 4, b)
+        # the ranks' fp16 partials (rank 0 adds the bias), as the oracle computes them
+        kl = K // world
+        parts = [oracle.linear_bias_forward(X[:, :kl], pn[:, :kl // 2], sn, 4, b)]
+        parts += [oracle.linear_forward(X[:, r * kl:(r + 1) * kl], pn[:, r * kl // 2:(r + 1) * kl // 2], sn, 4)
+                  for r in range(1, world)]
+        exact = np.sum([pt.astype(np.float64) for pt in parts], axis=0)
+        for _, out in got:
+            Yc, Yr = out[N]
+            assert np.array_equal(Yc.view(np.uint16), ref.view(np.uint16))        # column: identical
+            assert oracle.relative_max_error(Yr, ref) <= 5e-3
+            if world == 2:
+                # one fp16 rounding of the sum of the two partials (exact in fp32)
+                two = (parts[0].astype(np.float32) + parts[1].astype(np.float32)).astype(np.float16)
+                assert np.array_equal(Yr.view(np.uint16), two.view(np.uint16))
+            else:
+                # world - 1 fp16 roundings of partial sums, in the collective's order
+                bound = (world - 1) * 2.0 ** -11 * np.abs(exact).max() * 2
+                assert np.abs(Yr.astype(np.float64) - exact).max() <= bound

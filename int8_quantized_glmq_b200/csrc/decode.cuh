@@ -17,15 +17,19 @@
 //    (32 KB), the matching activations of the MP token rows (in the order the
 //    MMA fragments read them) and a per-token bias for the biased dequantization.
 //    The ring has kStages stages (5 or 6, whatever fits in shared memory).
-//  * Warp 16 is the weight producer: one lane issues, per stage, one 2-D TMA tile
-//    load of the weight box (128-byte swizzle, L2 evict-first hint). Rows past N and
-//    bytes past K are zero-filled by the TMA unit.
-//  * Warps 17..19 are activation producers: warp 17 + i fills the activation slot of
-//    every third stage (sequence number i mod 3), reading X[:, k0 : k0 + 256] from
-//    global memory (it is small and L2-resident), permuting it into fragment order,
-//    dividing the high-nibble slots by 16 (see below) and summing the
-//    per-token bias. Three of them keep several stages in flight, so the L2 latency of
-//    one warp is hidden behind the others.
+//  * Warp 16 is the producer: one lane issues, per stage, two 2-D TMA tile loads:
+//    the stage's activations X[0 : MP, k0 : k0 + SK] (rows past M and values past K
+//    are zero-filled by the TMA unit) into the stage's activation slot, and the weight
+//    box (128-byte swizzle, L2 evict-first hint; rows past N and bytes past K
+//    zero-filled).
+//  * Warps 17.. are activation warps (one for M <= 2, three for larger M; warp 17 + i
+//    takes the stages with sequence number i mod their count). Once a slot's raw
+//    activations have landed the warp
+//    rewrites them in place into fragment order, dividing the high-nibble slots by 16
+//    (see below), with a lane-to-unit mapping under which both the reads and the
+//    writes of shared memory are free of bank conflicts; the per-token bias of the
+//    stage is then one short MMA chain on the slot's fragments (for M <= 2, where most
+//    of that chain's columns would be padding, a warp reduction of the lanes' sums).
 //  * Warps 0..15 are consumers: warp w owns rows 16w .. 16w+15 of the tile and
 //    reads the whole stage's K segment for them. Codes are dequantized in
 //    registers with exponent-bias tricks (a code c becomes the fp16 number
@@ -54,11 +58,19 @@
 
 namespace glmq {
 
+#ifndef DECODE_WAIT_P
+#define DECODE_WAIT_P mbar_wait
+#endif
+#ifndef DECODE_WAIT_X
+#define DECODE_WAIT_X mbar_wait_warp
+#endif
+#ifndef DECODE_WAIT_C
+#define DECODE_WAIT_C mbar_wait_warp
+#endif
+
 constexpr int kDecodeConsumerWarps = 16;
 constexpr int kDecodeProducerWarp = 16;                               // weight TMA
-constexpr int kDecodeXWarp0 = 17;                                     // activation producers 17..19
-constexpr int kDecodeXWarps = 3;   // 20 warps in all: ptxas then allows 96 registers per thread
-constexpr int kDecodeThreads = (kDecodeConsumerWarps + 1 + kDecodeXWarps) * 32;
+constexpr int kDecodeXWarp0 = 17;                                     // activation warps 17..
 constexpr int kDecodeRows = 16 * kDecodeConsumerWarps;                // rows per tile (256)
 constexpr int kDecodeSegB = 128;         // packed bytes per row per stage (one TMA box width)
 constexpr int kDecodeStageBytes = kDecodeRows * kDecodeSegB;          // 32 KB: one TMA box per stage
@@ -87,12 +99,16 @@ struct DecodeCfg {
   static constexpr int TW = TB / 4;                 // 32-bit words per thread per row per stage (8)
   static constexpr int XU = TK / 8;                 // 16-byte activation units per thread per stage
   static constexpr int kChains = CHAINS;            // independent MMA accumulator chains per token block
+  // activation warps: one keeps up with the small slots of M <= 2; three for M >= 4 (at
+  // most 20 warps in all, so ptxas still allows 96 registers per thread)
+  static constexpr int kXWarps = MP >= 4 ? 3 : 1;
+  static constexpr int kThreads = (kDecodeConsumerWarps + 1 + kXWarps) * 32;
   static constexpr int X_UNITS = XU * MP * 4;       // 16-byte units in a stage's activation slot
   static constexpr int X_BYTES = X_UNITS * 16;
   // per stage and token: the bias of the biased dequantization (INT4), then (zero point)
   // the sum of x over the stage
   static constexpr int B_FLOATS = ZP ? 32 : 16;
-  static constexpr int STAGE_TOTAL = kDecodeStageBytes + X_BYTES + B_FLOATS * 4 + 3 * 8;
+  static constexpr int STAGE_TOTAL = kDecodeStageBytes + X_BYTES + B_FLOATS * 4 + 4 * 8;
   static constexpr int kStages = (kDecodeSmemLimit - 1024) / STAGE_TOTAL < kDecodeMaxStages
                                      ? (kDecodeSmemLimit - 1024) / STAGE_TOTAL : kDecodeMaxStages;
   static constexpr int SMEM_BYTES = kStages * STAGE_TOTAL + 1024;   // + alignment slack
@@ -255,79 +271,145 @@ __device__ __forceinline__ void decode_segment(uint32_t box, uint32_t xseg, uint
 }
 
 
-// Fills one stage's activation slot (and bias slot) for the k range [k0, k0 + SK) of
-// X, called by all 32 lanes of an activation-producer warp. Lane L serves token
-// n = L / (32 / MP); the 32 / MP lanes of a token split its units between them and
-// combine their bias sums with shuffles. Each unit: 8 consecutive values of X,
+// Rewrites one stage's activation slot in place, called by all 32 lanes of an
+// activation warp once the slot's raw activations have landed. Raw layout (the TMA
+// box): token n's SK values at n * SK * 2 bytes, i.e. 16-byte unit (n, kr / 8) for the
+// 8 values from k0 + kr. Fragment layout: unit x_unit(jj, n, c) holds the 8 values lane
+// c multiplies with its codes jj*8 .. jj*8+7, i.e. kr = c * TK + jj * 8; INT4 values are
 // permuted to the MMA k order (0,4),(1,5),(2,6),(3,7) with the high-nibble slots (1,5)
-// and (3,7) divided by 16 (exact: a power of two); INT8 keeps the natural order.
-// Units of tokens >= M are not written (no fragment of a real token reads them);
-// values past K are written as zero.
+// and (3,7) divided by 16 (exact: a power of two); INT8 values keep their order.
+// Every lane first reads all its units, the warp synchronizes, then every lane writes
+// them back, so the permutation can be done in place. Lane (p, l) = (L / 8, L % 8)
+// handles, for its i-th unit, jj = l (INT4) and a rotation of the remaining indices by
+// (i, p), chosen so that within each 8-lane phase of a 16-byte access the raw units
+// read fall in 8 distinct bank groups (distinct raw unit index mod 8) and so do the
+// fragment units written (distinct (4n + c) mod 8).
+// Unit (jj, n, c) of lane `lane`'s i-th unit in transform_activation_stage.
 template <class C>
-__device__ __forceinline__ void fill_activation_stage(const __half* __restrict__ X, int K, int M, int k0,
-                                                      uint8_t* xslot, float* bslot, int lane) {
-  constexpr int LPT = 32 / C::kMP;          // lanes per token
-  constexpr int UPT = C::XU * 4;            // units per token
-  const int n = lane / LPT;
-  const int sub = lane - n * LPT;
-  float bias = 0.0f, sx = 0.0f;
-  if (n < M) {
-    const __half* xrow = X + static_cast<long long>(n) * K + k0;
-    uint4 v[(UPT + LPT - 1) / LPT];
-#pragma unroll
-    for (int i = 0; i < (UPT + LPT - 1) / LPT; ++i) {
-      const int r = sub + i * LPT;
-      const int kr = (r & 3) * C::TK + (r >> 2) * 8;
-      v[i] = make_uint4(0, 0, 0, 0);
-      if (r < UPT && k0 + kr < K) v[i] = __ldg(reinterpret_cast<const uint4*>(xrow + kr));
+__device__ __forceinline__ void transform_unit(int i, int lane, int& jj, int& n, int& c) {
+  constexpr int MP = C::kMP;
+  const int p = lane >> 3, l = lane & 7;
+  if constexpr (C::kBits == 4) {
+    if constexpr (MP == 1) {
+      jj = lane & 7; n = 0; c = lane >> 3;
+    } else {
+      const int z = i * 4 + p, q = (l + (z & 7)) & 7;
+      jj = l; n = 2 * (z >> 3) + (q >> 2); c = q & 3;
     }
-#pragma unroll
-    for (int i = 0; i < (UPT + LPT - 1) / LPT; ++i) {
-      const int r = sub + i * LPT;
-      if (r >= UPT) continue;
-      uint4 o;
-      if constexpr (C::kBits == 4) {
-        const __half2 kSixteenth = __halves2half2(__ushort_as_half(0x2C00), __ushort_as_half(0x2C00));
-        o.x = prmt(v[i].x, v[i].z, 0x5410u);
-        uint32_t hy = prmt(v[i].x, v[i].z, 0x7632u);
-        o.z = prmt(v[i].y, v[i].w, 0x5410u);
-        uint32_t hw = prmt(v[i].y, v[i].w, 0x7632u);
-        __half2 sy = __hmul2(*reinterpret_cast<__half2*>(&hy), kSixteenth);
-        __half2 sw = __hmul2(*reinterpret_cast<__half2*>(&hw), kSixteenth);
-        o.y = *reinterpret_cast<uint32_t*>(&sy);
-        o.w = *reinterpret_cast<uint32_t*>(&sw);
-        const float2 fx = __half22float2(*reinterpret_cast<const __half2*>(&o.x));
-        const float2 fy = __half22float2(*reinterpret_cast<const __half2*>(&o.y));
-        const float2 fz = __half22float2(*reinterpret_cast<const __half2*>(&o.z));
-        const float2 fw = __half22float2(*reinterpret_cast<const __half2*>(&o.w));
-        const float lo = (fx.x + fx.y) + (fz.x + fz.y);
-        const float hi = (fy.x + fy.y) + (fw.x + fw.y);
-        bias += C::kLowBias * lo + C::kHighBias * hi;
-        if constexpr (C::kZP) sx += lo + 16.0f * hi;
-      } else {
-        o = v[i];
-      }
-      *reinterpret_cast<uint4*>(xslot + 16u * x_unit<C>(r >> 2, n, r & 3)) = o;
+  } else {
+    if constexpr (MP == 1) {
+      jj = lane & 3; n = 0; c = (lane >> 2) & 3;
+    } else {
+      const int z = i * 4 + p, w = ((l & 3) + (z & 3)) & 3;
+      jj = l & 3; n = 2 * (z >> 2) + (w >> 1); c = 2 * (w & 1) + (l >> 2);
     }
   }
-  if constexpr (C::kBits == 4) {
+}
+
+template <class C>
+__device__ __forceinline__ void transform_activation_stage(uint32_t slot, int lane, float (&bsum)[2],
+                                                           float (&ssum)[2]) {
+  constexpr int MP = C::kMP;
+  constexpr int RAW_UNITS = C::SK / 8;                    // 16-byte units per token row
+  constexpr int PER = (C::kBits == 4) ? MP : (MP == 1 ? 1 : MP / 2);
+  const bool live = !(C::kBits == 8 && MP == 1) || lane < 16;
+  uint4 v[PER];
 #pragma unroll
-    for (int off = LPT / 2; off > 0; off >>= 1) {
-      bias += __shfl_xor_sync(0xffffffffu, bias, off);
-      if constexpr (C::kZP) sx += __shfl_xor_sync(0xffffffffu, sx, off);
+  for (int i = 0; i < PER; ++i) {
+    int jj, n, c;
+    transform_unit<C>(i, lane, jj, n, c);
+    if (live) v[i] = lds_v4(slot + 16u * static_cast<uint32_t>(n * RAW_UNITS + (c * C::TK + jj * 8) / 8));
+  }
+  __syncwarp();
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    int jj, n, c;
+    transform_unit<C>(i, lane, jj, n, c);
+    uint4 o = v[i];
+    if constexpr (C::kBits == 4) {
+      const __half2 kSixteenth = __halves2half2(__ushort_as_half(0x2C00), __ushort_as_half(0x2C00));
+      o.x = prmt(v[i].x, v[i].z, 0x5410u);
+      uint32_t hy = prmt(v[i].x, v[i].z, 0x7632u);
+      o.z = prmt(v[i].y, v[i].w, 0x5410u);
+      uint32_t hw = prmt(v[i].y, v[i].w, 0x7632u);
+      __half2 sy = __hmul2(*reinterpret_cast<__half2*>(&hy), kSixteenth);
+      __half2 sw = __hmul2(*reinterpret_cast<__half2*>(&hw), kSixteenth);
+      o.y = *reinterpret_cast<uint32_t*>(&sy);
+      o.w = *reinterpret_cast<uint32_t*>(&sw);
     }
-    if (sub == 0 && n < M) {
-      bslot[n] = bias;
-      if constexpr (C::kZP) bslot[16 + n] = sx;
+    if (live) sts_v4(slot + 16u * x_unit<C>(jj, n, c), o);
+    if constexpr (C::kBits == 4 && MP <= 2) {
+      // this unit's share of the token's bias (and sum of x): see stage_sums_mma
+      const float2 fx = __half22float2(*reinterpret_cast<const __half2*>(&o.x));
+      const float2 fy = __half22float2(*reinterpret_cast<const __half2*>(&o.y));
+      const float2 fz = __half22float2(*reinterpret_cast<const __half2*>(&o.z));
+      const float2 fw = __half22float2(*reinterpret_cast<const __half2*>(&o.w));
+      const float lo = (fx.x + fx.y) + (fz.x + fz.y), hi = (fy.x + fy.y) + (fw.x + fw.y);
+      const float b = C::kLowBias * lo + C::kHighBias * hi, sx = lo + 16.0f * hi;
+      bsum[0] += n == 0 ? b : 0.0f;
+      bsum[1] += n == 1 ? b : 0.0f;
+      ssum[0] += n == 0 ? sx : 0.0f;
+      ssum[1] += n == 1 ? sx : 0.0f;
+    }
+  }
+}
+
+// INT4: the per-token sums a stage's activation slot needs, written into its bias slot:
+// bias[t] = sum_k (kLowBias or kHighBias) * B[k][t] over the stage (what the biased
+// dequantization adds to every output of token t), and, for zero-point codes,
+// sx[t] = sum_k x[t,k] (B holds x in low-nibble slots, x / 16 in high ones). They are
+// computed on the tensor cores with the same fragments the consumers read: a constant
+// A operand whose rows 0..7 hold the bias coefficients of each slot and rows 8..15
+// the sum-of-x coefficients (1 low, 16 high), times the slot's B fragments. Row 0 of
+// the product holds bias[t] and row 8 sx[t] for the 8 tokens of each n8 block. Called
+// by all 32 lanes of the warp after the slot is written and the warp synchronized.
+template <class C>
+__device__ __forceinline__ void stage_sums_mma(uint32_t xslot_u32, float* bslot, int M, int lane) {
+  constexpr uint32_t kJStride = static_cast<uint32_t>(C::kMP) * 64u;
+  const __half2 lo = __float2half2_rn(C::kLowBias), hi = __float2half2_rn(C::kHighBias);
+  const __half2 one = __float2half2_rn(1.0f), sixteen = __float2half2_rn(16.0f);
+  const uint32_t a0 = *reinterpret_cast<const uint32_t*>(&lo), a2 = *reinterpret_cast<const uint32_t*>(&hi);
+  const uint32_t a1 = *reinterpret_cast<const uint32_t*>(&one), a3 = *reinterpret_cast<const uint32_t*>(&sixteen);
+  const int r = lane >> 2, c = lane & 3;
+  // four independent accumulator chains per n8 block keep the chain latency short
+  float d[C::kNB][4][4];
+#pragma unroll
+  for (int nb = 0; nb < C::kNB; ++nb)
+#pragma unroll
+    for (int h = 0; h < 4; ++h)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) d[nb][h][i] = 0.0f;
+#pragma unroll
+  for (int j = 0; j < C::XU; ++j) {
+#pragma unroll
+    for (int nb = 0; nb < C::kNB; ++nb) {
+      const uint4 bf = lds_v4(xslot_u32 + 16u * x_unit<C>(0, min(8 * nb + r, M - 1), c) + j * kJStride);
+      mma_16816(d[nb][2 * (j & 1)], a0, a1, a2, a3, bf.x, bf.y);
+      mma_16816(d[nb][2 * (j & 1) + 1], a0, a1, a2, a3, bf.z, bf.w);
+    }
+  }
+#pragma unroll
+  for (int nb = 0; nb < C::kNB; ++nb) {
+    float dd[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) dd[i] = (d[nb][0][i] + d[nb][1][i]) + (d[nb][2][i] + d[nb][3][i]);
+    const int t = 8 * nb + 2 * c;
+    if (r == 0 && t < M) {
+      bslot[t] = dd[0];
+      if constexpr (C::kZP) bslot[16 + t] = dd[2];
+    }
+    if (r == 0 && t + 1 < M) {
+      bslot[t + 1] = dd[1];
+      if constexpr (C::kZP) bslot[16 + t + 1] = dd[3];
     }
   }
 }
 
 // ---------------------------------------------------------------- the kernel
 template <class C>
-__global__ void __launch_bounds__(kDecodeThreads, 1)
-    decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_next,
-                  const DecodeArgs a) {
+__global__ void __launch_bounds__(C::kThreads, 1)
+    decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
+                  const __grid_constant__ CUtensorMap tmap_next, const DecodeArgs a) {
   constexpr int S = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -335,7 +417,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   uint8_t* xring = smem + S * kDecodeStageBytes;                   // S activation slots
   float* bring = reinterpret_cast<float*>(xring + S * C::X_BYTES); // S bias slots
   uint64_t* fullw = reinterpret_cast<uint64_t*>(bring + S * C::B_FLOATS);   // weight box landed (1 + tx)
-  uint64_t* fullx = fullw + S;                                     // activation slot written (1)
+  uint64_t* fullr = fullw + S;                                     // raw activations landed (1 + tx)
+  uint64_t* fullx = fullr + S;                                     // activation slot rewritten (1)
   uint64_t* empty = fullx + S;                                     // stage released (16 consumer warps)
 
   const int warp = threadIdx.x >> 5;
@@ -348,13 +431,14 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(&fullw[s], 1);
+      mbar_init(&fullr[s], 1);
       mbar_init(&fullx[s], 1);
       mbar_init(&empty[s], kDecodeConsumerWarps);
     }
     fence_barrier_init();
   }
   // bias slots of tokens no activation producer writes (M <= token < 16) read as zero
-  for (int i = threadIdx.x; i < S * C::B_FLOATS; i += kDecodeThreads) bring[i] = 0.0f;
+  for (int i = threadIdx.x; i < S * C::B_FLOATS; i += C::kThreads) bring[i] = 0.0f;
   __syncthreads();
   // everything above touches only shared memory; X, W, Y and the scratch may belong
   // to the previous kernel in the stream
@@ -376,11 +460,14 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         const int plen = min(a.KPP, K - pk0);
         const int nst = (plen + C::SK - 1) / C::SK;
         for (int ks = 0; ks < nst; ++ks) {
-          if (!mbar_wait(&empty[stage], phase ^ 1)) { ok = false; break; }
-          const int xb0 = (pk0 + ks * C::SK) / C::KPB;            // first packed byte of the stage
+          if (!DECODE_WAIT_P(&empty[stage], phase ^ 1)) { ok = false; break; }
+          const int k0 = pk0 + ks * C::SK;
+          mbar_arrive_expect_tx(&fullr[stage], static_cast<uint32_t>(C::X_BYTES));
+          tma_load_2d(xring + stage * C::X_BYTES, &tmap_x, k0, 0, &fullr[stage]);
           mbar_arrive_expect_tx(&fullw[stage], static_cast<uint32_t>(kDecodeStageBytes));
           armed[stage] = phase + 1;
-          tma_load_2d_hint(wring + stage * kDecodeStageBytes, &tmap_w, xb0, t * kDecodeRows, &fullw[stage], pol);
+          tma_load_2d_hint(wring + stage * kDecodeStageBytes, &tmap_w, k0 / C::KPB, t * kDecodeRows, &fullw[stage],
+                           pol);
           if (++stage == S) { stage = 0; phase ^= 1; }
         }
       }
@@ -407,7 +494,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       // never leave while TMA writes into this CTA's shared memory may be in flight
       bool drained = true;
       for (int s = 0; s < S; ++s)
-        if (armed[s] && !mbar_wait_drain(&fullw[s], armed[s] - 1)) drained = false;
+        if (armed[s] && (!mbar_wait_drain(&fullw[s], armed[s] - 1) || !mbar_wait_drain(&fullr[s], armed[s] - 1)))
+          drained = false;
       if (!ok || !drained) report_error(kErrDecodeProducerWait);
     }
     return;
@@ -424,13 +512,34 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       const int plen = min(a.KPP, K - pk0);
       const int nst = (plen + C::SK - 1) / C::SK;
       for (int ks = 0; ks < nst; ++ks, ++q) {
-        if (q % kDecodeXWarps != xw) continue;
+        if (C::kXWarps > 1 && q % C::kXWarps != xw) continue;
         const int stage = q % S;
         const uint32_t phase = static_cast<uint32_t>(q / S) & 1u;
-        if (!mbar_wait_warp(&empty[stage], phase ^ 1)) { ok = false; break; }
-        fill_activation_stage<C>(a.X, K, M, pk0 + ks * C::SK, xring + stage * C::X_BYTES, bring + stage * C::B_FLOATS,
-                                 lane);
+        if (!DECODE_WAIT_X(&fullr[stage], phase)) { ok = false; break; }
+        const uint32_t slot = smem_u32(xring + stage * C::X_BYTES);
+        float bsum[2] = {0.0f, 0.0f}, ssum[2] = {0.0f, 0.0f};
+        transform_activation_stage<C>(slot, lane, bsum, ssum);
         __syncwarp();
+        if constexpr (C::kBits == 4 && C::kMP <= 2) {
+          float* bs = bring + stage * C::B_FLOATS;
+#pragma unroll
+          for (int t = 0; t < C::kMP; ++t) {
+            float b = bsum[t], sx = ssum[t];
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+              b += __shfl_xor_sync(0xffffffffu, b, off);
+              if constexpr (C::kZP) sx += __shfl_xor_sync(0xffffffffu, sx, off);
+            }
+            if (lane == 0) {
+              bs[t] = b;
+              if constexpr (C::kZP) bs[16 + t] = sx;
+            }
+          }
+          __syncwarp();
+        } else if constexpr (C::kBits == 4) {
+          stage_sums_mma<C>(slot, bring + stage * C::B_FLOATS, M, lane);
+          __syncwarp();
+        }
         if (lane == 0) mbar_arrive(&fullx[stage]);
       }
     }
@@ -472,7 +581,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
 
     const int nst = (plen + C::SK - 1) / C::SK;
     for (int ks = 0; ks < nst; ++ks) {
-      if (!mbar_wait_warp(&fullx[stage], phase) || !mbar_wait_warp(&fullw[stage], phase)) { ok = false; break; }
+      if (!DECODE_WAIT_C(&fullx[stage], phase) || !DECODE_WAIT_C(&fullw[stage], phase)) { ok = false; break; }
       const uint32_t box = wring_u32 + stage * kDecodeStageBytes;
       const uint32_t xseg = xring_u32 + stage * C::X_BYTES;
       const float* bias_seg = bring + stage * C::B_FLOATS;

@@ -388,6 +388,11 @@ glmq_status launch_decode_cfg(const DeviceInfo& dev, const void* X, int M, const
   glmq_status st = make_map_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, packed, row_bytes, N, row_bytes, kDecodeSegB,
                                kDecodeRows, CU_TENSOR_MAP_SWIZZLE_128B);
   if (st != GLMQ_OK) return st;
+  // the activations: box of SK values x MP token rows (rows past M read as zero)
+  CUtensorMap tx;
+  st = make_map_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, X, K, M, uint64_t(K) * 2, C::SK, C::kMP,
+                   CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (st != GLMQ_OK) return st;
   // next-call hint: the same map and plan the next decode call will use
   CUtensorMap tn = tw;
   DecodePlan npl = {};
@@ -421,7 +426,7 @@ glmq_status launch_decode_cfg(const DeviceInfo& dev, const void* X, int M, const
   a.nxt_stages = npl.stages;
   if (pl.parts > 1 && (st = decode_scratch(static_cast<size_t>(M) * N, &a.ws)) != GLMQ_OK) return st;
   if ((st = allow_smem(decode_kernel<C>, pl.smem)) != GLMQ_OK) return st;
-  if ((st = launch_pdl(decode_kernel<C>, dim3(pl.grid), dim3(kDecodeThreads), pl.smem, s, tw, tn, a)) != GLMQ_OK)
+  if ((st = launch_pdl(decode_kernel<C>, dim3(pl.grid), dim3(C::kThreads), pl.smem, s, tw, tx, tn, a)) != GLMQ_OK)
     return st;
   if (pl.parts > 1) {
     st = (e.bias || e.geglu) ? launch_finalize_epi(a.ws, a.scale, e, a.Y, M, N, s)
@@ -608,6 +613,10 @@ glmq_status launch_decode_noalloc_cfg(const DeviceInfo& dev, const void* X, int 
   glmq_status st = make_map_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, packed, row_bytes, N, row_bytes, kDecodeSegB,
                                kDecodeRows, CU_TENSOR_MAP_SWIZZLE_128B);
   if (st != GLMQ_OK) return st;
+  CUtensorMap tx;
+  st = make_map_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, X, K, M, uint64_t(K) * 2, C::SK, C::kMP,
+                   CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (st != GLMQ_OK) return st;
   DecodeArgs a;
   a.X = static_cast<const __half*>(X);
   a.scale = static_cast<const __half*>(scale);
@@ -635,7 +644,7 @@ glmq_status launch_decode_noalloc_cfg(const DeviceInfo& dev, const void* X, int 
       return cuda_fail(e);
   }
   if ((st = allow_smem(decode_kernel<C>, pl.smem)) != GLMQ_OK) return st;
-  if ((st = launch_pdl(decode_kernel<C>, dim3(pl.grid), dim3(kDecodeThreads), pl.smem, s, tw, tw, a)) != GLMQ_OK)
+  if ((st = launch_pdl(decode_kernel<C>, dim3(pl.grid), dim3(C::kThreads), pl.smem, s, tw, tx, tw, a)) != GLMQ_OK)
     return st;
   if (pl.parts > 1) {
     if ((st = launch_finalize(a.ws, a.scale, a.Y, M, N, s)) != GLMQ_OK) return st;

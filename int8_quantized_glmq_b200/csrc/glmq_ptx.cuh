@@ -206,6 +206,15 @@ __device__ __forceinline__ uint64_t policy_evict_first() {
   return p;
 }
 
+// 2-D TMA tile load (no multicast) whose completion is counted on an mbarrier.
+__device__ __forceinline__ void tma_load_2d(void* smem_dst, const void* map, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+      "[%4];" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
 // L2 prefetch of a contiguous global range (a hint: nothing waits for it). Address
 // 16-byte aligned, size a multiple of 16.
 __device__ __forceinline__ void bulk_prefetch_l2(const void* gmem, uint32_t bytes) {
@@ -237,6 +246,11 @@ __device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
   return v;
 }
 
+__device__ __forceinline__ void sts_v4(uint32_t addr, const uint4 v) {
+  asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
+}
+
 __device__ __forceinline__ uint4 lds_v4(uint32_t addr) {
   uint4 v;
   asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
@@ -248,6 +262,13 @@ __device__ __forceinline__ uint32_t lop3_and_xor(uint32_t a, uint32_t b, uint32_
   // (a & b) ^ c
   uint32_t d;
   asm("lop3.b32 %0, %1, %2, %3, 0x6a;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
+__device__ __forceinline__ uint32_t lop3_sel(uint32_t a, uint32_t b, uint32_t m) {
+  // (a & m) | (b & ~m)
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0xe4;" : "=r"(d) : "r"(a), "r"(b), "r"(m));
   return d;
 }
 

@@ -58,35 +58,70 @@ __device__ __forceinline__ int exact_code(float w, float sf, float kf) {
   return exact_code_d<(1 << (BITS - 1)) - 1>(w, sf, kf);
 }
 
+// Packed fp32 pairs (sm_100 f32x2 arithmetic): one instruction does two IEEE fp32
+// operations, each rounded to nearest even exactly as the scalar instruction.
+__device__ __forceinline__ float2 fma2_rn(float2 a, float2 b, float2 c) {
+  unsigned long long d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;"
+      : "=l"(d)
+      : "l"(*reinterpret_cast<unsigned long long*>(&a)), "l"(*reinterpret_cast<unsigned long long*>(&b)),
+        "l"(*reinterpret_cast<unsigned long long*>(&c)));
+  return *reinterpret_cast<float2*>(&d);
+}
+
+__device__ __forceinline__ float2 sub2_rn(float2 a, float2 b) {
+  unsigned long long d;
+  asm("sub.rn.f32x2 %0, %1, %2;"
+      : "=l"(d)
+      : "l"(*reinterpret_cast<unsigned long long*>(&a)), "l"(*reinterpret_cast<unsigned long long*>(&b)));
+  return *reinterpret_cast<float2*>(&d);
+}
+
 // Codes for the 8 halves of one 16-byte chunk, as 32-bit words whose low bits hold
-// the two's-complement code. Returns nothing; writes u[8].
+// the two's-complement code (the low byte is the int8 code; the low nibble the INT4
+// code). Candidates and residuals are computed on fp32 pairs; a chunk whose largest
+// residual reaches the margin (or every chunk of a row with a subnormal scale) takes
+// the exact comparison path for all its elements.
 template <int BITS>
 __device__ __forceinline__ void chunk_codes(const uint4 v, float sf, float r, bool exact_all, uint32_t (&u)[8]) {
-  const uint32_t words[4] = {v.x, v.y, v.z, v.w};
-  float w[8];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const __half2 h = *reinterpret_cast<const __half2*>(&words[i]);
-    const float2 f = __half22float2(h);
-    w[2 * i] = f.x;
-    w[2 * i + 1] = f.y;
-  }
   constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
   constexpr float kMargin = 0.5f - 0x1p-15f;
-  float kf[8];
-  bool near = exact_all;
+  const uint32_t words[4] = {v.x, v.y, v.z, v.w};
+  const float2 r2 = make_float2(r, r), nr2 = make_float2(-r, -r), m2 = make_float2(kMagic, kMagic);
+  float2 w[4], k[4];
+  float emax = 0.0f;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const float t = fmaf(w[i], r, kMagic);
-    kf[i] = t - kMagic;
-    const float e = fmaf(w[i], r, -kf[i]);
-    near |= fabsf(e) >= kMargin;
-    u[i] = __float_as_uint(t);
+  for (int i = 0; i < 4; ++i) {
+    w[i] = __half22float2(*reinterpret_cast<const __half2*>(&words[i]));
+    const float2 t = fma2_rn(w[i], r2, m2);          // RNE(w * r) in the low mantissa bits
+    k[i] = sub2_rn(t, m2);                           // that integer, as a float
+    const float2 e = fma2_rn(w[i], nr2, k[i]);       // k - w * r, exact
+    emax = fmaxf(emax, fmaxf(fabsf(e.x), fabsf(e.y)));
+    u[2 * i] = __float_as_uint(t.x);
+    u[2 * i + 1] = __float_as_uint(t.y);
   }
-  if (near) {
+  if (exact_all || emax >= kMargin) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) u[i] = static_cast<uint32_t>(exact_code<BITS>(w[i], sf, kf[i]));
+    for (int i = 0; i < 4; ++i) {
+      u[2 * i] = static_cast<uint32_t>(exact_code<BITS>(w[i].x, sf, k[i].x));
+      u[2 * i + 1] = static_cast<uint32_t>(exact_code<BITS>(w[i].y, sf, k[i].y));
+    }
   }
+}
+
+// Bytes [u0.b0, u1.b0, u2.b0, u3.b0]: the low bytes of four code words.
+__device__ __forceinline__ uint32_t low_bytes4(uint32_t u0, uint32_t u1, uint32_t u2, uint32_t u3) {
+  return prmt(prmt(u0, u1, 0x0040u), prmt(u2, u3, 0x0040u), 0x5410u);
+}
+
+// INT4: 8 code words -> one packed word, nibble j = code j & 0xF (low nibble = even k).
+__device__ __forceinline__ uint32_t pack_int4_word(const uint32_t (&u)[8]) {
+  const uint32_t b0 = low_bytes4(u[0], u[1], u[2], u[3]);       // code bytes k0..k3
+  const uint32_t b1 = low_bytes4(u[4], u[5], u[6], u[7]);
+  // byte 2i of y: (k_{2i} & 0xF) | (k_{2i+1} & 0xF) << 4  (odd bytes unused)
+  const uint32_t y0 = lop3_sel(b0, b0 >> 4, 0x0F0F0F0Fu);
+  const uint32_t y1 = lop3_sel(b1, b1 >> 4, 0x0F0F0F0Fu);
+  return prmt(y0, y1, 0x6420u);
 }
 
 // One CTA of T threads per row; each thread holds CPT 16-byte chunks of the row.
@@ -109,10 +144,8 @@ __global__ void __launch_bounds__(T) quantize_kernel(const __half* __restrict__ 
     const int c = threadIdx.x + i * T;
     if (c < nchunks) {
       v[i] = ld_stream_v4(src + c);
-      m = __vmaxu2(m, v[i].x & 0x7fff7fffu);
-      m = __vmaxu2(m, v[i].y & 0x7fff7fffu);
-      m = __vmaxu2(m, v[i].z & 0x7fff7fffu);
-      m = __vmaxu2(m, v[i].w & 0x7fff7fffu);
+      m = __vimax3_u16x2(m, v[i].x & 0x7fff7fffu, v[i].y & 0x7fff7fffu);
+      m = __vimax3_u16x2(m, v[i].z & 0x7fff7fffu, v[i].w & 0x7fff7fffu);
     } else {
       v[i] = make_uint4(0, 0, 0, 0);
     }
@@ -150,14 +183,9 @@ __global__ void __launch_bounds__(T) quantize_kernel(const __half* __restrict__ 
       chunk_codes<BITS>(v[i], sf, r, exact_all, u);
     }
     if constexpr (BITS == 4) {
-      uint32_t word = 0;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) word |= (u[j] & 0xFu) << (4 * j);
-      reinterpret_cast<uint32_t*>(packed + row * static_cast<long long>(K / 2))[c] = word;
+      reinterpret_cast<uint32_t*>(packed + row * static_cast<long long>(K / 2))[c] = pack_int4_word(u);
     } else {
-      uint2 out;
-      out.x = (u[0] & 0xFFu) | ((u[1] & 0xFFu) << 8) | ((u[2] & 0xFFu) << 16) | ((u[3] & 0xFFu) << 24);
-      out.y = (u[4] & 0xFFu) | ((u[5] & 0xFFu) << 8) | ((u[6] & 0xFFu) << 16) | ((u[7] & 0xFFu) << 24);
+      const uint2 out = make_uint2(low_bytes4(u[0], u[1], u[2], u[3]), low_bytes4(u[4], u[5], u[6], u[7]));
       reinterpret_cast<uint2*>(packed + row * static_cast<long long>(K))[c] = out;
     }
   }

@@ -47,6 +47,13 @@ constexpr int kSkinnyProducerWarp = 20;
 constexpr int kSkinnyMmaWarp = 21;
 constexpr int kSkinnyThreads = 22 * 32;
 constexpr int kSkinnyASlots = 8;           // A operand slots in TMEM (one 64-wide K block each)
+static_assert((kSkinnyASlots & (kSkinnyASlots - 1)) == 0, "slot index by mask");
+#ifndef SKINNY_ACC_CHAINS
+#define SKINNY_ACC_CHAINS 1
+#endif
+// Independent accumulators per tile (consecutive MMAs of a K block alternate between
+// them and the epilogue sums them). One by default: two measured no faster here.
+constexpr int kSkinnyAccChains = SKINNY_ACC_CHAINS;
 
 template <int BITS, int BN, int ZP = 0>
 struct SkinnyCfg {
@@ -63,7 +70,7 @@ struct SkinnyCfg {
   static constexpr int STAGE_BYTES = W_BYTES + KB * XT_BYTES;
   static constexpr int kStages = (kPrefillSmemBudget / STAGE_BYTES) < kPrefillMaxStages
                                      ? (kPrefillSmemBudget / STAGE_BYTES) : kPrefillMaxStages;
-  static constexpr int ACC_COLS = 2 * BN;                 // two accumulators of BN fp32 columns
+  static constexpr int ACC_COLS = 2 * kSkinnyAccChains * BN;   // 2 tiles x chains x BN fp32 columns
   static constexpr int TMEM_COLS = 512;
   static constexpr int SMEM_BYTES = kStages * STAGE_BYTES + 1024 /*align*/ + 512 /*barriers*/;
   static_assert(BN == 16 || BN == 32 || BN == 64, "skinny token tiles");
@@ -81,6 +88,20 @@ __device__ __forceinline__ void umma_f16_tmem_a(uint32_t d_tmem, uint32_t a_tmem
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
       "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// The same MMA with the B descriptor given as its two 32-bit halves (the issuing loop
+// offsets the low half, which holds the start address, with plain 32-bit adds).
+template <uint32_t kAccumulate>
+__device__ __forceinline__ void umma_f16_tmem_a_lh(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo, uint32_t b_hi,
+                                                   uint32_t idesc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b64 bd;\n\t"
+      "setp.ne.b32 p, %5, 0;\n\t"
+      "mov.b64 bd, {%2, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], bd, %4, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "r"(b_lo), "r"(b_hi), "r"(idesc), "r"(kAccumulate)
       : "memory");
 }
 
@@ -279,12 +300,19 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
     if (!ok && lane == 0) report_error(kErrPrefillWait);
   } else if (warp == kSkinnyMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
+    // A single thread issues every MMA, so its instruction stream is kept short: the B
+    // descriptors of a stage come from one base by 32-bit adds to the low half (start
+    // address in 16-byte units) and the accumulate flag is a compile-time constant per
+    // K block. Its waits suspend in hardware like the other roles' (polling took issue
+    // slots from the dequantizer warps sharing its scheduler and was slower).
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
       int kseq = 0;
       int it = 0;
       uint32_t acc_armed[2] = {};
+      const uint64_t desc0 = umma_desc_sw128(0);
+      const uint32_t desc_hi = static_cast<uint32_t>(desc0 >> 32);
       for (int u = blockIdx.x; u < a.units && ok; u += G, ++it) {
         const int p = u / a.tiles;
         const int st0 = p * a.kbp;
@@ -293,23 +321,32 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
         const uint32_t aphase = (it >> 1) & 1;
         if (!mbar_wait_suspend(&accempty[ab], aphase ^ 1)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + ab * C::kBN;
+        const uint32_t d_tmem = tmem_base + ab * kSkinnyAccChains * C::kBN;
         bool first = true;
         for (int ks = st0; ks < st1 && ok; ++ks) {
           const int nkb = skinny_stage_kblocks(ks * C::SK, K, C::KB);
-          uint8_t* st = smem + stage * C::STAGE_BYTES;
+          // low descriptor half of the stage's first activation tile (start address >> 4)
+          const uint32_t b_lo0 = static_cast<uint32_t>(desc0) |
+                                 ((smem_u32(smem + stage * C::STAGE_BYTES + C::W_BYTES) >> 4) & 0x3FFFu);
           for (int j = 0; j < nkb; ++j, ++kseq) {
-            const int slot = kseq % NA;
+            const int slot = kseq & (NA - 1);
             if (!mbar_wait_suspend(&afull[slot], (kseq / NA) & 1)) { ok = false; break; }
             tc_fence_after();
-            const uint32_t x_addr = smem_u32(st + C::W_BYTES + j * C::XT_BYTES);
+            const uint32_t b_lo = b_lo0 + static_cast<uint32_t>(j * (C::XT_BYTES >> 4));
             const uint32_t a_tmem = tmem_base + C::ACC_COLS + slot * 32;
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              umma_f16_tmem_a(d_tmem, a_tmem + kk * 8, umma_desc_sw128(x_addr + kk * 32), C::IDESC,
-                              first ? 0u : 1u);
+            // k sub-block kk: A columns kk * 8, B start address + kk * 32 bytes
+            if (first) {
+              umma_f16_tmem_a_lh<0>(d_tmem, a_tmem, b_lo, desc_hi, C::IDESC);
+              umma_f16_tmem_a_lh<(kSkinnyAccChains > 1) ? 0 : 1>(d_tmem + (1 % kSkinnyAccChains) * C::kBN,
+                                                                    a_tmem + 8, b_lo + 2, desc_hi, C::IDESC);
               first = false;
+            } else {
+              umma_f16_tmem_a_lh<1>(d_tmem, a_tmem, b_lo, desc_hi, C::IDESC);
+              umma_f16_tmem_a_lh<1>(d_tmem + (1 % kSkinnyAccChains) * C::kBN, a_tmem + 8, b_lo + 2, desc_hi,
+                                    C::IDESC);
             }
+            umma_f16_tmem_a_lh<1>(d_tmem + (2 % kSkinnyAccChains) * C::kBN, a_tmem + 16, b_lo + 4, desc_hi, C::IDESC);
+            umma_f16_tmem_a_lh<1>(d_tmem + (3 % kSkinnyAccChains) * C::kBN, a_tmem + 24, b_lo + 6, desc_hi, C::IDESC);
             umma_commit(&aempty[slot]);
           }
           if (!ok) break;
@@ -345,7 +382,7 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
       const int mt = t - nt * a.tiles_m;
       const int n = nt * C::BM + quarter * 32 + lane;
       const float s = (n < a.N) ? __half2float(a.scale[n]) : 0.0f;
-      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + ab * C::kBN;
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + ab * kSkinnyAccChains * C::kBN;
       constexpr int kChunk = (C::kBN < 32) ? C::kBN : 32;
 #pragma unroll 1
       for (int cb = 0; cb < C::kBN / kChunk; ++cb) {
@@ -354,6 +391,14 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
         uint32_t v[32];
         if constexpr (kChunk == 16) tmem_ld16(t_row + cb * kChunk, v);
         else tmem_ld32(t_row + cb * kChunk, v);
+#pragma unroll
+        for (int h = 1; h < kSkinnyAccChains; ++h) {
+          uint32_t w[32];
+          if constexpr (kChunk == 16) tmem_ld16(t_row + h * C::kBN + cb * kChunk, w);
+          else tmem_ld32(t_row + h * C::kBN + cb * kChunk, w);
+#pragma unroll
+          for (int jj = 0; jj < kChunk; ++jj) v[jj] = __float_as_uint(__uint_as_float(v[jj]) + __uint_as_float(w[jj]));
+        }
         const int mend = min(kChunk, a.M - m0);
         if (split) {
           if (n < a.N) {

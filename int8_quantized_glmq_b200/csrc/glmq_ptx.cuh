@@ -66,6 +66,14 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
       : "memory");
 }
 
+// Arrival that counts as `count` arrivals.
+__device__ __forceinline__ void mbar_arrive_cnt(uint64_t* bar, uint32_t count) {
+  asm volatile(
+      "{\n\t.reg .b64 st;\n\t"
+      "mbarrier.arrive.release.cta.shared::cta.b64 st, [%0], %1;\n\t}" ::"r"(smem_u32(bar)), "r"(count)
+      : "memory");
+}
+
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
   asm volatile(
       "{\n\t.reg .b64 st;\n\t"
@@ -171,10 +179,18 @@ __device__ __forceinline__ bool mbar_wait_warp_suspend(uint64_t* bar, uint32_t p
   return __all_sync(0xffffffffu, mbar_wait_suspend(bar, parity));
 }
 
+__device__ __forceinline__ bool mbar_wait_drain_warp_suspend(uint64_t* bar, uint32_t parity) {
+  return __all_sync(0xffffffffu, mbar_wait_drain_suspend(bar, parity));
+}
+
 // Warp-uniform wait: every lane waits, and the warp agrees on the outcome, so the
 // result can gate warp-collective instructions (mma.sync, tcgen05.ld, __syncwarp).
 __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity) {
   return __all_sync(0xffffffffu, mbar_wait(bar, parity));
+}
+
+__device__ __forceinline__ bool mbar_wait_drain_warp(uint64_t* bar, uint32_t parity) {
+  return __all_sync(0xffffffffu, mbar_wait_drain(bar, parity));
 }
 
 // ---------------------------------------------------------------- programmatic dependent launch

@@ -127,8 +127,12 @@ __device__ __forceinline__ uint32_t pack_int4_word(const uint32_t (&u)[8]) {
 // One CTA of T threads per row; each thread holds CPT 16-byte chunks of the row.
 // geglu_half = F > 0 writes the GeGLU row layout (output row 16g + r from input row
 // 8g + r, r < 8, or F + 8g + r - 8); 0 keeps the natural order.
+// At least 40 warps resident per SM (registers capped to fit): a row's loads are issued
+// all at once and then waited for, so occupancy is what hides the memory latency.
+constexpr int quantize_min_blocks(int T) { return T <= 256 ? 5 : (T <= 512 ? 2 : 1); }
+
 template <int BITS, int CPT, int T>
-__global__ void __launch_bounds__(T) quantize_kernel(const __half* __restrict__ W, int K,
+__global__ void __launch_bounds__(T, quantize_min_blocks(T)) quantize_kernel(const __half* __restrict__ W, int K,
                                                      uint8_t* __restrict__ packed, __half* __restrict__ scale,
                                                      int geglu_half) {
   constexpr int D = (1 << (BITS - 1)) - 1;

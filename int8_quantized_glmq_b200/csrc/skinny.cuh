@@ -8,23 +8,29 @@
 //
 // With few tokens the packed weights are the working set, so the kernel is built
 // around a wide weight stream and cheap dequantization:
-//  * Stages hold one TMA box of 128 weight rows x 128 packed bytes (256 k for INT4,
-//    128 k for INT8; 128-byte swizzle) plus the matching activation tiles
-//    (BN tokens x 64 k each). Wide box rows matter: the TMA path serves a roughly
-//    fixed number of box rows per microsecond, so 128-byte rows stream several
-//    times faster than the 32-byte rows of a 64-wide K block, and the activation
-//    tiles do not take box rows at all: a small pre-pass (skinny_pack_x_kernel)
-//    writes X once per call as the exact shared-memory image of every tile (128-byte
-//    swizzle, INT4 k order, zero rows past M), and each stage fetches its tiles with
-//    one contiguous bulk copy.
+//  * Two rings. The weight ring holds TMA boxes of 128 weight rows x 128 packed
+//    bytes (256 k for INT4, 128 k for INT8; 128-byte swizzle). Wide box rows
+//    matter: the TMA path serves a roughly fixed number of box rows per
+//    microsecond, so 128-byte rows stream several times faster than the 32-byte
+//    rows of a 64-wide K block. The activation ring holds the matching activation
+//    tiles (BN tokens x 64 k each), which take no box rows: a small pre-pass
+//    (skinny_pack_x_kernel) writes X once per call as the exact shared-memory image
+//    of every tile (128-byte swizzle, INT4 k order, zero rows past M), and a second
+//    producer warp fetches a stage's tiles with one contiguous bulk copy.
+//  * A weight box is released as soon as the dequantizers hold its codes in
+//    registers; only the activation tiles wait for the MMAs. The weight ring's
+//    round trip is therefore about one TMA latency, and with most of shared memory
+//    given to it (8 to 13 boxes) enough bytes stay in flight to stream at HBM rate.
 //  * The dequantized weights never touch shared memory: they are the MMA's A
 //    operand in tensor memory. Four dequantizer groups of 128 threads (thread =
 //    weight row = TMEM lane) take the 64-wide K blocks of the stream round-robin
 //    (group g: blocks g, g+4, ...), turn 64 codes into fp16 in registers and write
-//    them with one tcgen05.st into a ring of A slots.
-//  * One thread issues tcgen05.mma (kind::f16, A from TMEM, B from shared memory,
-//    fp32 accumulator in TMEM); the epilogue warps read the accumulator with
-//    tcgen05.ld, multiply by s[n] and store fp16 (or add into the split-K scratch).
+//    them with one tcgen05.st into a ring of A slots. The four slots of one slot
+//    group are filled together and handed to the MMA warp with one barrier.
+//  * One warp runs the MMA loop and its elected lane issues tcgen05.mma (kind::f16,
+//    A from TMEM, B from shared memory, fp32 accumulator in TMEM); the epilogue
+//    warps read the accumulator with tcgen05.ld, multiply by s[n] and store fp16
+//    (or add into the split-K scratch).
 //  * INT4 codes are dequantized in the order (0,4,1,5,2,6,3,7) within each group
 //    of 8, which costs no byte shuffle; the pre-pass writes the activations in the
 //    same order (the MMA's k order is immaterial when both operands share it).
@@ -43,17 +49,18 @@ namespace glmq {
 constexpr int kSkinnyDequantWarps = 16;    // 4 groups of 4 warps
 constexpr int kSkinnyGroups = 4;
 constexpr int kSkinnyEpilogueWarp0 = 16;   // warps 16..19
-constexpr int kSkinnyProducerWarp = 20;
+constexpr int kSkinnyProducerWarp = 20;    // weight boxes
 constexpr int kSkinnyMmaWarp = 21;
-constexpr int kSkinnyThreads = 22 * 32;
-constexpr int kSkinnyASlots = 8;           // A operand slots in TMEM (one 64-wide K block each)
-static_assert((kSkinnyASlots & (kSkinnyASlots - 1)) == 0, "slot index by mask");
-#ifndef SKINNY_ACC_CHAINS
-#define SKINNY_ACC_CHAINS 1
-#endif
-// Independent accumulators per tile (consecutive MMAs of a K block alternate between
-// them and the epilogue sums them). One by default: two measured no faster here.
-constexpr int kSkinnyAccChains = SKINNY_ACC_CHAINS;
+constexpr int kSkinnyXWarp = 22;           // activation tiles
+constexpr int kSkinnyThreads = 23 * 32;
+constexpr int kSkinnyMaxWStages = 16;
+// A operand slots in TMEM, one 64-wide K block (32 columns) each, in groups of 4: the
+// dequantizer groups fill one slot group (4 consecutive K blocks of a work unit)
+// together, and the MMA warp consumes it with one wait, 16 back-to-back MMAs and one
+// commit. Three slot groups (384 columns) fit beside two accumulators of up to 64
+// columns.
+constexpr int kSkinnySlotGroups = 3;
+constexpr int kSkinnyGroupBlocks = 4;
 
 template <int BITS, int BN, int ZP = 0>
 struct SkinnyCfg {
@@ -67,16 +74,20 @@ struct SkinnyCfg {
   static constexpr int KB = SK / 64;                      // 64-wide K blocks per stage (4 or 2)
   static constexpr int W_BYTES = BM * WB;                 // 16 KB
   static constexpr int XT_BYTES = BN * 128;               // one activation tile (BN x 64 fp16)
-  static constexpr int STAGE_BYTES = W_BYTES + KB * XT_BYTES;
-  static constexpr int kStages = (kPrefillSmemBudget / STAGE_BYTES) < kPrefillMaxStages
-                                     ? (kPrefillSmemBudget / STAGE_BYTES) : kPrefillMaxStages;
-  static constexpr int ACC_COLS = 2 * kSkinnyAccChains * BN;   // 2 tiles x chains x BN fp32 columns
+  static constexpr int XS_BYTES = KB * XT_BYTES;          // one stage's activation tiles
+  // Two rings: activation stages (about 64 KB, at least 3) and weight boxes in the rest.
+  static constexpr int kXStages = (65536 / XS_BYTES) < 3 ? 3 : ((65536 / XS_BYTES) > 12 ? 12 : 65536 / XS_BYTES);
+  static constexpr int kWStagesFit = (kPrefillSmemBudget - kXStages * XS_BYTES) / W_BYTES;
+  static constexpr int kWStages = kWStagesFit < kSkinnyMaxWStages ? kWStagesFit : kSkinnyMaxWStages;
+  static constexpr int ACC_COLS = 2 * BN;                      // 2 tiles x BN fp32 columns
   static constexpr int TMEM_COLS = 512;
-  static constexpr int SMEM_BYTES = kStages * STAGE_BYTES + 1024 /*align*/ + 512 /*barriers*/;
+  static constexpr int SMEM_BYTES = kWStages * W_BYTES + kXStages * XS_BYTES + 1024 /*align*/ + 512 /*barriers*/;
+  static_assert(kWStages >= 4, "weight pipeline depth");
+  static_assert(2 * kWStages + 2 * kXStages + 2 * kSkinnySlotGroups + 5 < 512 / 8, "barrier area");
   static_assert(BN == 16 || BN == 32 || BN == 64, "skinny token tiles");
   static_assert(XT_BYTES % 1024 == 0, "swizzle atoms stay 1024-byte aligned");
-  static_assert(kStages >= 3, "pipeline depth");
-  static_assert(ACC_COLS + kSkinnyASlots * 32 <= TMEM_COLS, "tensor memory budget");
+  static_assert(ACC_COLS + kSkinnySlotGroups * kSkinnyGroupBlocks * 32 <= TMEM_COLS, "tensor memory budget");
+  static_assert(KB == 2 || KB == 4, "a slot group spans one INT4 stage or two INT8 stages");
   // kind::f16, fp32 accumulator, fp16 A (tensor memory) and B (shared memory), K-major, N = BN, M = 128
   static constexpr uint32_t IDESC = (1u << 4) | (uint32_t(BN >> 3) << 17) | (uint32_t(BM >> 4) << 24);
 };
@@ -93,16 +104,29 @@ __device__ __forceinline__ void umma_f16_tmem_a(uint32_t d_tmem, uint32_t a_tmem
 
 // The same MMA with the B descriptor given as its two 32-bit halves (the issuing loop
 // offsets the low half, which holds the start address, with plain 32-bit adds).
+// Issued by the elected lane only (leader != 0 in exactly one lane of the issuing warp).
 template <uint32_t kAccumulate>
 __device__ __forceinline__ void umma_f16_tmem_a_lh(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo, uint32_t b_hi,
-                                                   uint32_t idesc) {
+                                                   uint32_t idesc, uint32_t leader) {
   asm volatile(
-      "{\n\t.reg .pred p;\n\t.reg .b64 bd;\n\t"
+      "{\n\t.reg .pred p, e;\n\t.reg .b64 bd;\n\t"
       "setp.ne.b32 p, %5, 0;\n\t"
+      "setp.ne.b32 e, %6, 0;\n\t"
       "mov.b64 bd, {%2, %3};\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], bd, %4, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "r"(b_lo), "r"(b_hi), "r"(idesc), "r"(kAccumulate)
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], bd, %4, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "r"(b_lo), "r"(b_hi), "r"(idesc), "n"(kAccumulate), "r"(leader)
       : "memory");
+}
+
+// One 64-wide K block: 4 MMAs (K = 16 each). Sub-block kk reads A columns kk * 8 of
+// the slot and B from the tile's start address + kk * 32 bytes (+2 in the low
+// descriptor half). kFirst: the block opens the accumulator (no accumulate).
+template <bool kFirst, class C>
+__device__ __forceinline__ void skinny_mma_block(uint32_t d, uint32_t a, uint32_t b_lo, uint32_t b_hi, uint32_t leader) {
+  umma_f16_tmem_a_lh<kFirst ? 0u : 1u>(d, a, b_lo, b_hi, C::IDESC, leader);
+  umma_f16_tmem_a_lh<1>(d, a + 8, b_lo + 2, b_hi, C::IDESC, leader);
+  umma_f16_tmem_a_lh<1>(d, a + 16, b_lo + 4, b_hi, C::IDESC, leader);
+  umma_f16_tmem_a_lh<1>(d, a + 24, b_lo + 6, b_hi, C::IDESC, leader);
 }
 
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32]) {
@@ -151,17 +175,22 @@ __device__ __forceinline__ int skinny_stage_kblocks(int k0, int K, int KB) { ret
 template <class C>
 __global__ void __launch_bounds__(kSkinnyThreads, 1)
     skinny_kernel(const __grid_constant__ CUtensorMap tmap_w, const PrefillArgs a) {
-  constexpr int S = C::kStages;
-  constexpr int NA = kSkinnyASlots;
+  constexpr int SW = C::kWStages;
+  constexpr int SX = C::kXStages;
+  constexpr int NG = kSkinnySlotGroups;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::STAGE_BYTES);
-  uint64_t* full = bars;                  // stage bytes landed            (count 1 + tx)
-  uint64_t* empty = bars + S;             // stage's MMAs done             (tcgen05.commit)
-  uint64_t* afull = bars + 2 * S;         // A slot written                (count 4 warps)
-  uint64_t* aempty = afull + NA;          // A slot's MMAs done            (tcgen05.commit)
-  uint64_t* accfull = aempty + NA;        // accumulator ready             (tcgen05.commit), x2
-  uint64_t* accempty = accfull + 2;       // accumulator drained           (count 4 warps), x2
+  uint8_t* wring = smem;                                  // SW weight boxes
+  uint8_t* xring = smem + SW * C::W_BYTES;                // SX stages of activation tiles
+  uint64_t* bars = reinterpret_cast<uint64_t*>(xring + SX * C::XS_BYTES);
+  uint64_t* wfull = bars;                 // weight box landed                  (count 1 + tx)
+  uint64_t* wempty = wfull + SW;          // weight box read into registers     (count 4 * KB warps)
+  uint64_t* xfull = wempty + SW;          // activation tiles landed            (count 1 + tx)
+  uint64_t* xempty = xfull + SX;          // activation tiles' MMAs done        (tcgen05.commit)
+  uint64_t* afull = xempty + SX;          // slot group written                 (count 16 warps)
+  uint64_t* aempty = afull + NG;          // slot group's MMAs done             (tcgen05.commit)
+  uint64_t* accfull = aempty + NG;        // accumulator ready                  (tcgen05.commit), x2
+  uint64_t* accempty = accfull + 2;       // accumulator drained                (count 4 warps), x2
   uint64_t* final_bar = accempty + 2;     // all MMAs done, on the failure path (tcgen05.commit)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(final_bar + 1);
 
@@ -172,12 +201,16 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
   const int G = gridDim.x;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < S; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
+    for (int s = 0; s < SW; ++s) {
+      mbar_init(&wfull[s], 1);
+      mbar_init(&wempty[s], kSkinnyDequantWarps / kSkinnyGroups * C::KB);
     }
-    for (int i = 0; i < NA; ++i) {
-      mbar_init(&afull[i], kSkinnyDequantWarps / kSkinnyGroups);
+    for (int s = 0; s < SX; ++s) {
+      mbar_init(&xfull[s], 1);
+      mbar_init(&xempty[s], 1);
+    }
+    for (int i = 0; i < NG; ++i) {
+      mbar_init(&afull[i], kSkinnyDequantWarps);
       mbar_init(&aempty[i], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -200,173 +233,240 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
   bool ok = true;
 
   if (warp == kSkinnyProducerWarp) {
-    // ------------------------------------------------------------ TMA producer
+    // ------------------------------------------------------------ weight boxes (TMA)
     if (lane == 0) {
-      uint32_t armed[S] = {};
-      int stage = 0;
-      uint32_t phase = 0;
+      uint32_t armed[SW] = {};
+      int r = 0;
+      uint32_t ph = 0;
       for (int u = blockIdx.x; u < a.units && ok; u += G) {
         const int p = u / a.tiles;
-        const int t = u - p * a.tiles;
-        const int nt = t / a.tiles_m;
-        const int mt = t - nt * a.tiles_m;
+        const int nt = (u - p * a.tiles) / a.tiles_m;
         const int st1 = min(num_st, (p + 1) * a.kbp);
         for (int ks = p * a.kbp; ks < st1; ++ks) {
-          if (!mbar_wait_suspend(&empty[stage], phase ^ 1)) { ok = false; break; }
-          const int k0 = ks * C::SK;
-          const int nkb = skinny_stage_kblocks(k0, K, C::KB);
-          uint8_t* st = smem + stage * C::STAGE_BYTES;
-          mbar_arrive_expect_tx(&full[stage], C::W_BYTES + nkb * C::XT_BYTES);
-          armed[stage] = phase + 1;
-          tma_load_2d(st, &tmap_w, k0 / C::KPB, nt * C::BM, &full[stage]);
-          bulk_g2s(st + C::W_BYTES, a.xs + (static_cast<long long>(mt) * (K / 64) + k0 / 64) * C::XT_BYTES,
-                   static_cast<uint32_t>(nkb * C::XT_BYTES), &full[stage]);
-          if (++stage == S) { stage = 0; phase ^= 1; }
+          if (!mbar_wait_suspend(&wempty[r], ph ^ 1)) { ok = false; break; }
+          mbar_arrive_expect_tx(&wfull[r], C::W_BYTES);
+          armed[r] = ph + 1;
+          tma_load_2d(wring + r * C::W_BYTES, &tmap_w, ks * C::WB, nt * C::BM, &wfull[r]);
+          if (++r == SW) { r = 0; ph ^= 1; }
         }
       }
       bool drained = true;
-      for (int s = 0; s < S; ++s)
-        if (armed[s] && !mbar_wait_drain_suspend(&full[s], armed[s] - 1)) drained = false;
+      for (int s = 0; s < SW; ++s)
+        if (armed[s] && !mbar_wait_drain_suspend(&wfull[s], armed[s] - 1)) drained = false;
+      if (!ok || !drained) report_error(kErrPrefillWait);
+    }
+  } else if (warp == kSkinnyXWarp) {
+    // ------------------------------------------------------------ activation tiles (bulk copies)
+    if (lane == 0) {
+      uint32_t armed[SX] = {};
+      int r = 0;
+      uint32_t ph = 0;
+      for (int u = blockIdx.x; u < a.units && ok; u += G) {
+        const int p = u / a.tiles;
+        const int mt = (u - p * a.tiles) % a.tiles_m;
+        const int st1 = min(num_st, (p + 1) * a.kbp);
+        for (int ks = p * a.kbp; ks < st1; ++ks) {
+          const int k0 = ks * C::SK;
+          const int nkb = skinny_stage_kblocks(k0, K, C::KB);
+          if (!mbar_wait_suspend(&xempty[r], ph ^ 1)) { ok = false; break; }
+          mbar_arrive_expect_tx(&xfull[r], nkb * C::XT_BYTES);
+          armed[r] = ph + 1;
+          bulk_g2s(xring + r * C::XS_BYTES, a.xs + (static_cast<long long>(mt) * (K / 64) + k0 / 64) * C::XT_BYTES,
+                   static_cast<uint32_t>(nkb * C::XT_BYTES), &xfull[r]);
+          if (++r == SX) { r = 0; ph ^= 1; }
+        }
+      }
+      bool drained = true;
+      for (int s = 0; s < SX; ++s)
+        if (armed[s] && !mbar_wait_drain_suspend(&xfull[s], armed[s] - 1)) drained = false;
       if (!ok || !drained) report_error(kErrPrefillWait);
     }
   } else if (warp < kSkinnyDequantWarps) {
     // ------------------------------------------------------------ dequantizer groups
-    const int grp = warp >> 2;                      // K blocks with sequence number % 4 == grp
+    // The K blocks of a work unit are numbered b = 0, 1, ...; block b sits in stage
+    // b / KB of the unit (position b % KB there) and in slot group b / 4 (slot b % 4).
+    // Group g dequantizes the blocks b with b % 4 == g. A warp releases the weight box
+    // as soon as its block's codes are in registers; the slot group is released by the
+    // MMAs that read it.
+    constexpr int kUnits = C::kBits == 4 ? 2 : 4;   // 16-byte units of a row per block
+    const int grp = warp >> 2;
     const int row = ((warp & 3) << 5) + lane;       // weight row of the tile = TMEM lane
     const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    int stage = 0;
-    uint32_t phase = 0;
-    int kseq = 0;
+    int gst = 0;   // stages of the earlier units
+    int gsg = 0;   // slot groups of the earlier units
     for (int u = blockIdx.x; u < a.units && ok; u += G) {
       const int p = u / a.tiles;
-      const int st1 = min(num_st, (p + 1) * a.kbp);
+      const int st0 = p * a.kbp;
+      const int st1 = min(num_st, st0 + a.kbp);
+      const int nb = (min(K, st1 * C::SK) - st0 * C::SK) >> 6;   // K blocks of the unit
       Int4Dequant dq = int4_dequant_symmetric();
       if constexpr (C::kZP) {
         const int wrow = ((u - p * a.tiles) / a.tiles_m) * C::BM + row;
         dq = int4_dequant_zero_point(wrow < a.N ? a.zero[wrow] : 0);
       }
-      for (int ks = p * a.kbp; ks < st1 && ok; ++ks) {
-        const int nkb = skinny_stage_kblocks(ks * C::SK, K, C::KB);
-        bool waited = false;
-        for (int j = 0; j < nkb; ++j, ++kseq) {
-          if ((kseq & (kSkinnyGroups - 1)) != grp) continue;
-          if (!waited) {
-            if (!mbar_wait_warp_suspend(&full[stage], phase)) { ok = false; break; }
-            waited = true;
-          }
-          const int slot = kseq % NA;
-          if (!mbar_wait_warp_suspend(&aempty[slot], ((kseq / NA) & 1) ^ 1)) { ok = false; break; }
-          tc_fence_after();
-          uint8_t* st = smem + stage * C::STAGE_BYTES;
-          const uint32_t w_tile = smem_u32(st);
-          uint32_t h[32];
-          if constexpr (C::kBits == 4) {
-            // bytes [32j, 32j+32) of this row: 16-byte units 2j and 2j+1, 128-byte swizzle
+      for (int b = grp; b < nb; b += kSkinnyGroups) {
+        const int j = b % C::KB;                    // block within the stage
+        const int sq = gst + b / C::KB;             // stage sequence number
+        const int r = sq % SW;
+        const int gq = gsg + (b >> 2);              // slot-group sequence number
+        const int sg = gq % NG;
+        if (!mbar_wait_warp_suspend(&wfull[r], (sq / SW) & 1)) { ok = false; break; }
+        const uint32_t w_tile = smem_u32(wring + r * C::W_BYTES);
+        uint4 raw[kUnits];
 #pragma unroll
-            for (int q = 0; q < 2; ++q) {
-              const uint32_t unit = static_cast<uint32_t>((2 * j + q) ^ (row & 7));
-              const uint4 v = lds_v4(w_tile + row * 128 + (unit << 4));
-              const uint32_t words[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-              for (int wv = 0; wv < 4; ++wv) {
-                const uint4 o = dequant_int4_paired(words[wv], dq);
-                h[16 * q + 4 * wv + 0] = o.x;
-                h[16 * q + 4 * wv + 1] = o.y;
-                h[16 * q + 4 * wv + 2] = o.z;
-                h[16 * q + 4 * wv + 3] = o.w;
-              }
-            }
-          } else {
-            // bytes [64j, 64j+64) of this row: units 4j .. 4j+3
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const uint32_t unit = static_cast<uint32_t>((4 * j + q) ^ (row & 7));
-              const uint4 v = lds_v4(w_tile + row * 128 + (unit << 4));
-              const uint2 d0 = dequant_int8_natural(v.x), d1 = dequant_int8_natural(v.y);
-              const uint2 d2 = dequant_int8_natural(v.z), d3 = dequant_int8_natural(v.w);
-              h[8 * q + 0] = d0.x; h[8 * q + 1] = d0.y; h[8 * q + 2] = d1.x; h[8 * q + 3] = d1.y;
-              h[8 * q + 4] = d2.x; h[8 * q + 5] = d2.y; h[8 * q + 6] = d3.x; h[8 * q + 7] = d3.y;
-            }
-          }
-          tmem_st32(tmem_base + lane_addr + C::ACC_COLS + slot * 32, h);
-          asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&afull[slot]);
+        for (int q = 0; q < kUnits; ++q) {
+          // 128-byte swizzle: 16-byte unit v of a row sits at v ^ (row & 7)
+          const uint32_t unit = static_cast<uint32_t>((kUnits * j + q) ^ (row & 7));
+          raw[q] = lds_v4(w_tile + row * 128 + (unit << 4));
         }
-        if (++stage == S) { stage = 0; phase ^= 1; }
+        __syncwarp();
+        if (lane == 0) {
+          // A stage with fewer than KB blocks (the K tail) counts its missing blocks'
+          // arrivals on its last block.
+          const int nkb = min(C::KB, nb - (b - j));
+          mbar_arrive_cnt(&wempty[r], j == nkb - 1 ? 1u + static_cast<uint32_t>(C::KB - nkb) : 1u);
+        }
+        if (!mbar_wait_warp_suspend(&aempty[sg], ((gq / NG) & 1) ^ 1)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t h[32];
+        if constexpr (C::kBits == 4) {
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            const uint32_t words[4] = {raw[q].x, raw[q].y, raw[q].z, raw[q].w};
+#pragma unroll
+            for (int wv = 0; wv < 4; ++wv) {
+              const uint4 o = dequant_int4_paired(words[wv], dq);
+              h[16 * q + 4 * wv + 0] = o.x;
+              h[16 * q + 4 * wv + 1] = o.y;
+              h[16 * q + 4 * wv + 2] = o.z;
+              h[16 * q + 4 * wv + 3] = o.w;
+            }
+          }
+        } else {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const uint2 d0 = dequant_int8_natural(raw[q].x), d1 = dequant_int8_natural(raw[q].y);
+            const uint2 d2 = dequant_int8_natural(raw[q].z), d3 = dequant_int8_natural(raw[q].w);
+            h[8 * q + 0] = d0.x; h[8 * q + 1] = d0.y; h[8 * q + 2] = d1.x; h[8 * q + 3] = d1.y;
+            h[8 * q + 4] = d2.x; h[8 * q + 5] = d2.y; h[8 * q + 6] = d3.x; h[8 * q + 7] = d3.y;
+          }
+        }
+        tmem_st32(tmem_base + lane_addr + C::ACC_COLS + (sg * kSkinnyGroups + grp) * 32, h);
+        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&afull[sg]);
       }
+      if (ok && (nb & 3) != 0 && grp >= (nb & 3)) {
+        // The unit's last slot group is partial and holds no block of this group: it
+        // still takes part in that group's handshake (same waits, no data).
+        const int gq = gsg + (nb >> 2);
+        const int sg = gq % NG;
+        if (!mbar_wait_warp_suspend(&aempty[sg], ((gq / NG) & 1) ^ 1)) {
+          ok = false;
+        } else if (lane == 0) {
+          mbar_arrive(&afull[sg]);
+        }
+      }
+      gst += st1 - st0;
+      gsg += (nb + 3) >> 2;
     }
     if (!ok && lane == 0) report_error(kErrPrefillWait);
   } else if (warp == kSkinnyMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
-    // A single thread issues every MMA, so its instruction stream is kept short: the B
-    // descriptors of a stage come from one base by 32-bit adds to the low half (start
-    // address in 16-byte units) and the accumulate flag is a compile-time constant per
-    // K block. Its waits suspend in hardware like the other roles' (polling took issue
-    // slots from the dequantizer warps sharing its scheduler and was slower).
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      int kseq = 0;
-      int it = 0;
-      uint32_t acc_armed[2] = {};
-      const uint64_t desc0 = umma_desc_sw128(0);
-      const uint32_t desc_hi = static_cast<uint32_t>(desc0 >> 32);
-      for (int u = blockIdx.x; u < a.units && ok; u += G, ++it) {
-        const int p = u / a.tiles;
-        const int st0 = p * a.kbp;
-        const int st1 = min(num_st, st0 + a.kbp);
-        const int ab = it & 1;
-        const uint32_t aphase = (it >> 1) & 1;
-        if (!mbar_wait_suspend(&accempty[ab], aphase ^ 1)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t d_tmem = tmem_base + ab * kSkinnyAccChains * C::kBN;
-        bool first = true;
-        for (int ks = st0; ks < st1 && ok; ++ks) {
-          const int nkb = skinny_stage_kblocks(ks * C::SK, K, C::KB);
-          // low descriptor half of the stage's first activation tile (start address >> 4)
-          const uint32_t b_lo0 = static_cast<uint32_t>(desc0) |
-                                 ((smem_u32(smem + stage * C::STAGE_BYTES + C::W_BYTES) >> 4) & 0x3FFFu);
-          for (int j = 0; j < nkb; ++j, ++kseq) {
-            const int slot = kseq & (NA - 1);
-            if (!mbar_wait_suspend(&afull[slot], (kseq / NA) & 1)) { ok = false; break; }
+    // The whole warp runs the issue loop, so the B descriptors (one base per activation
+    // stage plus 32-bit adds to the low half, which holds the start address in 16-byte
+    // units) and the TMEM addresses are warp-uniform; the elected lane issues the MMAs
+    // and commits. One wait per slot group, then its 16 MMAs back to back.
+    const uint32_t leader = elect_one_sync();
+    int gst = 0, gsg = 0, it = 0;
+    uint32_t acc_armed[2] = {};
+    const uint64_t desc0 = umma_desc_sw128(0);
+    const uint32_t desc_hi = static_cast<uint32_t>(desc0 >> 32);
+    // low descriptor half of activation stage 0's first tile (start address >> 4)
+    const uint32_t b_lo_base = static_cast<uint32_t>(desc0) | ((smem_u32(xring) >> 4) & 0x3FFFu);
+    constexpr uint32_t kStageLo = C::XS_BYTES >> 4;
+    constexpr uint32_t kTileLo = C::XT_BYTES >> 4;
+    for (int u = blockIdx.x; u < a.units && ok; u += G, ++it) {
+      const int p = u / a.tiles;
+      const int st0 = p * a.kbp;
+      const int st1 = min(num_st, st0 + a.kbp);
+      const int nb = (min(K, st1 * C::SK) - st0 * C::SK) >> 6;
+      const int ngr = (nb + 3) >> 2;
+      const int ab = it & 1;
+      const uint32_t aphase = (it >> 1) & 1;
+      if (!mbar_wait_warp_suspend(&accempty[ab], aphase ^ 1)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t d = tmem_base + ab * C::kBN;
+      for (int g = 0; g < ngr; ++g) {
+        const int gq = gsg + g;
+        const int sg = gq % NG;
+        const int b0 = 4 * g;                       // first block; it opens an activation stage
+        const int sq0 = gst + b0 / C::KB;
+        const int x0 = sq0 % SX;
+        if (!mbar_wait_warp_suspend(&afull[sg], (gq / NG) & 1)) { ok = false; break; }
+        if (!mbar_wait_warp_suspend(&xfull[x0], (sq0 / SX) & 1)) { ok = false; break; }
+        const uint32_t a_g = tmem_base + C::ACC_COLS + sg * (kSkinnyGroupBlocks * 32);
+        const uint32_t lo0 = b_lo_base + x0 * kStageLo;
+        if (b0 + 4 <= nb) {
+          // whole slot group: one INT4 stage, or two INT8 stages
+          if constexpr (C::KB == 4) {
             tc_fence_after();
-            const uint32_t b_lo = b_lo0 + static_cast<uint32_t>(j * (C::XT_BYTES >> 4));
-            const uint32_t a_tmem = tmem_base + C::ACC_COLS + slot * 32;
-            // k sub-block kk: A columns kk * 8, B start address + kk * 32 bytes
-            if (first) {
-              umma_f16_tmem_a_lh<0>(d_tmem, a_tmem, b_lo, desc_hi, C::IDESC);
-              umma_f16_tmem_a_lh<(kSkinnyAccChains > 1) ? 0 : 1>(d_tmem + (1 % kSkinnyAccChains) * C::kBN,
-                                                                    a_tmem + 8, b_lo + 2, desc_hi, C::IDESC);
-              first = false;
-            } else {
-              umma_f16_tmem_a_lh<1>(d_tmem, a_tmem, b_lo, desc_hi, C::IDESC);
-              umma_f16_tmem_a_lh<1>(d_tmem + (1 % kSkinnyAccChains) * C::kBN, a_tmem + 8, b_lo + 2, desc_hi,
-                                    C::IDESC);
+            if (g == 0) skinny_mma_block<true, C>(d, a_g, lo0, desc_hi, leader);
+            else skinny_mma_block<false, C>(d, a_g, lo0, desc_hi, leader);
+            skinny_mma_block<false, C>(d, a_g + 32, lo0 + kTileLo, desc_hi, leader);
+            skinny_mma_block<false, C>(d, a_g + 64, lo0 + 2 * kTileLo, desc_hi, leader);
+            skinny_mma_block<false, C>(d, a_g + 96, lo0 + 3 * kTileLo, desc_hi, leader);
+            umma_commit_elected(&aempty[sg], leader);
+            umma_commit_elected(&xempty[x0], leader);
+          } else {
+            const int x1 = (x0 + 1 == SX) ? 0 : x0 + 1;
+            if (!mbar_wait_warp_suspend(&xfull[x1], ((sq0 + 1) / SX) & 1)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t lo1 = b_lo_base + x1 * kStageLo;
+            if (g == 0) skinny_mma_block<true, C>(d, a_g, lo0, desc_hi, leader);
+            else skinny_mma_block<false, C>(d, a_g, lo0, desc_hi, leader);
+            skinny_mma_block<false, C>(d, a_g + 32, lo0 + kTileLo, desc_hi, leader);
+            skinny_mma_block<false, C>(d, a_g + 64, lo1, desc_hi, leader);
+            skinny_mma_block<false, C>(d, a_g + 96, lo1 + kTileLo, desc_hi, leader);
+            umma_commit_elected(&aempty[sg], leader);
+            umma_commit_elected(&xempty[x0], leader);
+            umma_commit_elected(&xempty[x1], leader);
+          }
+        } else {
+          // the unit's last, partial slot group
+          tc_fence_after();
+          for (int b = b0; b < nb; ++b) {
+            const int sq = gst + b / C::KB;
+            const int x = sq % SX;
+            if (b > b0 && b % C::KB == 0) {
+              if (!mbar_wait_warp_suspend(&xfull[x], (sq / SX) & 1)) { ok = false; break; }
+              tc_fence_after();
             }
-            umma_f16_tmem_a_lh<1>(d_tmem + (2 % kSkinnyAccChains) * C::kBN, a_tmem + 16, b_lo + 4, desc_hi, C::IDESC);
-            umma_f16_tmem_a_lh<1>(d_tmem + (3 % kSkinnyAccChains) * C::kBN, a_tmem + 24, b_lo + 6, desc_hi, C::IDESC);
-            umma_commit(&aempty[slot]);
+            const uint32_t lo = b_lo_base + x * kStageLo + (b % C::KB) * kTileLo;
+            if (b == 0) skinny_mma_block<true, C>(d, a_g + (b - b0) * 32, lo, desc_hi, leader);
+            else skinny_mma_block<false, C>(d, a_g + (b - b0) * 32, lo, desc_hi, leader);
+            if (b % C::KB == C::KB - 1 || b == nb - 1) umma_commit_elected(&xempty[x], leader);
           }
           if (!ok) break;
-          umma_commit(&empty[stage]);
-          if (++stage == S) { stage = 0; phase ^= 1; }
+          umma_commit_elected(&aempty[sg], leader);
         }
-        if (!ok) break;
-        umma_commit(&accfull[ab]);
-        acc_armed[ab] = aphase + 1;
       }
-      bool drained = true;
-      for (int b = 0; b < 2; ++b)
-        if (acc_armed[b] && !mbar_wait_drain_suspend(&accfull[b], acc_armed[b] - 1)) drained = false;
-      if (!ok) {
-        // a wait gave up mid-unit: MMAs may have been issued after the last commit above
-        umma_commit(final_bar);
-        if (!mbar_wait_drain_suspend(final_bar, 0)) drained = false;
-      }
-      if (!ok || !drained) report_error(kErrPrefillWait);
+      if (!ok) break;
+      umma_commit_elected(&accfull[ab], leader);
+      acc_armed[ab] = aphase + 1;
+      gst += st1 - st0;
+      gsg += ngr;
     }
+    bool drained = true;
+    for (int b = 0; b < 2; ++b)
+      if (acc_armed[b] && !mbar_wait_drain_warp_suspend(&accfull[b], acc_armed[b] - 1)) drained = false;
+    if (!ok) {
+      // a wait gave up mid-unit: MMAs may have been issued after the last commit above
+      umma_commit_elected(final_bar, leader);
+      if (!mbar_wait_drain_warp_suspend(final_bar, 0)) drained = false;
+    }
+    if ((!ok || !drained) && lane == 0) report_error(kErrPrefillWait);
   } else {
     // ------------------------------------------------------------ epilogue warps 16..19
     const int quarter = warp & 3;
@@ -382,7 +482,7 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
       const int mt = t - nt * a.tiles_m;
       const int n = nt * C::BM + quarter * 32 + lane;
       const float s = (n < a.N) ? __half2float(a.scale[n]) : 0.0f;
-      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + ab * kSkinnyAccChains * C::kBN;
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + ab * C::kBN;
       constexpr int kChunk = (C::kBN < 32) ? C::kBN : 32;
 #pragma unroll 1
       for (int cb = 0; cb < C::kBN / kChunk; ++cb) {
@@ -391,14 +491,6 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
         uint32_t v[32];
         if constexpr (kChunk == 16) tmem_ld16(t_row + cb * kChunk, v);
         else tmem_ld32(t_row + cb * kChunk, v);
-#pragma unroll
-        for (int h = 1; h < kSkinnyAccChains; ++h) {
-          uint32_t w[32];
-          if constexpr (kChunk == 16) tmem_ld16(t_row + h * C::kBN + cb * kChunk, w);
-          else tmem_ld32(t_row + h * C::kBN + cb * kChunk, w);
-#pragma unroll
-          for (int jj = 0; jj < kChunk; ++jj) v[jj] = __float_as_uint(__uint_as_float(v[jj]) + __uint_as_float(w[jj]));
-        }
         const int mend = min(kChunk, a.M - m0);
         if (split) {
           if (n < a.N) {

@@ -46,21 +46,18 @@
 
 namespace glmq {
 
-constexpr int kSkinnyDequantWarps = 16;    // 4 groups of 4 warps
-constexpr int kSkinnyGroups = 4;
-constexpr int kSkinnyEpilogueWarp0 = 16;   // warps 16..19
-constexpr int kSkinnyProducerWarp = 20;    // weight boxes
-constexpr int kSkinnyMmaWarp = 21;
-constexpr int kSkinnyXWarp = 22;           // activation tiles
-constexpr int kSkinnyThreads = 23 * 32;
-constexpr int kSkinnyMaxWStages = 16;
-// A operand slots in TMEM, one 64-wide K block (32 columns) each, in groups of 4: the
-// dequantizer groups fill one slot group (4 consecutive K blocks of a work unit)
-// together, and the MMA warp consumes it with one wait, 16 back-to-back MMAs and one
-// commit. Three slot groups (384 columns) fit beside two accumulators of up to 64
-// columns.
+// Slot groups of 4 K blocks (32 TMEM columns each) hold the MMA's A operand; three
+// fit beside two accumulators of up to 64 columns. Each slot group has its own crew
+// of 4 dequantizer warps (one per TMEM lane quarter).
 constexpr int kSkinnySlotGroups = 3;
 constexpr int kSkinnyGroupBlocks = 4;
+constexpr int kSkinnyDequantWarps = 4 * kSkinnySlotGroups;   // warps 0..11
+constexpr int kSkinnyEpilogueWarp0 = 12;   // warps 12..15
+constexpr int kSkinnyProducerWarp = 16;    // weight boxes
+constexpr int kSkinnyMmaWarp = 17;
+constexpr int kSkinnyXWarp = 18;           // activation tiles
+constexpr int kSkinnyThreads = 19 * 32;
+constexpr int kSkinnyMaxCrewWStages = 5;
 
 template <int BITS, int BN, int ZP = 0>
 struct SkinnyCfg {
@@ -75,14 +72,20 @@ struct SkinnyCfg {
   static constexpr int W_BYTES = BM * WB;                 // 16 KB
   static constexpr int XT_BYTES = BN * 128;               // one activation tile (BN x 64 fp16)
   static constexpr int XS_BYTES = KB * XT_BYTES;          // one stage's activation tiles
-  // Two rings: activation stages (about 64 KB, at least 3) and weight boxes in the rest.
-  static constexpr int kXStages = (65536 / XS_BYTES) < 3 ? 3 : ((65536 / XS_BYTES) > 12 ? 12 : 65536 / XS_BYTES);
-  static constexpr int kWStagesFit = (kPrefillSmemBudget - kXStages * XS_BYTES) / W_BYTES;
-  static constexpr int kWStages = kWStagesFit < kSkinnyMaxWStages ? kWStagesFit : kSkinnyMaxWStages;
+  // Weight boxes: a ring of kCrewWStages boxes per crew (each box is waited on by the one
+  // crew that reads it, so no wait can run a phase ahead of its barrier, whatever order
+  // the copies land in); activation tiles: the rest of shared memory, at least three
+  // slot groups' worth.
+  static constexpr int kMinXStages = 3 * (4 / KB);
+  static constexpr int kCrewWFit = (kPrefillSmemBudget - kMinXStages * XS_BYTES) / (kSkinnySlotGroups * W_BYTES);
+  static constexpr int kCrewWStages = kCrewWFit < kSkinnyMaxCrewWStages ? kCrewWFit : kSkinnyMaxCrewWStages;
+  static constexpr int kWStages = kSkinnySlotGroups * kCrewWStages;
+  static constexpr int kXFit = (kPrefillSmemBudget - kWStages * W_BYTES) / XS_BYTES;
+  static constexpr int kXStages = kXFit < 12 ? kXFit : 12;
   static constexpr int ACC_COLS = 2 * BN;                      // 2 tiles x BN fp32 columns
   static constexpr int TMEM_COLS = 512;
   static constexpr int SMEM_BYTES = kWStages * W_BYTES + kXStages * XS_BYTES + 1024 /*align*/ + 512 /*barriers*/;
-  static_assert(kWStages >= 4, "weight pipeline depth");
+  static_assert(kCrewWStages >= 2 && kXStages >= kMinXStages, "pipeline depth");
   static_assert(2 * kWStages + 2 * kXStages + 2 * kSkinnySlotGroups + 5 < 512 / 8, "barrier area");
   static_assert(BN == 16 || BN == 32 || BN == 64, "skinny token tiles");
   static_assert(XT_BYTES % 1024 == 0, "swizzle atoms stay 1024-byte aligned");
@@ -184,10 +187,10 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
   uint8_t* xring = smem + SW * C::W_BYTES;                // SX stages of activation tiles
   uint64_t* bars = reinterpret_cast<uint64_t*>(xring + SX * C::XS_BYTES);
   uint64_t* wfull = bars;                 // weight box landed                  (count 1 + tx)
-  uint64_t* wempty = wfull + SW;          // weight box read into registers     (count 4 * KB warps)
+  uint64_t* wempty = wfull + SW;          // weight box read into registers     (count 4 warps)
   uint64_t* xfull = wempty + SW;          // activation tiles landed            (count 1 + tx)
   uint64_t* xempty = xfull + SX;          // activation tiles' MMAs done        (tcgen05.commit)
-  uint64_t* afull = xempty + SX;          // slot group written                 (count 16 warps)
+  uint64_t* afull = xempty + SX;          // slot group written                 (count 4 warps)
   uint64_t* aempty = afull + NG;          // slot group's MMAs done             (tcgen05.commit)
   uint64_t* accfull = aempty + NG;        // accumulator ready                  (tcgen05.commit), x2
   uint64_t* accempty = accfull + 2;       // accumulator drained                (count 4 warps), x2
@@ -203,14 +206,14 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < SW; ++s) {
       mbar_init(&wfull[s], 1);
-      mbar_init(&wempty[s], kSkinnyDequantWarps / kSkinnyGroups * C::KB);
+      mbar_init(&wempty[s], 4);
     }
     for (int s = 0; s < SX; ++s) {
       mbar_init(&xfull[s], 1);
       mbar_init(&xempty[s], 1);
     }
     for (int i = 0; i < NG; ++i) {
-      mbar_init(&afull[i], kSkinnyDequantWarps);
+      mbar_init(&afull[i], 4);
       mbar_init(&aempty[i], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -234,25 +237,33 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
 
   if (warp == kSkinnyProducerWarp) {
     // ------------------------------------------------------------ weight boxes (TMA)
+    // Stage i of a unit belongs to slot group (gsg + i / (4 / KB)) and so to that
+    // group's crew; each crew's boxes cycle through its own kCrewWStages entries.
     if (lane == 0) {
+      constexpr int SC = C::kCrewWStages;
       uint32_t armed[SW] = {};
-      int r = 0;
-      uint32_t ph = 0;
+      int cnt[NG] = {};        // boxes issued to each crew so far
+      int gsg = 0;
       for (int u = blockIdx.x; u < a.units && ok; u += G) {
         const int p = u / a.tiles;
         const int nt = (u - p * a.tiles) / a.tiles_m;
-        const int st1 = min(num_st, (p + 1) * a.kbp);
-        for (int ks = p * a.kbp; ks < st1; ++ks) {
-          if (!mbar_wait_suspend(&wempty[r], ph ^ 1)) { ok = false; break; }
+        const int st0 = p * a.kbp;
+        const int st1 = min(num_st, st0 + a.kbp);
+        for (int ks = st0; ks < st1; ++ks) {
+          const int crew = (gsg + (ks - st0) / (4 / C::KB)) % NG;
+          const int n = cnt[crew]++;
+          const int r = crew * SC + n % SC;
+          const uint32_t ph = (n / SC) & 1;
+          if (!mbar_wait(&wempty[r], ph ^ 1)) { ok = false; break; }
           mbar_arrive_expect_tx(&wfull[r], C::W_BYTES);
           armed[r] = ph + 1;
           tma_load_2d(wring + r * C::W_BYTES, &tmap_w, ks * C::WB, nt * C::BM, &wfull[r]);
-          if (++r == SW) { r = 0; ph ^= 1; }
         }
+        gsg += (((min(K, st1 * C::SK) - st0 * C::SK) >> 6) + 3) >> 2;
       }
       bool drained = true;
       for (int s = 0; s < SW; ++s)
-        if (armed[s] && !mbar_wait_drain_suspend(&wfull[s], armed[s] - 1)) drained = false;
+        if (armed[s] && !mbar_wait_drain(&wfull[s], armed[s] - 1)) drained = false;
       if (!ok || !drained) report_error(kErrPrefillWait);
     }
   } else if (warp == kSkinnyXWarp) {
@@ -268,7 +279,7 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
         for (int ks = p * a.kbp; ks < st1; ++ks) {
           const int k0 = ks * C::SK;
           const int nkb = skinny_stage_kblocks(k0, K, C::KB);
-          if (!mbar_wait_suspend(&xempty[r], ph ^ 1)) { ok = false; break; }
+          if (!mbar_wait(&xempty[r], ph ^ 1)) { ok = false; break; }
           mbar_arrive_expect_tx(&xfull[r], nkb * C::XT_BYTES);
           armed[r] = ph + 1;
           bulk_g2s(xring + r * C::XS_BYTES, a.xs + (static_cast<long long>(mt) * (K / 64) + k0 / 64) * C::XT_BYTES,
@@ -278,99 +289,104 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
       }
       bool drained = true;
       for (int s = 0; s < SX; ++s)
-        if (armed[s] && !mbar_wait_drain_suspend(&xfull[s], armed[s] - 1)) drained = false;
+        if (armed[s] && !mbar_wait_drain(&xfull[s], armed[s] - 1)) drained = false;
       if (!ok || !drained) report_error(kErrPrefillWait);
     }
   } else if (warp < kSkinnyDequantWarps) {
-    // ------------------------------------------------------------ dequantizer groups
+    // ------------------------------------------------------------ dequantizer crews
     // The K blocks of a work unit are numbered b = 0, 1, ...; block b sits in stage
     // b / KB of the unit (position b % KB there) and in slot group b / 4 (slot b % 4).
-    // Group g dequantizes the blocks b with b % 4 == g. A warp releases the weight box
-    // as soon as its block's codes are in registers; the slot group is released by the
-    // MMAs that read it.
+    // Slot groups are numbered across units; slot group q uses TMEM slot group q % 3
+    // and is dequantized by crew q % 3 (warps 4c .. 4c+3, TMEM lanes 32 (w % 4) ...),
+    // which writes all of its blocks (one INT4 stage or two INT8 stages): a warp
+    // synchronises once per stage and per slot group, not once per block. A crew reads
+    // its weight boxes from its own ring, in order, and releases each box as soon as
+    // its rows' codes are in registers; the slot group is released by the MMAs.
     constexpr int kUnits = C::kBits == 4 ? 2 : 4;   // 16-byte units of a row per block
-    const int grp = warp >> 2;
+    const int crew = warp >> 2;                     // = the TMEM slot group it fills
     const int row = ((warp & 3) << 5) + lane;       // weight row of the tile = TMEM lane
     const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    int gst = 0;   // stages of the earlier units
+    const uint32_t slots = tmem_base + lane_addr + C::ACC_COLS + crew * (kSkinnyGroupBlocks * 32);
+    int wn = 0;    // boxes this crew has read (its ring position)
     int gsg = 0;   // slot groups of the earlier units
     for (int u = blockIdx.x; u < a.units && ok; u += G) {
       const int p = u / a.tiles;
       const int st0 = p * a.kbp;
       const int st1 = min(num_st, st0 + a.kbp);
       const int nb = (min(K, st1 * C::SK) - st0 * C::SK) >> 6;   // K blocks of the unit
+      const int ngr = (nb + 3) >> 2;
       Int4Dequant dq = int4_dequant_symmetric();
       if constexpr (C::kZP) {
         const int wrow = ((u - p * a.tiles) / a.tiles_m) * C::BM + row;
         dq = int4_dequant_zero_point(wrow < a.N ? a.zero[wrow] : 0);
       }
-      for (int b = grp; b < nb; b += kSkinnyGroups) {
-        const int j = b % C::KB;                    // block within the stage
-        const int sq = gst + b / C::KB;             // stage sequence number
-        const int r = sq % SW;
-        const int gq = gsg + (b >> 2);              // slot-group sequence number
-        const int sg = gq % NG;
-        if (!mbar_wait_warp_suspend(&wfull[r], (sq / SW) & 1)) { ok = false; break; }
-        const uint32_t w_tile = smem_u32(wring + r * C::W_BYTES);
-        uint4 raw[kUnits];
+      for (int g = ((crew - gsg) % NG + NG) % NG; g < ngr; g += NG) {
+        const int gq = gsg + g;                     // slot-group sequence number; gq % NG == crew
+        const int b0 = kSkinnyGroupBlocks * g;
+        const int nblk = min(kSkinnyGroupBlocks, nb - b0);
+        for (int i = 0; i < nblk; i += C::KB) {     // the group's stages
+          const int r = crew * C::kCrewWStages + wn % C::kCrewWStages;   // this crew's next box
+          const uint32_t wph = (wn / C::kCrewWStages) & 1;
+          ++wn;
+          const int nks = min(C::KB, nblk - i);     // blocks of this stage
+          if (!mbar_wait_warp(&wfull[r], wph)) { ok = false; break; }
+          const uint32_t w_row = smem_u32(wring + r * C::W_BYTES) + row * 128;
+          uint4 raw[C::KB * kUnits];                // the row's 128 bytes of the box
 #pragma unroll
-        for (int q = 0; q < kUnits; ++q) {
-          // 128-byte swizzle: 16-byte unit v of a row sits at v ^ (row & 7)
-          const uint32_t unit = static_cast<uint32_t>((kUnits * j + q) ^ (row & 7));
-          raw[q] = lds_v4(w_tile + row * 128 + (unit << 4));
-        }
-        __syncwarp();
-        if (lane == 0) {
-          // A stage with fewer than KB blocks (the K tail) counts its missing blocks'
-          // arrivals on its last block.
-          const int nkb = min(C::KB, nb - (b - j));
-          mbar_arrive_cnt(&wempty[r], j == nkb - 1 ? 1u + static_cast<uint32_t>(C::KB - nkb) : 1u);
-        }
-        if (!mbar_wait_warp_suspend(&aempty[sg], ((gq / NG) & 1) ^ 1)) { ok = false; break; }
-        tc_fence_after();
-        uint32_t h[32];
-        if constexpr (C::kBits == 4) {
+          for (int v = 0; v < C::KB * kUnits; ++v)
+            raw[v] = lds_v4(w_row + ((static_cast<uint32_t>(v) ^ static_cast<uint32_t>(row & 7)) << 4));
+          if (i == 0) {
+            if (!mbar_wait_warp(&aempty[crew], ((gq / NG) & 1) ^ 1)) { ok = false; break; }
+            tc_fence_after();
+          }
 #pragma unroll
-          for (int q = 0; q < 2; ++q) {
-            const uint32_t words[4] = {raw[q].x, raw[q].y, raw[q].z, raw[q].w};
+          for (int jj = 0; jj < C::KB; ++jj) {
+            if (jj < nks) {
+              uint32_t h[32];
+              if constexpr (C::kBits == 4) {
 #pragma unroll
-            for (int wv = 0; wv < 4; ++wv) {
-              const uint4 o = dequant_int4_paired(words[wv], dq);
-              h[16 * q + 4 * wv + 0] = o.x;
-              h[16 * q + 4 * wv + 1] = o.y;
-              h[16 * q + 4 * wv + 2] = o.z;
-              h[16 * q + 4 * wv + 3] = o.w;
+                for (int q = 0; q < 2; ++q) {
+                  const uint32_t words[4] = {raw[2 * jj + q].x, raw[2 * jj + q].y, raw[2 * jj + q].z, raw[2 * jj + q].w};
+#pragma unroll
+                  for (int wv = 0; wv < 4; ++wv) {
+                    const uint4 o = dequant_int4_paired(words[wv], dq);
+                    h[16 * q + 4 * wv + 0] = o.x;
+                    h[16 * q + 4 * wv + 1] = o.y;
+                    h[16 * q + 4 * wv + 2] = o.z;
+                    h[16 * q + 4 * wv + 3] = o.w;
+                  }
+                }
+              } else {
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                  const uint4 w4 = raw[4 * jj + q];
+                  const uint2 d0 = dequant_int8_natural(w4.x), d1 = dequant_int8_natural(w4.y);
+                  const uint2 d2 = dequant_int8_natural(w4.z), d3 = dequant_int8_natural(w4.w);
+                  h[8 * q + 0] = d0.x; h[8 * q + 1] = d0.y; h[8 * q + 2] = d1.x; h[8 * q + 3] = d1.y;
+                  h[8 * q + 4] = d2.x; h[8 * q + 5] = d2.y; h[8 * q + 6] = d3.x; h[8 * q + 7] = d3.y;
+                }
+              }
+              // tcgen05.st is asynchronous: h is reused by the next block only after this
+              // store has completed
+              tmem_st32(slots + (i + jj) * 32, h);
+              asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
             }
           }
-        } else {
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const uint2 d0 = dequant_int8_natural(raw[q].x), d1 = dequant_int8_natural(raw[q].y);
-            const uint2 d2 = dequant_int8_natural(raw[q].z), d3 = dequant_int8_natural(raw[q].w);
-            h[8 * q + 0] = d0.x; h[8 * q + 1] = d0.y; h[8 * q + 2] = d1.x; h[8 * q + 3] = d1.y;
-            h[8 * q + 4] = d2.x; h[8 * q + 5] = d2.y; h[8 * q + 6] = d3.x; h[8 * q + 7] = d3.y;
-          }
+          // The box is released only after the dequantization above has consumed every
+          // loaded register, so the loads have returned before the producer may refill it.
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&wempty[r]);
         }
-        tmem_st32(tmem_base + lane_addr + C::ACC_COLS + (sg * kSkinnyGroups + grp) * 32, h);
+        if (!ok) break;
         asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&afull[sg]);
+        if (lane == 0) mbar_arrive(&afull[crew]);
       }
-      if (ok && (nb & 3) != 0 && grp >= (nb & 3)) {
-        // The unit's last slot group is partial and holds no block of this group: it
-        // still takes part in that group's handshake (same waits, no data).
-        const int gq = gsg + (nb >> 2);
-        const int sg = gq % NG;
-        if (!mbar_wait_warp_suspend(&aempty[sg], ((gq / NG) & 1) ^ 1)) {
-          ok = false;
-        } else if (lane == 0) {
-          mbar_arrive(&afull[sg]);
-        }
-      }
-      gst += st1 - st0;
-      gsg += (nb + 3) >> 2;
+      gsg += ngr;
     }
+    // a crew that gave up may have stores in flight: none may reach TMEM after release
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
     if (!ok && lane == 0) report_error(kErrPrefillWait);
   } else if (warp == kSkinnyMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
@@ -395,7 +411,7 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
       const int ngr = (nb + 3) >> 2;
       const int ab = it & 1;
       const uint32_t aphase = (it >> 1) & 1;
-      if (!mbar_wait_warp_suspend(&accempty[ab], aphase ^ 1)) { ok = false; break; }
+      if (!mbar_wait_warp(&accempty[ab], aphase ^ 1)) { ok = false; break; }
       tc_fence_after();
       const uint32_t d = tmem_base + ab * C::kBN;
       for (int g = 0; g < ngr; ++g) {
@@ -404,8 +420,8 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
         const int b0 = 4 * g;                       // first block; it opens an activation stage
         const int sq0 = gst + b0 / C::KB;
         const int x0 = sq0 % SX;
-        if (!mbar_wait_warp_suspend(&afull[sg], (gq / NG) & 1)) { ok = false; break; }
-        if (!mbar_wait_warp_suspend(&xfull[x0], (sq0 / SX) & 1)) { ok = false; break; }
+        if (!mbar_wait_warp(&afull[sg], (gq / NG) & 1)) { ok = false; break; }
+        if (!mbar_wait_warp(&xfull[x0], (sq0 / SX) & 1)) { ok = false; break; }
         const uint32_t a_g = tmem_base + C::ACC_COLS + sg * (kSkinnyGroupBlocks * 32);
         const uint32_t lo0 = b_lo_base + x0 * kStageLo;
         if (b0 + 4 <= nb) {
@@ -421,7 +437,7 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
             umma_commit_elected(&xempty[x0], leader);
           } else {
             const int x1 = (x0 + 1 == SX) ? 0 : x0 + 1;
-            if (!mbar_wait_warp_suspend(&xfull[x1], ((sq0 + 1) / SX) & 1)) { ok = false; break; }
+            if (!mbar_wait_warp(&xfull[x1], ((sq0 + 1) / SX) & 1)) { ok = false; break; }
             tc_fence_after();
             const uint32_t lo1 = b_lo_base + x1 * kStageLo;
             if (g == 0) skinny_mma_block<true, C>(d, a_g, lo0, desc_hi, leader);
@@ -440,7 +456,7 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
             const int sq = gst + b / C::KB;
             const int x = sq % SX;
             if (b > b0 && b % C::KB == 0) {
-              if (!mbar_wait_warp_suspend(&xfull[x], (sq / SX) & 1)) { ok = false; break; }
+              if (!mbar_wait_warp(&xfull[x], (sq / SX) & 1)) { ok = false; break; }
               tc_fence_after();
             }
             const uint32_t lo = b_lo_base + x * kStageLo + (b % C::KB) * kTileLo;
@@ -460,22 +476,22 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
     }
     bool drained = true;
     for (int b = 0; b < 2; ++b)
-      if (acc_armed[b] && !mbar_wait_drain_warp_suspend(&accfull[b], acc_armed[b] - 1)) drained = false;
+      if (acc_armed[b] && !mbar_wait_drain_warp(&accfull[b], acc_armed[b] - 1)) drained = false;
     if (!ok) {
       // a wait gave up mid-unit: MMAs may have been issued after the last commit above
       umma_commit_elected(final_bar, leader);
-      if (!mbar_wait_drain_warp_suspend(final_bar, 0)) drained = false;
+      if (!mbar_wait_drain_warp(final_bar, 0)) drained = false;
     }
     if ((!ok || !drained) && lane == 0) report_error(kErrPrefillWait);
   } else {
-    // ------------------------------------------------------------ epilogue warps 16..19
+    // ------------------------------------------------------------ epilogue warps 12..15
     const int quarter = warp & 3;
     const bool split = a.parts > 1;
     int it = 0;
     for (int u = blockIdx.x; u < a.units && ok; u += G, ++it) {
       const int ab = it & 1;
       const uint32_t aphase = (it >> 1) & 1;
-      if (!mbar_wait_warp_suspend(&accfull[ab], aphase)) { ok = false; break; }
+      if (!mbar_wait_warp(&accfull[ab], aphase)) { ok = false; break; }
       tc_fence_after();
       const int t = u % a.tiles;
       const int nt = t / a.tiles_m;

@@ -209,17 +209,22 @@ def time_launches(torch, fn, iters: int, warmup: int = 2):
     return e0.elapsed_time(e1) / 1e3 / iters
 
 
-def time_launches_cold(torch, fn, iters: int, warmup: int = 2):
-    """Average device time of fn() per call with L2 flushed before each call (a
-    256 MB write between calls, outside the timed events)."""
-    flush = torch.empty((256 << 20,), dtype=torch.uint8, device="cuda")
+def time_launches_cold(torch, fn, iters: int, warmup: int = 8):
+    """Average device time of fn() per call with L2 made cold before each call: a read
+    of a 256 MB buffer between calls, outside the timed events. A read leaves clean
+    lines behind, so the timed call does not pay the write-back of a flush buffer's
+    dirty lines (a 256 MB write before each call added about 126 MB of DRAM writes to
+    the timed call). Eight warm-up calls let the SM clock settle after the work that
+    ran before."""
+    flush = torch.ones((64 << 20,), dtype=torch.int32, device="cuda")
     for _ in range(warmup):
+        flush.amax()
         fn()
     s = torch.cuda.current_stream()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(iters)]
     torch.cuda.synchronize()
     for e0, e1 in ev:
-        flush.zero_()
+        flush.amax()
         e0.record(s)
         fn()
         e1.record(s)

@@ -102,6 +102,11 @@ struct DecodeCfg {
   // activation warps: one keeps up with the small slots of M <= 2; three for M >= 4 (at
   // most 20 warps in all, so ptxas still allows 96 registers per thread)
   static constexpr int kXWarps = MP >= 4 ? 3 : 1;
+  // M <= 4: the activation warp also waits for the stage's weight box before releasing
+  // the stage, so the consumers wait on one barrier per stage instead of two (measured
+  // about 5 us faster per four-call M=1 or M=4 group; slower at M=16, where three
+  // activation warps take turns and the consumers keep both waits)
+  static constexpr bool kGateW = MP <= 4;
   static constexpr int kThreads = (kDecodeConsumerWarps + 1 + kXWarps) * 32;
   static constexpr int X_UNITS = XU * MP * 4;       // 16-byte units in a stage's activation slot
   static constexpr int X_BYTES = X_UNITS * 16;
@@ -540,6 +545,12 @@ __global__ void __launch_bounds__(C::kThreads, 1)
           stage_sums_mma<C>(slot, bring + stage * C::B_FLOATS, M, lane);
           __syncwarp();
         }
+        if constexpr (C::kGateW) {
+          // this warp also gates the weight box: once it has landed, order the TMA's
+          // writes before the generic loads of the consumers that acquire fullx
+          if (!DECODE_WAIT_X(&fullw[stage], phase)) { ok = false; break; }
+          fence_proxy_async_smem();
+        }
         if (lane == 0) mbar_arrive(&fullx[stage]);
       }
     }
@@ -581,7 +592,10 @@ __global__ void __launch_bounds__(C::kThreads, 1)
 
     const int nst = (plen + C::SK - 1) / C::SK;
     for (int ks = 0; ks < nst; ++ks) {
-      if (!DECODE_WAIT_C(&fullx[stage], phase) || !DECODE_WAIT_C(&fullw[stage], phase)) { ok = false; break; }
+      if (!DECODE_WAIT_C(&fullx[stage], phase) || (!C::kGateW && !DECODE_WAIT_C(&fullw[stage], phase))) {
+        ok = false;
+        break;
+      }
       const uint32_t box = wring_u32 + stage * kDecodeStageBytes;
       const uint32_t xseg = xring_u32 + stage * C::X_BYTES;
       const float* bias_seg = bring + stage * C::B_FLOATS;

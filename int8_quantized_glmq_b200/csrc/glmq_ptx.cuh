@@ -140,48 +140,6 @@ __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) 
   return mbar_wait_for(bar, parity, kDrainLimitNs);
 }
 
-// Same wait, but each try_wait may suspend the thread in hardware (up to 20 us per
-// try, still bounded by kWaitLimitNs overall) instead of returning at once, so a
-// waiting warp stops taking issue slots. Used by kernels whose waiting warps share
-// an SM sub-partition with a latency-critical issuer (the skinny kernel's MMA thread).
-__device__ __forceinline__ bool mbar_try_wait_suspend(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity), "r"(20000u)
-      : "memory");
-  return ok != 0;
-}
-
-__device__ __forceinline__ bool mbar_wait_suspend_for(uint64_t* bar, uint32_t parity, unsigned long long limit_ns) {
-  if (mbar_try_wait_suspend(bar, parity)) return true;
-  const unsigned long long t0 = globaltimer_ns();
-  while (true) {
-    if (mbar_try_wait_suspend(bar, parity)) return true;
-    if (globaltimer_ns() - t0 > limit_ns) return false;
-  }
-}
-
-__device__ __forceinline__ bool mbar_wait_suspend(uint64_t* bar, uint32_t parity) {
-  const unsigned long long limit = g_wait_limit_ns;
-  if (limit < kWaitLimitNs) return mbar_poll_for(bar, parity, limit);
-  return mbar_wait_suspend_for(bar, parity, limit);
-}
-
-__device__ __forceinline__ bool mbar_wait_drain_suspend(uint64_t* bar, uint32_t parity) {
-  return mbar_wait_suspend_for(bar, parity, kDrainLimitNs);
-}
-
-__device__ __forceinline__ bool mbar_wait_warp_suspend(uint64_t* bar, uint32_t parity) {
-  return __all_sync(0xffffffffu, mbar_wait_suspend(bar, parity));
-}
-
-__device__ __forceinline__ bool mbar_wait_drain_warp_suspend(uint64_t* bar, uint32_t parity) {
-  return __all_sync(0xffffffffu, mbar_wait_drain_suspend(bar, parity));
-}
 
 // Warp-uniform wait: every lane waits, and the warp agrees on the outcome, so the
 // result can gate warp-collective instructions (mma.sync, tcgen05.ld, __syncwarp).
@@ -192,6 +150,10 @@ __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity) {
 __device__ __forceinline__ bool mbar_wait_drain_warp(uint64_t* bar, uint32_t parity) {
   return __all_sync(0xffffffffu, mbar_wait_drain(bar, parity));
 }
+
+// Orders this thread's view of shared memory between the generic proxy (ld/st) and the
+// async proxy (TMA, tcgen05 operand reads).
+__device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 // ---------------------------------------------------------------- programmatic dependent launch
 // A kernel launched with programmatic stream serialization may start while the

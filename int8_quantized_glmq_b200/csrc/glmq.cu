@@ -572,7 +572,13 @@ glmq_status launch_prefill(const DeviceInfo& dev, const void* X, int M, const vo
   if (M <= 16) return launch_skinny_cfg<SkinnyCfg<BITS, 16, ZP>>(dev, X, M, packed, scale, N, K, Y, s, e);
   if (M <= 32) return launch_skinny_cfg<SkinnyCfg<BITS, 32, ZP>>(dev, X, M, packed, scale, N, K, Y, s, e);
   if (M <= 64) return launch_skinny_cfg<SkinnyCfg<BITS, 64, ZP>>(dev, X, M, packed, scale, N, K, Y, s, e);
+  // tensor-core prefill: 128-token tiles with two accumulators up to M = 128; above 256
+  // tokens INT4 uses 192-token tiles, whose two accumulators still fit in TMEM beside
+  // four A slots (measured faster than 256-token tiles with one accumulator: B200, INT4,
+  // M = 512 and 2048 on the four GLM shapes); otherwise 256-token tiles
   if (M <= 128) return launch_prefill_cfg<PrefillCfg<BITS, 128, ZP>>(dev, X, M, packed, scale, N, K, Y, s, e);
+  if (BITS == 4 && M > 256)
+    return launch_prefill_cfg<PrefillCfg<BITS, 192, ZP>>(dev, X, M, packed, scale, N, K, Y, s, e);
   return launch_prefill_cfg<PrefillCfg<BITS, 256, ZP>>(dev, X, M, packed, scale, N, K, Y, s, e);
 }
 

@@ -18,15 +18,17 @@
 //                128-byte swizzle) and of the packed weight tile (128 rows of
 //                32 / 64 bytes, 32- / 64-byte swizzle) into a kStages ring;
 //   warps 0..15  dequantizers, four independent groups of 128 threads (one weight
-//                row per thread); group g takes every fourth K block, so four K
-//                blocks are dequantized at once. A thread turns its row's 64 codes
-//                into fp16, writes them into the A tile in the canonical K-major
-//                128-byte-swizzled layout and fences the generic->async proxy;
+//                row per thread = one TMEM lane); group g takes every fourth K
+//                block, so four K blocks are dequantized at once. A thread turns its
+//                row's 64 codes into fp16 and writes them with one tcgen05.st into
+//                one of 8 A slots in tensor memory (the A operand never touches
+//                shared memory, which then carries only the X and packed tiles);
 //   warp 21      MMA issuer: the warp runs the issue loop and its elected lane
-//                issues 4 tcgen05.mma (K=16) per 64-wide K block into one of two
-//                TMEM accumulators and commits each stage back to the producer;
+//                issues 4 tcgen05.mma (K=16, A from TMEM, X from shared memory)
+//                per 64-wide K block and commits the A slot and the stage;
 //   warps 16..19 epilogue: tcgen05.ld of its 32 TMEM lanes, times s[n], fp16
-//                stores; frees the accumulator for the next-but-one tile.
+//                stores. Two accumulators when they fit beside the A slots
+//                (BN <= 128), else one, which the next tile's MMAs wait for.
 // Work units are (tile, K part) pairs. Large problems use one part per tile; when
 // there are fewer tiles than SMs (small M), tiles are split over K parts so every
 // SM has work, each unit adds its fp32 partial tile into a scratch buffer with
@@ -47,7 +49,6 @@ constexpr int kPrefillEpilogueWarp0 = 16;
 constexpr int kPrefillProducerWarp = 20;
 constexpr int kPrefillMmaWarp = 21;
 constexpr int kPrefillThreads = 22 * 32;
-constexpr int kPrefillMaxStages = 8;
 constexpr int kPrefillSmemBudget = 232448 - 1024 /*alignment*/ - 512 /*barriers*/;
 
 template <int BITS, int BN, int ZP = 0>
@@ -58,18 +59,28 @@ struct PrefillCfg {
   static constexpr int BM = 128;
   static constexpr int BK = 64;
   static constexpr int X_BYTES = BN * BK * 2;           // B operand tile
-  static constexpr int A_BYTES = BM * BK * 2;           // dequantized A tile
   static constexpr int WROW = BK * BITS / 8;            // packed bytes per row per K block (32 or 64)
   static constexpr int W_BYTES = BM * WROW;
-  static constexpr int STAGE_BYTES = X_BYTES + A_BYTES + W_BYTES;
-  static constexpr int kStages = (kPrefillSmemBudget / STAGE_BYTES) < kPrefillMaxStages
-                                     ? (kPrefillSmemBudget / STAGE_BYTES) : kPrefillMaxStages;
-  static constexpr int TMEM_COLS = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64 : (2 * BN <= 128) ? 128
-                                 : (2 * BN <= 256) ? 256 : 512;
+  static constexpr int STAGE_BYTES = X_BYTES + W_BYTES;
+  // The stage count is a multiple of the dequantizer groups, so each stage (and each A
+  // slot) is only ever waited on by the one group that reads every phase of it.
+  static constexpr int kStageSets = kPrefillSmemBudget / (kPrefillDequantGroups * STAGE_BYTES);
+  static constexpr int kStages = kPrefillDequantGroups * (kStageSets < 2 ? kStageSets : 2);
+  // TMEM: one or two fp32 accumulators of BN columns and the dequantized A operand in
+  // NA slots of one 64-k block (32 columns) each: two accumulators whenever at least
+  // one A slot per dequantizer group fits beside them (at most two per group).
+  static constexpr int kAccBufs = (512 - 2 * BN) / 32 >= kPrefillDequantGroups ? 2 : 1;
+  static constexpr int ACC_COLS = kAccBufs * BN;
+  static constexpr int kSlotsFit = (512 - ACC_COLS) / 32;
+  static constexpr int NA = kSlotsFit >= 2 * kPrefillDequantGroups ? 2 * kPrefillDequantGroups
+                                                                     : kPrefillDequantGroups;
+  static constexpr int A_COLS = NA * 32;
+  static constexpr int TMEM_COLS = 512;
   static constexpr int SMEM_BYTES = kStages * STAGE_BYTES + 1024 /*align*/ + 512 /*barriers*/;
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N for M=128");
   static_assert(X_BYTES % 1024 == 0, "swizzle atoms stay 1024-byte aligned");
-  static_assert(kStages >= 2, "at least double buffering");
+  static_assert(kStages >= kPrefillDequantGroups, "one stage per dequantizer group at least");
+  static_assert(ACC_COLS + A_COLS <= TMEM_COLS, "tensor memory budget");
   // kind::f16, fp32 accumulator, fp16 A and B, both K-major, N = BN, M = 128
   static constexpr uint32_t IDESC = (1u << 4) | (uint32_t(BN >> 3) << 17) | (uint32_t(BM >> 4) << 24);
 };
@@ -182,6 +193,38 @@ __device__ __forceinline__ void umma_commit_elected(uint64_t* bar, uint32_t lead
       : "memory");
 }
 
+// tcgen05.mma kind::f16 with the A operand in TMEM and B in shared memory, the B
+// descriptor given as its two 32-bit halves (an issuing loop offsets the low half,
+// which holds the start address, with plain 32-bit adds). Issued by the elected lane
+// only (leader != 0 in exactly one lane of the issuing warp).
+template <uint32_t kAccumulate>
+__device__ __forceinline__ void umma_f16_tmem_a_lh(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo, uint32_t b_hi,
+                                                   uint32_t idesc, uint32_t leader) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t.reg .b64 bd;\n\t"
+      "setp.ne.b32 p, %5, 0;\n\t"
+      "setp.ne.b32 e, %6, 0;\n\t"
+      "mov.b64 bd, {%2, %3};\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], bd, %4, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "r"(b_lo), "r"(b_hi), "r"(idesc), "n"(kAccumulate), "r"(leader)
+      : "memory");
+}
+
+// Writes 32 consecutive 32-bit TMEM columns of this warp's 32 lanes (lane i: row i of
+// the warp's lane quarter). Asynchronous: tcgen05.wait::st before reusing v.
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
+      "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]),
+      "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]),
+      "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+      : "memory");
+}
+
+
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
@@ -209,17 +252,6 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[32]) {
 }
 
 
-__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-  asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
-}
-
-// Byte offset of 16-byte chunk `c` (8 fp16 along K) of row `row` in a K-major,
-// 128-byte-swizzled tile whose rows are 128 bytes (64 fp16).
-__device__ __forceinline__ uint32_t sw128_off(int row, int c) {
-  return static_cast<uint32_t>((row >> 3) * 1024 + (row & 7) * 128 + ((c ^ (row & 7)) << 4));
-}
-
-// INT4 packed word (8 codes, k = 0..7) -> 4 words of fp16 pairs in natural k order.
 // INT4 word (8 codes) -> fp16 values. A code nibble c OR-ed into the mantissa of 1024
 // (low nibbles: XOR constant xlo) or of 1024 at 16x weight (high nibbles: xhi) gives
 // an exact fp16 integer; adding b0 (low) or scaling by 1/16 and adding b1 (high)
@@ -286,15 +318,18 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                    const PrefillArgs a) {
   constexpr int S = C::kStages;
+  constexpr int NA = C::NA;
+  constexpr int NB = C::kAccBufs;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::STAGE_BYTES);
-  uint64_t* full = bars;                  // TMA bytes landed          (count 1 + tx)
-  uint64_t* afull = bars + S;             // A tile dequantized        (count 4 warps)
-  uint64_t* empty = bars + 2 * S;         // MMAs of the stage done    (tcgen05.commit)
-  uint64_t* accfull = bars + 3 * S;       // accumulator ready         (tcgen05.commit), x2
-  uint64_t* accempty = accfull + 2;       // accumulator drained       (count 4 warps), x2
-  uint64_t* final_bar = accempty + 2;     // all MMAs done, on the failure path (tcgen05.commit)
+  uint64_t* full = bars;                  // X and W tiles landed            (count 1 + tx)
+  uint64_t* empty = bars + S;             // stage's MMAs done               (tcgen05.commit)
+  uint64_t* afull = bars + 2 * S;         // A slot written                  (count 4 warps)
+  uint64_t* aempty = afull + NA;          // A slot's MMAs done              (tcgen05.commit)
+  uint64_t* accfull = aempty + NA;        // accumulator ready               (tcgen05.commit), x NB
+  uint64_t* accempty = accfull + NB;      // accumulator drained             (count 4 warps), x NB
+  uint64_t* final_bar = accempty + NB;    // all MMAs done, on the failure path (tcgen05.commit)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(final_bar + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -304,10 +339,13 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&afull[s], kPrefillDequantWarps / kPrefillDequantGroups);
       mbar_init(&empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int i = 0; i < NA; ++i) {
+      mbar_init(&afull[i], kPrefillDequantWarps / kPrefillDequantGroups);
+      mbar_init(&aempty[i], 1);
+    }
+    for (int b = 0; b < NB; ++b) {
       mbar_init(&accfull[b], 1);
       mbar_init(&accempty[b], 4);
     }
@@ -346,7 +384,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           mbar_arrive_expect_tx(&full[stage], C::X_BYTES + C::W_BYTES);
           armed[stage] = phase + 1;
           tma_load_2d(st, &tmap_x, kb * C::BK, mt * C::kBN, &full[stage]);
-          tma_load_2d(st + C::X_BYTES + C::A_BYTES, &tmap_w, kb * C::WROW, nt * C::BM, &full[stage]);
+          tma_load_2d(st + C::X_BYTES, &tmap_w, kb * C::WROW, nt * C::BM, &full[stage]);
           if (++stage == S) { stage = 0; phase ^= 1; }
         }
       }
@@ -357,10 +395,12 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     }
   } else if (warp < kPrefillDequantWarps) {
     // ------------------------------------------------------------ dequantizers
-    const int row = threadIdx.x & 127;   // tile row (TMEM lane / weight row)
-    const int grp = threadIdx.x >> 7;    // dequant group: K blocks with sequence number % 4 == grp
-    int stage = 0;
-    uint32_t phase = 0;
+    // Group g (warps 4g .. 4g+3, TMEM lanes 32 (w % 4) ...) takes the K blocks with
+    // sequence number % 4 == g: stage seq % S and A slot seq % NA are then always the
+    // group's own, so each barrier it waits on is one whose every phase it takes.
+    const int row = ((warp & 3) << 5) + lane;        // tile row = TMEM lane
+    const int grp = warp >> 2;
+    const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
     int seq = 0;                         // K-block sequence number across this CTA's units
     for (int u = blockIdx.x; u < a.units && ok; u += G) {
       const int p = u / a.tiles;
@@ -371,73 +411,85 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         dq = int4_dequant_zero_point(wrow < a.N ? a.zero[wrow] : 0);
       }
       for (int kb = p * a.kbp; kb < kb1; ++kb, ++seq) {
-        if ((seq & (kPrefillDequantGroups - 1)) == grp) {
-          if (!mbar_wait_warp(&full[stage], phase)) { ok = false; break; }
-          uint8_t* st = smem + stage * C::STAGE_BYTES;
-          const uint32_t a_tile = smem_u32(st + C::X_BYTES);
-          const uint32_t w_tile = smem_u32(st + C::X_BYTES + C::A_BYTES);
-          if constexpr (C::kBits == 4) {
-            // 32-byte rows, 32-byte swizzle: 16-byte unit u sits at u ^ ((row >> 2) & 1)
+        if ((seq & (kPrefillDequantGroups - 1)) != grp) continue;
+        const int stage = seq % S;
+        const int slot = seq % NA;
+        if (!mbar_wait_warp(&full[stage], (seq / S) & 1)) { ok = false; break; }
+        const uint32_t w_tile = smem_u32(smem + stage * C::STAGE_BYTES + C::X_BYTES);
+        uint32_t h[32];                   // the row's 64 fp16 values, natural k order
+        if constexpr (C::kBits == 4) {
+          // 32-byte rows, 32-byte swizzle: 16-byte unit u sits at u ^ ((row >> 2) & 1)
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const uint4 v = lds_v4(w_tile + row * 32 + ((h ^ ((row >> 2) & 1)) << 4));
-              const uint32_t words[4] = {v.x, v.y, v.z, v.w};
+          for (int hh = 0; hh < 2; ++hh) {
+            const uint4 v = lds_v4(w_tile + row * 32 + ((hh ^ ((row >> 2) & 1)) << 4));
+            const uint32_t words[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                const uint4 o = dequant_int4_natural(words[j], dq);
-                st_shared_v4(a_tile + sw128_off(row, 4 * h + j), o.x, o.y, o.z, o.w);
-              }
-            }
-          } else {
-            // 64-byte rows, 64-byte swizzle: unit u sits at u ^ ((row >> 1) & 3)
-#pragma unroll
-            for (int uu = 0; uu < 4; ++uu) {
-              const uint4 v = lds_v4(w_tile + row * 64 + ((uu ^ ((row >> 1) & 3)) << 4));
-              const uint2 lo0 = dequant_int8_natural(v.x), lo1 = dequant_int8_natural(v.y);
-              const uint2 hi0 = dequant_int8_natural(v.z), hi1 = dequant_int8_natural(v.w);
-              st_shared_v4(a_tile + sw128_off(row, 2 * uu), lo0.x, lo0.y, lo1.x, lo1.y);
-              st_shared_v4(a_tile + sw128_off(row, 2 * uu + 1), hi0.x, hi0.y, hi1.x, hi1.y);
+            for (int j = 0; j < 4; ++j) {
+              const uint4 o = dequant_int4_natural(words[j], dq);
+              h[16 * hh + 4 * j + 0] = o.x;
+              h[16 * hh + 4 * j + 1] = o.y;
+              h[16 * hh + 4 * j + 2] = o.z;
+              h[16 * hh + 4 * j + 3] = o.w;
             }
           }
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&afull[stage]);
+        } else {
+          // 64-byte rows, 64-byte swizzle: unit u sits at u ^ ((row >> 1) & 3)
+#pragma unroll
+          for (int uu = 0; uu < 4; ++uu) {
+            const uint4 v = lds_v4(w_tile + row * 64 + ((uu ^ ((row >> 1) & 3)) << 4));
+            const uint2 d0 = dequant_int8_natural(v.x), d1 = dequant_int8_natural(v.y);
+            const uint2 d2 = dequant_int8_natural(v.z), d3 = dequant_int8_natural(v.w);
+            h[8 * uu + 0] = d0.x; h[8 * uu + 1] = d0.y; h[8 * uu + 2] = d1.x; h[8 * uu + 3] = d1.y;
+            h[8 * uu + 4] = d2.x; h[8 * uu + 5] = d2.y; h[8 * uu + 6] = d3.x; h[8 * uu + 7] = d3.y;
+          }
         }
-        if (++stage == S) { stage = 0; phase ^= 1; }
+        if (!mbar_wait_warp(&aempty[slot], ((seq / NA) & 1) ^ 1)) { ok = false; break; }
+        tc_fence_after();
+        tmem_st32(tmem_base + lane_addr + C::ACC_COLS + slot * 32, h);
+        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&afull[slot]);
       }
     }
     if (!ok && lane == 0) report_error(kErrPrefillWait);
   } else if (warp == kPrefillMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
-    // The whole warp runs the loop; the elected lane issues the MMAs and commits.
+    // The whole warp runs the loop; the elected lane issues the MMAs (A from TMEM, the X
+    // tile from shared memory) and commits.
     const uint32_t leader = elect_one_sync();
-    int stage = 0;
-    uint32_t phase = 0;
+    int seq = 0;
     int it = 0;
-    uint32_t acc_armed[2] = {};
+    uint32_t acc_armed[NB] = {};
+    const uint64_t desc0 = umma_desc_sw128(0);
+    const uint32_t desc_hi = static_cast<uint32_t>(desc0 >> 32);
+    // low descriptor half of stage 0's X tile (start address >> 4)
+    const uint32_t x_lo_base = static_cast<uint32_t>(desc0) | ((smem_u32(smem) >> 4) & 0x3FFFu);
+    constexpr uint32_t kStageLo = C::STAGE_BYTES >> 4;
     for (int u = blockIdx.x; u < a.units && ok; u += G, ++it) {
       const int p = u / a.tiles;
       const int kb0 = p * a.kbp;
       const int kb1 = min(num_kb, kb0 + a.kbp);
-      const int ab = it & 1;
-      const uint32_t aphase = (it >> 1) & 1;
+      const int ab = it % NB;
+      const uint32_t aphase = (it / NB) & 1;
       if (!mbar_wait_warp(&accempty[ab], aphase ^ 1)) { ok = false; break; }
       tc_fence_after();
       const uint32_t d_tmem = tmem_base + ab * C::kBN;
-      for (int kb = kb0; kb < kb1; ++kb) {
-        if (!mbar_wait_warp(&afull[stage], phase)) { ok = false; break; }
+      for (int kb = kb0; kb < kb1; ++kb, ++seq) {
+        const int stage = seq % S;
+        const int slot = seq % NA;
+        if (!mbar_wait_warp(&afull[slot], (seq / NA) & 1)) { ok = false; break; }
         tc_fence_after();
-        uint8_t* st = smem + stage * C::STAGE_BYTES;
-        const uint64_t x_desc = umma_desc_sw128(smem_u32(st));
-        const uint64_t a_desc = umma_desc_sw128(smem_u32(st + C::X_BYTES));
-        // k sub-block kk: both operands start kk * 32 bytes further (2 in the descriptor's 16-byte units)
-        if (kb == kb0) umma_f16_elected<0>(d_tmem, a_desc, x_desc, C::IDESC, leader);
-        else umma_f16_elected<1>(d_tmem, a_desc, x_desc, C::IDESC, leader);
-#pragma unroll
-        for (int kk = 1; kk < C::BK / 16; ++kk)
-          umma_f16_elected<1>(d_tmem, a_desc + 2 * kk, x_desc + 2 * kk, C::IDESC, leader);
+        const uint32_t a_tmem = tmem_base + C::ACC_COLS + slot * 32;
+        const uint32_t x_lo = x_lo_base + stage * kStageLo;
+        // k sub-block kk: A columns kk * 8, X start address + kk * 32 bytes
+        if (kb == kb0) umma_f16_tmem_a_lh<0>(d_tmem, a_tmem, x_lo, desc_hi, C::IDESC, leader);
+        else umma_f16_tmem_a_lh<1>(d_tmem, a_tmem, x_lo, desc_hi, C::IDESC, leader);
+        umma_f16_tmem_a_lh<1>(d_tmem, a_tmem + 8, x_lo + 2, desc_hi, C::IDESC, leader);
+        umma_f16_tmem_a_lh<1>(d_tmem, a_tmem + 16, x_lo + 4, desc_hi, C::IDESC, leader);
+        umma_f16_tmem_a_lh<1>(d_tmem, a_tmem + 24, x_lo + 6, desc_hi, C::IDESC, leader);
+        umma_commit_elected(&aempty[slot], leader);
         umma_commit_elected(&empty[stage], leader);
-        if (++stage == S) { stage = 0; phase ^= 1; }
       }
       if (!ok) break;
       umma_commit_elected(&accfull[ab], leader);
@@ -446,7 +498,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     // make sure no MMA is still reading shared memory or writing TMEM before the CTA
     // exits and the allocation is released
     bool drained = true;
-    for (int b = 0; b < 2; ++b)
+    for (int b = 0; b < NB; ++b)
       if (acc_armed[b] && !mbar_wait_drain_warp(&accfull[b], acc_armed[b] - 1)) drained = false;
     if (!ok) {
       // a wait gave up mid-unit: MMAs may have been issued after the last commit above
@@ -455,13 +507,13 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     }
     if ((!ok || !drained) && lane == 0) report_error(kErrPrefillWait);
   } else {
-    // ------------------------------------------------------------ epilogue warps 8..11
+    // ------------------------------------------------------------ epilogue warps 16..19
     const int quarter = warp & 3;   // TMEM lanes 32*quarter .. 32*quarter+31
     const bool split = a.parts > 1;
     int it = 0;
     for (int u = blockIdx.x; u < a.units && ok; u += G, ++it) {
-      const int ab = it & 1;
-      const uint32_t aphase = (it >> 1) & 1;
+      const int ab = it % NB;
+      const uint32_t aphase = (it / NB) & 1;
       if (!mbar_wait_warp(&accfull[ab], aphase)) { ok = false; break; }
       tc_fence_after();
       const int t = u % a.tiles;

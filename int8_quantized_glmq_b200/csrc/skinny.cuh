@@ -95,32 +95,6 @@ struct SkinnyCfg {
   static constexpr uint32_t IDESC = (1u << 4) | (uint32_t(BN >> 3) << 17) | (uint32_t(BM >> 4) << 24);
 };
 
-__device__ __forceinline__ void umma_f16_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
-                                                uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// The same MMA with the B descriptor given as its two 32-bit halves (the issuing loop
-// offsets the low half, which holds the start address, with plain 32-bit adds).
-// Issued by the elected lane only (leader != 0 in exactly one lane of the issuing warp).
-template <uint32_t kAccumulate>
-__device__ __forceinline__ void umma_f16_tmem_a_lh(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo, uint32_t b_hi,
-                                                   uint32_t idesc, uint32_t leader) {
-  asm volatile(
-      "{\n\t.reg .pred p, e;\n\t.reg .b64 bd;\n\t"
-      "setp.ne.b32 p, %5, 0;\n\t"
-      "setp.ne.b32 e, %6, 0;\n\t"
-      "mov.b64 bd, {%2, %3};\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], bd, %4, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "r"(b_lo), "r"(b_hi), "r"(idesc), "n"(kAccumulate), "r"(leader)
-      : "memory");
-}
-
 // One 64-wide K block: 4 MMAs (K = 16 each). Sub-block kk reads A columns kk * 8 of
 // the slot and B from the tile's start address + kk * 32 bytes (+2 in the low
 // descriptor half). kFirst: the block opens the accumulator (no accumulate).
@@ -130,18 +104,6 @@ __device__ __forceinline__ void skinny_mma_block(uint32_t d, uint32_t a, uint32_
   umma_f16_tmem_a_lh<1>(d, a + 8, b_lo + 2, b_hi, C::IDESC, leader);
   umma_f16_tmem_a_lh<1>(d, a + 16, b_lo + 4, b_hi, C::IDESC, leader);
   umma_f16_tmem_a_lh<1>(d, a + 24, b_lo + 6, b_hi, C::IDESC, leader);
-}
-
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
-      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
-      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
-      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
-      "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]),
-      "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]),
-      "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
-      : "memory");
 }
 
 // Pre-pass: X fp16 [M, K] -> the shared-memory image of every activation tile the

@@ -209,6 +209,15 @@ def time_launches(torch, fn, iters: int, warmup: int = 2):
     return e0.elapsed_time(e1) / 1e3 / iters
 
 
+def settle(torch, seconds: float = 0.3):
+    """Idle the GPU briefly between a tensor-heavy measurement and a memory-bound one:
+    right after the M=2048 GEMMs the SM clock sits below its maximum under the power
+    cap for a while, and the first memory-bound measurement after them read 10-25%
+    slow."""
+    torch.cuda.synchronize()
+    time.sleep(seconds)
+
+
 def time_launches_cold(torch, fn, iters: int, warmup: int = 8):
     """Average device time of fn() per call with L2 made cold before each call: a read
     of a 256 MB buffer between calls, outside the timed events. A read leaves clean
@@ -499,6 +508,7 @@ def run_extras(torch, glmq, W16, quant, peaks):
     # ridge of the roofline, so both roofs are reported with the one that binds. L2 is
     # flushed before each timed call (attn-out's 75 MB of codes would otherwise stay in L2).
     out["int4_m64"] = {}
+    settle(torch)
     for name in PROJECTION_ORDER:
         N, K = GLM_PROJECTIONS[name]
         packed, scale = quant[name]
@@ -580,6 +590,7 @@ def run_extras(torch, glmq, W16, quant, peaks):
         s8 = torch.empty((N,), dtype=torch.float16, device="cuda")
         tq = time_launches(torch, lambda: glmq.quantize(W16[name], 8, out=(p8, s8)), 3)
         res = {"quantize_us": round(tq * 1e6, 1), "quantize_gbs": round((N * K * 3 + N * 2) / tq / 1e9, 1)}
+        settle(torch)
         for M in (1, 64, 2048):
             g = torch.Generator(device="cuda").manual_seed(4000 + M)
             X = torch.randn((M, K), generator=g, device="cuda", dtype=torch.float32).half()
@@ -733,9 +744,14 @@ class Sweep:
         self.kernels_per_replay = glmq.kernel_launches() - n0
 
     def _step(self, glmq):
-        for layer, p, n in self.order:
+        # each call names the next one (the next projection, or layer 0's first after the
+        # last layer) so that its weights' first tiles are prefetched into L2 while this
+        # call's ring drains, as a serving loop through the layers would call it
+        for i, (layer, p, n) in enumerate(self.order):
             out = self.kept.get((layer, n), self.ys[n])
-            glmq.gemm(self.xs[n], self.quant[layer][p][0], self.quant[layer][p][1], 4, out=out)
+            nl, np_, _ = self.order[(i + 1) % len(self.order)]
+            glmq.gemm_decode_prefetch(self.xs[n], self.quant[layer][p][0], self.quant[layer][p][1], 4,
+                                      next_packed=self.quant[nl][np_][0], next_M=1, out=out)
 
     def time_replays(self, torch, steps: int, warmup: int, world: int = 1):
         """Device seconds of `steps` replays (CUDA events on the current stream)."""

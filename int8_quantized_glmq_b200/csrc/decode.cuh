@@ -23,7 +23,8 @@
 //    box (128-byte swizzle, L2 evict-first hint; rows past N and bytes past K
 //    zero-filled).
 //  * Warps 17.. are activation warps (one for M <= 2, three for larger M; warp 17 + i
-//    takes the stages with sequence number i mod their count). Once a slot's raw
+//    takes the stages with sequence number i mod their count, each only after the
+//    previous phase of its ring stage has been handed on). Once a slot's raw
 //    activations have landed the warp
 //    rewrites them in place into fragment order, dividing the high-nibble slots by 16
 //    (see below), with a lane-to-unit mapping under which both the reads and the
@@ -520,6 +521,13 @@ __global__ void __launch_bounds__(C::kThreads, 1)
         if (C::kXWarps > 1 && q % C::kXWarps != xw) continue;
         const int stage = q % S;
         const uint32_t phase = static_cast<uint32_t>(q / S) & 1u;
+        if (C::kXWarps > 1 && S % C::kXWarps != 0 && q >= S) {
+          // Successive phases of this stage fall to different warps (3 warps, 5 stages
+          // at MP = 16). A parity wait on phase n + 1 passes at once while phase n is
+          // still incomplete, so first wait until the stage's previous phase has been
+          // released to the consumers: fullr is then at the phase waited on below.
+          if (!DECODE_WAIT_X(&fullx[stage], phase ^ 1u)) { ok = false; break; }
+        }
         if (!DECODE_WAIT_X(&fullr[stage], phase)) { ok = false; break; }
         const uint32_t slot = smem_u32(xring + stage * C::X_BYTES);
         float bsum[2] = {0.0f, 0.0f}, ssum[2] = {0.0f, 0.0f};

@@ -12,19 +12,21 @@
 
 namespace glmq {
 
-// Y[m, n] = fp16(s[n] * ws[m, n]) for split calls; returns ws to zero.
-// Grid: x covers the columns in groups of VEC per thread (one pass), y the token rows
-// (rows m = blockIdx.y, blockIdx.y + gridDim.y, ...). VEC = 4 needs N % 4 == 0, so
-// every group is 16-byte aligned in ws and 8-byte aligned in Y and scale.
+// Y[m, n] = fp16(s[n] * ws[m, n]) for split calls, columns n0 <= n < N (the split
+// tiles' rows of W); returns those ws entries to zero.
+// Grid: x covers the columns from n0 in groups of VEC per thread (one pass), y the
+// token rows (rows m = blockIdx.y, blockIdx.y + gridDim.y, ...). VEC = 4 needs N % 4
+// == 0 and n0 % 4 == 0, so every group is 16-byte aligned in ws and 8-byte aligned in
+// Y and scale.
 template <int VEC>
 __global__ void __launch_bounds__(256) decode_finalize_kernel(float* __restrict__ ws, const __half* __restrict__ scale,
-                                                              __half* __restrict__ Y, int M, int N) {
+                                                              __half* __restrict__ Y, int M, int N, int n0) {
   // Let the next kernel in the stream launch now: its CTAs take their SM slots and run
   // their shared-memory prologue while this pass waits; every kernel launched with a
   // grid dependency here waits (griddep_wait) for this one before touching memory.
   griddep_launch_dependents();
   griddep_wait();   // the partial sums come from the kernel before this one
-  const int n = (blockIdx.x * 256 + threadIdx.x) * VEC;
+  const int n = n0 + (blockIdx.x * 256 + threadIdx.x) * VEC;
   if (n >= N) return;
   if constexpr (VEC == 4) {
     const uint2 sv = __ldg(reinterpret_cast<const uint2*>(scale + n));
@@ -53,17 +55,18 @@ __global__ void __launch_bounds__(256) decode_finalize_kernel(float* __restrict_
 }
 
 // The same pass with a fused epilogue (a bias, and/or GeGLU over a GeGLU-layout
-// weight): one thread per output column j of a token row, Y of width N (bias only) or
-// N / 2 (GeGLU). For GeGLU, output j reads packed rows pa = 16 (j / 8) + j % 8 and
-// pa + 8, and returns both scratch entries to zero.
+// weight): one thread per output column j >= j0 of a token row, Y of width N (bias
+// only) or N / 2 (GeGLU). For GeGLU, output j reads packed rows pa = 16 (j / 8) + j % 8
+// and pa + 8, and returns both scratch entries to zero; the packed rows from n0 on are
+// the outputs from j0 = n0 / 2 on (n0 a multiple of 16).
 __global__ void __launch_bounds__(256) finalize_epilogue_kernel(float* __restrict__ ws,
                                                                 const __half* __restrict__ scale,
                                                                 const __half* __restrict__ bias, int geglu,
-                                                                __half* __restrict__ Y, int M, int N) {
+                                                                __half* __restrict__ Y, int M, int N, int j0) {
   griddep_launch_dependents();   // as in decode_finalize_kernel
   griddep_wait();   // the partial sums come from the kernel before this one
   const int width = geglu ? (N >> 1) : N;
-  const int j = blockIdx.x * 256 + threadIdx.x;
+  const int j = j0 + blockIdx.x * 256 + threadIdx.x;
   if (j >= width) return;
   if (!geglu) {
     const float sj = __half2float(scale[j]);

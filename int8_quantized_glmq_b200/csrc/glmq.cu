@@ -272,22 +272,25 @@ struct Epi {
 };
 
 // Launches finalize_epilogue_kernel: one thread per output column of every token row.
+// Columns (packed rows of W) n0 .. N-1 only: the rows of the tiles that were split.
 glmq_status launch_finalize_epi(float* ws, const __half* scale, const Epi& e, __half* Y, int M, int N,
-                                cudaStream_t s) {
+                                cudaStream_t s, int n0 = 0) {
   const int width = e.geglu ? N / 2 : N;
-  const dim3 grid(static_cast<unsigned>((width + 255) / 256), static_cast<unsigned>(std::min(M, 65535)));
-  return launch_pdl(finalize_epilogue_kernel, grid, dim3(256), 0, s, ws, scale, e.bias, e.geglu, Y, M, N);
+  const int j0 = e.geglu ? n0 / 2 : n0;
+  const dim3 grid(static_cast<unsigned>((width - j0 + 255) / 256), static_cast<unsigned>(std::min(M, 65535)));
+  return launch_pdl(finalize_epilogue_kernel, grid, dim3(256), 0, s, ws, scale, e.bias, e.geglu, Y, M, N, j0);
 }
 
 // Launches decode_finalize_kernel: one thread per group of 4 columns (1 when N is not
 // a multiple of 4) of every token row, all in one pass (rows beyond the grid's y
 // extent loop).
-glmq_status launch_finalize(float* ws, const __half* scale, __half* Y, int M, int N, cudaStream_t s) {
+// Columns n0 .. N-1 only (n0 a multiple of 16): the rows of the tiles that were split.
+glmq_status launch_finalize(float* ws, const __half* scale, __half* Y, int M, int N, cudaStream_t s, int n0 = 0) {
   const bool vec = (N % 4) == 0;
-  const int groups = vec ? N / 4 : N;
+  const int groups = vec ? (N - n0) / 4 : N - n0;
   const dim3 grid(static_cast<unsigned>((groups + 255) / 256), static_cast<unsigned>(std::min(M, 65535)));
-  if (vec) return launch_pdl(decode_finalize_kernel<4>, grid, dim3(256), 0, s, ws, scale, Y, M, N);
-  return launch_pdl(decode_finalize_kernel<1>, grid, dim3(256), 0, s, ws, scale, Y, M, N);
+  if (vec) return launch_pdl(decode_finalize_kernel<4>, grid, dim3(256), 0, s, ws, scale, Y, M, N, n0);
+  return launch_pdl(decode_finalize_kernel<1>, grid, dim3(256), 0, s, ws, scale, Y, M, N, n0);
 }
 
 // Per-device buffer for the skinny kernel's pre-swizzled activation tiles (grown on
@@ -447,6 +450,32 @@ glmq_status launch_decode(const DeviceInfo& dev, const void* X, int M, const voi
 }
 
 // ---------------------------------------------------------------- prefill
+// With at least as many tiles as SMs, whole tiles fill waves = tiles / sms rounds of
+// the persistent CTAs, and a last, partial round would keep the CTAs that have a tile
+// in it busy for a whole tile time while the others idle. Instead, the tiles from the
+// weight-row band that contains tile waves * sms on (a band is tiles_m tiles, so the
+// split tiles cover whole rows of W and the finalize pass covers only those rows) are
+// split over P K parts: the first (tiles before the band) stay whole. The split units
+// fill the CTAs left idle in the last whole round and then at most one more round of
+// 1/P of a tile: about waves + 1/P tile times instead of waves + 1. Taken when P >= 2
+// and the tile time saved (at ~10 TFLOP/s per SM) is above the ~5 us of a finalize
+// launch. Sets *full and *parts; leaves them alone otherwise.
+void plan_tail_split(int tiles, int tiles_m, int num_steps, int min_steps_per_part, int sms, double tile_flops,
+                     int* full, int* parts) {
+  if (tiles < sms || tiles % sms == 0) return;
+  const int waves = tiles / sms;
+  const int whole = (waves * sms / tiles_m) * tiles_m;
+  const int rest = tiles - whole;
+  const int idle = waves * sms - whole;            // CTAs without a whole tile in the last whole round
+  int P = (sms + idle) / rest;
+  if (P > num_steps / min_steps_per_part) P = num_steps / min_steps_per_part;
+  if (P > 16) P = 16;
+  if (P < 2) return;
+  if (tile_flops * (1.0 - 1.0 / P) < 5e-6 * 1e13) return;
+  *full = whole;
+  *parts = P;
+}
+
 // Choose K parts for `tiles` tiles of `num_steps` K steps each: only when there are
 // fewer tiles than SMs, the split that spreads (tile, part) units most evenly,
 // preferring fewer parts (each split tile costs a round trip of fp32 partial sums
@@ -496,10 +525,15 @@ glmq_status launch_prefill_cfg(const DeviceInfo& dev, const void* X, int M, cons
   if (tiles > 0x7fffffffLL / 64) return GLMQ_ERR_BAD_SHAPE;
   a.tiles = static_cast<int>(tiles);
   const int num_kb = K / C::BK;
-  const int parts = plan_parts(a.tiles, num_kb, 4, dev.sms);
+  int parts = plan_parts(a.tiles, num_kb, 4, dev.sms);
+  a.full = 0;
+  if (parts == 1) {
+    const double tile_flops = 2.0 * C::BM * C::kBN * K;
+    plan_tail_split(a.tiles, a.tiles_m, num_kb, 4, dev.sms, tile_flops, &a.full, &parts);
+  }
   a.kbp = (num_kb + parts - 1) / parts;
   a.parts = (num_kb + a.kbp - 1) / a.kbp;
-  a.units = a.tiles * a.parts;
+  a.units = a.full + (a.tiles - a.full) * a.parts;
   if (a.parts > 1 && (st = decode_scratch(static_cast<size_t>(M) * N, &a.ws)) != GLMQ_OK) return st;
   if (C::SMEM_BYTES > dev.smem_optin) return GLMQ_ERR_BAD_SHAPE;
   if ((st = allow_smem(prefill_kernel<C>, C::SMEM_BYTES)) != GLMQ_OK) return st;
@@ -507,8 +541,10 @@ glmq_status launch_prefill_cfg(const DeviceInfo& dev, const void* X, int M, cons
   prefill_kernel<C><<<grid, kPrefillThreads, C::SMEM_BYTES, s>>>(tx, tw, a);
   if ((st = launched()) != GLMQ_OK) return st;
   if (a.parts > 1) {
-    st = (e.bias || e.geglu) ? launch_finalize_epi(a.ws, a.scale, e, a.Y, M, N, s)
-                             : launch_finalize(a.ws, a.scale, a.Y, M, N, s);
+    // the split tiles are the weight-row bands from full / tiles_m on
+    const int n0 = (a.full / a.tiles_m) * C::BM;
+    st = (e.bias || e.geglu) ? launch_finalize_epi(a.ws, a.scale, e, a.Y, M, N, s, n0)
+                             : launch_finalize(a.ws, a.scale, a.Y, M, N, s, n0);
     if (st != GLMQ_OK) return st;
   }
   return GLMQ_OK;
@@ -544,6 +580,7 @@ glmq_status launch_skinny_cfg(const DeviceInfo& dev, const void* X, int M, const
   const int parts = plan_parts(a.tiles, num_st, 2, dev.sms);
   a.kbp = (num_st + parts - 1) / parts;          // stages per part
   a.parts = (num_st + a.kbp - 1) / a.kbp;
+  a.full = 0;
   a.units = a.tiles * a.parts;
   if (a.parts > 1 && (st = decode_scratch(static_cast<size_t>(M) * N, &a.ws)) != GLMQ_OK) return st;
   if (C::SMEM_BYTES > dev.smem_optin) return GLMQ_ERR_BAD_SHAPE;

@@ -98,10 +98,41 @@ struct PrefillArgs {
   int K;
   int tiles_m;
   int tiles;
-  int parts;      // K parts per tile
+  int parts;      // K parts per split tile
   int kbp;        // K blocks per part
-  int units;      // tiles * parts
+  // prefill kernel: tiles 0 .. full-1 are whole units (units 0 .. full-1); tiles full ..
+  // tiles-1 are split over the parts, K-part major. full = 0: every tile is split
+  // (parts == 1: none is). The skinny kernel uses full = 0.
+  int full;
+  int units;      // full + (tiles - full) * parts
 };
+
+// Work unit u of the prefill kernel: tile t (= nt * tiles_m + mt), its K blocks
+// [kb0, kb1), and whether its sums go through the scratch (split tiles).
+struct PrefillUnit {
+  int t;
+  int kb0;
+  int kb1;
+  bool split;
+};
+__device__ __forceinline__ PrefillUnit prefill_unit(const PrefillArgs& a, int u, int num_kb) {
+  PrefillUnit w;
+  if (u < a.full) {
+    w.t = u;
+    w.kb0 = 0;
+    w.kb1 = num_kb;
+    w.split = false;
+    return w;
+  }
+  const int rest = a.tiles - a.full;
+  const int v = u - a.full;
+  const int p = v / rest;
+  w.t = a.full + (v - p * rest);
+  w.kb0 = p * a.kbp;
+  w.kb1 = min(num_kb, w.kb0 + a.kbp);
+  w.split = a.parts > 1;
+  return w;
+}
 
 // Epilogue of one TMEM lane (packed weight row n) for tokens m0 .. m0 + mend - 1,
 // called by all 32 lanes of an epilogue warp (the GeGLU pair of row n, n % 16 < 8,
@@ -373,12 +404,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       for (int u = blockIdx.x; u < a.units && ok; u += G) {
-        const int p = u / a.tiles;
-        const int t = u - p * a.tiles;
-        const int nt = t / a.tiles_m;
-        const int mt = t - nt * a.tiles_m;
-        const int kb1 = min(num_kb, (p + 1) * a.kbp);
-        for (int kb = p * a.kbp; kb < kb1; ++kb) {
+        const PrefillUnit w = prefill_unit(a, u, num_kb);
+        const int nt = w.t / a.tiles_m;
+        const int mt = w.t - nt * a.tiles_m;
+        for (int kb = w.kb0; kb < w.kb1; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1)) { ok = false; break; }
           uint8_t* st = smem + stage * C::STAGE_BYTES;
           mbar_arrive_expect_tx(&full[stage], C::X_BYTES + C::W_BYTES);
@@ -403,14 +432,13 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
     int seq = 0;                         // K-block sequence number across this CTA's units
     for (int u = blockIdx.x; u < a.units && ok; u += G) {
-      const int p = u / a.tiles;
-      const int kb1 = min(num_kb, (p + 1) * a.kbp);
+      const PrefillUnit w = prefill_unit(a, u, num_kb);
       Int4Dequant dq = int4_dequant_symmetric();
       if constexpr (C::kZP) {
-        const int wrow = ((u - p * a.tiles) / a.tiles_m) * C::BM + row;
+        const int wrow = (w.t / a.tiles_m) * C::BM + row;
         dq = int4_dequant_zero_point(wrow < a.N ? a.zero[wrow] : 0);
       }
-      for (int kb = p * a.kbp; kb < kb1; ++kb, ++seq) {
+      for (int kb = w.kb0; kb < w.kb1; ++kb, ++seq) {
         if ((seq & (kPrefillDequantGroups - 1)) != grp) continue;
         const int stage = seq % S;
         const int slot = seq % NA;
@@ -467,9 +495,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     const uint32_t x_lo_base = static_cast<uint32_t>(desc0) | ((smem_u32(smem) >> 4) & 0x3FFFu);
     constexpr uint32_t kStageLo = C::STAGE_BYTES >> 4;
     for (int u = blockIdx.x; u < a.units && ok; u += G, ++it) {
-      const int p = u / a.tiles;
-      const int kb0 = p * a.kbp;
-      const int kb1 = min(num_kb, kb0 + a.kbp);
+      const PrefillUnit w = prefill_unit(a, u, num_kb);
+      const int kb0 = w.kb0;
+      const int kb1 = w.kb1;
       const int ab = it % NB;
       const uint32_t aphase = (it / NB) & 1;
       if (!mbar_wait_warp(&accempty[ab], aphase ^ 1)) { ok = false; break; }
@@ -509,16 +537,16 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   } else {
     // ------------------------------------------------------------ epilogue warps 16..19
     const int quarter = warp & 3;   // TMEM lanes 32*quarter .. 32*quarter+31
-    const bool split = a.parts > 1;
     int it = 0;
     for (int u = blockIdx.x; u < a.units && ok; u += G, ++it) {
       const int ab = it % NB;
       const uint32_t aphase = (it / NB) & 1;
       if (!mbar_wait_warp(&accfull[ab], aphase)) { ok = false; break; }
       tc_fence_after();
-      const int t = u % a.tiles;
-      const int nt = t / a.tiles_m;
-      const int mt = t - nt * a.tiles_m;
+      const PrefillUnit w = prefill_unit(a, u, num_kb);
+      const bool split = w.split;
+      const int nt = w.t / a.tiles_m;
+      const int mt = w.t - nt * a.tiles_m;
       const int n = nt * C::BM + quarter * 32 + lane;
       const float s = (n < a.N) ? __half2float(a.scale[n]) : 0.0f;
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + ab * C::kBN;

@@ -2,6 +2,13 @@
 // sums of all parts have been added into a scratch buffer ws [M, N]; this kernel
 // applies the per-row scale, rounds to fp16 (the epilogue of the dequantizing linear
 // layer, Y = fp16(s[n] * sum_k X q)) and returns ws to zero for the next call.
+//
+// The pass sits on the critical path between two GEMM kernels, so it is built for
+// latency: each thread loads up to kFinalizeRows token rows of its columns at once, and
+// the per-column constants (scale, bias) are read before the grid-dependency wait. That
+// is safe: they are not written by the GEMM kernel this pass follows, and that kernel
+// had itself waited for every kernel before it (or, launched without a grid dependency,
+// started only after them) before this pass could launch.
 #pragma once
 
 #include <cuda_fp16.h>
@@ -12,12 +19,16 @@
 
 namespace glmq {
 
+// Token rows a thread of decode_finalize_kernel<4> handles with its loads in flight together.
+constexpr int kFinalizeRows = 16;
+
 // Y[m, n] = fp16(s[n] * ws[m, n]) for split calls, columns n0 <= n < N (the split
 // tiles' rows of W); returns those ws entries to zero.
-// Grid: x covers the columns from n0 in groups of VEC per thread (one pass), y the
-// token rows (rows m = blockIdx.y, blockIdx.y + gridDim.y, ...). VEC = 4 needs N % 4
-// == 0 and n0 % 4 == 0, so every group is 16-byte aligned in ws and 8-byte aligned in
-// Y and scale.
+// Grid: x covers the columns from n0 in groups of VEC per thread (one pass). VEC = 4:
+// y covers the token rows in blocks of kFinalizeRows (rows m0 .. m0 + 15 with m0 =
+// 16 blockIdx.y, 16 (blockIdx.y + gridDim.y), ...); it needs N % 4 == 0 and n0 % 4 ==
+// 0, so every group is 16-byte aligned in ws and 8-byte aligned in Y and scale.
+// VEC = 1: y covers single rows (m = blockIdx.y, blockIdx.y + gridDim.y, ...).
 template <int VEC>
 __global__ void __launch_bounds__(256) decode_finalize_kernel(float* __restrict__ ws, const __half* __restrict__ scale,
                                                               __half* __restrict__ Y, int M, int N, int n0) {
@@ -25,26 +36,41 @@ __global__ void __launch_bounds__(256) decode_finalize_kernel(float* __restrict_
   // their shared-memory prologue while this pass waits; every kernel launched with a
   // grid dependency here waits (griddep_wait) for this one before touching memory.
   griddep_launch_dependents();
-  griddep_wait();   // the partial sums come from the kernel before this one
   const int n = n0 + (blockIdx.x * 256 + threadIdx.x) * VEC;
-  if (n >= N) return;
+  const bool live = n < N;
+  uint2 sv = make_uint2(0, 0);
+  float sn = 0.0f;
+  if (live) {   // per-column constants before the wait (see the top of this file)
+    if constexpr (VEC == 4) sv = __ldg(reinterpret_cast<const uint2*>(scale + n));
+    else sn = __half2float(scale[n]);
+  }
+  griddep_wait();   // the partial sums come from the kernel before this one
+  if (!live) return;
   if constexpr (VEC == 4) {
-    const uint2 sv = __ldg(reinterpret_cast<const uint2*>(scale + n));
     const float2 s01 = __half22float2(*reinterpret_cast<const __half2*>(&sv.x));
     const float2 s23 = __half22float2(*reinterpret_cast<const __half2*>(&sv.y));
-    for (int m = blockIdx.y; m < M; m += gridDim.y) {
-      const long long idx = static_cast<long long>(m) * N + n;
-      const float4 v = __ldcg(reinterpret_cast<const float4*>(ws + idx));
-      __stcg(reinterpret_cast<float4*>(ws + idx), make_float4(0.0f, 0.0f, 0.0f, 0.0f));
-      const __half2 y01 = __floats2half2_rn(s01.x * v.x, s01.y * v.y);
-      const __half2 y23 = __floats2half2_rn(s23.x * v.z, s23.y * v.w);
-      uint2 o;
-      o.x = *reinterpret_cast<const uint32_t*>(&y01);
-      o.y = *reinterpret_cast<const uint32_t*>(&y23);
-      *reinterpret_cast<uint2*>(Y + idx) = o;
+    constexpr int R = kFinalizeRows;
+    for (int m0 = blockIdx.y * R; m0 < M; m0 += gridDim.y * R) {
+      float4 v[R];
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        const long long idx = static_cast<long long>(m0 + r) * N + n;
+        v[r] = (m0 + r < M) ? __ldcg(reinterpret_cast<const float4*>(ws + idx)) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        if (m0 + r >= M) break;
+        const long long idx = static_cast<long long>(m0 + r) * N + n;
+        __stcg(reinterpret_cast<float4*>(ws + idx), make_float4(0.0f, 0.0f, 0.0f, 0.0f));
+        const __half2 y01 = __floats2half2_rn(s01.x * v[r].x, s01.y * v[r].y);
+        const __half2 y23 = __floats2half2_rn(s23.x * v[r].z, s23.y * v[r].w);
+        uint2 o;
+        o.x = *reinterpret_cast<const uint32_t*>(&y01);
+        o.y = *reinterpret_cast<const uint32_t*>(&y23);
+        *reinterpret_cast<uint2*>(Y + idx) = o;
+      }
     }
   } else {
-    const float sn = __half2float(scale[n]);
     for (int m = blockIdx.y; m < M; m += gridDim.y) {
       const long long idx = static_cast<long long>(m) * N + n;
       const float v = __ldcg(ws + idx);
@@ -64,13 +90,24 @@ __global__ void __launch_bounds__(256) finalize_epilogue_kernel(float* __restric
                                                                 const __half* __restrict__ bias, int geglu,
                                                                 __half* __restrict__ Y, int M, int N, int j0) {
   griddep_launch_dependents();   // as in decode_finalize_kernel
-  griddep_wait();   // the partial sums come from the kernel before this one
   const int width = geglu ? (N >> 1) : N;
   const int j = j0 + blockIdx.x * 256 + threadIdx.x;
-  if (j >= width) return;
+  if (j >= width) {
+    griddep_wait();
+    return;
+  }
+  // per-column constants before the wait (see the top of this file)
+  const int F = N >> 1;
+  const int pa = geglu ? 16 * (j >> 3) + (j & 7) : j;
+  const int pb = pa + 8;
+  const float sa = __half2float(scale[pa]);
+  const float sb = geglu ? __half2float(scale[pb]) : 0.0f;
+  const float ba = bias ? __half2float(bias[j]) : 0.0f;
+  const float bb = (bias && geglu) ? __half2float(bias[F + j]) : 0.0f;
+  griddep_wait();   // the partial sums come from the kernel before this one
   if (!geglu) {
-    const float sj = __half2float(scale[j]);
-    const float bj = bias ? __half2float(bias[j]) : 0.0f;
+    const float sj = sa;
+    const float bj = ba;
     for (int m = blockIdx.y; m < M; m += gridDim.y) {
       const long long idx = static_cast<long long>(m) * N + j;
       const float v = __ldcg(ws + idx);
@@ -78,12 +115,6 @@ __global__ void __launch_bounds__(256) finalize_epilogue_kernel(float* __restric
       Y[idx] = __float2half_rn(sj * v + bj);
     }
   } else {
-    const int F = N >> 1;
-    const int pa = 16 * (j >> 3) + (j & 7);
-    const int pb = pa + 8;
-    const float sa = __half2float(scale[pa]), sb = __half2float(scale[pb]);
-    const float ba = bias ? __half2float(bias[j]) : 0.0f;
-    const float bb = bias ? __half2float(bias[F + j]) : 0.0f;
     for (int m = blockIdx.y; m < M; m += gridDim.y) {
       const long long row = static_cast<long long>(m) * N;
       const float va = __ldcg(ws + row + pa), vb = __ldcg(ws + row + pb);

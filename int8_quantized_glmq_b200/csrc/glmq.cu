@@ -281,14 +281,15 @@ glmq_status launch_finalize_epi(float* ws, const __half* scale, const Epi& e, __
   return launch_pdl(finalize_epilogue_kernel, grid, dim3(256), 0, s, ws, scale, e.bias, e.geglu, Y, M, N, j0);
 }
 
-// Launches decode_finalize_kernel: one thread per group of 4 columns (1 when N is not
-// a multiple of 4) of every token row, all in one pass (rows beyond the grid's y
-// extent loop).
+// Launches decode_finalize_kernel: one thread per group of 4 columns and block of
+// kFinalizeRows token rows (per column and row when N is not a multiple of 4), all in
+// one pass (rows beyond the grid's y extent loop).
 // Columns n0 .. N-1 only (n0 a multiple of 16): the rows of the tiles that were split.
 glmq_status launch_finalize(float* ws, const __half* scale, __half* Y, int M, int N, cudaStream_t s, int n0 = 0) {
   const bool vec = (N % 4) == 0;
   const int groups = vec ? (N - n0) / 4 : N - n0;
-  const dim3 grid(static_cast<unsigned>((groups + 255) / 256), static_cast<unsigned>(std::min(M, 65535)));
+  const int rows = vec ? (M + kFinalizeRows - 1) / kFinalizeRows : M;
+  const dim3 grid(static_cast<unsigned>((groups + 255) / 256), static_cast<unsigned>(std::min(rows, 65535)));
   if (vec) return launch_pdl(decode_finalize_kernel<4>, grid, dim3(256), 0, s, ws, scale, Y, M, N, n0);
   return launch_pdl(decode_finalize_kernel<1>, grid, dim3(256), 0, s, ws, scale, Y, M, N, n0);
 }

@@ -587,14 +587,22 @@ glmq_status launch_skinny_cfg(const DeviceInfo& dev, const void* X, int M, const
   if (C::SMEM_BYTES > dev.smem_optin) return GLMQ_ERR_BAD_SHAPE;
   if ((st = allow_smem(skinny_kernel<C>, C::SMEM_BYTES)) != GLMQ_OK) return st;
   const int grid = a.units < dev.sms ? a.units : dev.sms;
+  // Both launches carry a grid dependency. The pre-pass (one small block per SM at most,
+  // so a skinny CTA fits beside it) lets the skinny kernel launch at once; the
+  // skinny kernel's weight producer then streams weight boxes while the pre-pass runs,
+  // and only its activation producer (and epilogue) wait for the pre-pass. Reading the
+  // weights, scales and zero points early is safe: the pre-pass let the skinny kernel
+  // launch only after its own grid-dependency wait, i.e. after every earlier kernel
+  // had completed, and the pre-pass writes none of them.
   {
     const long long units16 = static_cast<long long>(K / 64) * C::kBN * 8;
-    const int blocks = static_cast<int>(std::min<long long>((units16 + 255) / 256, 8LL * dev.sms));
-    skinny_pack_x_kernel<C><<<blocks, 256, 0, s>>>(static_cast<const __half*>(X), M, K, xs);
-    if ((st = launched()) != GLMQ_OK) return st;
+    const int blocks = static_cast<int>(std::min<long long>((units16 + kPackThreads - 1) / kPackThreads, dev.sms));
+    if ((st = launch_pdl(skinny_pack_x_kernel<C>, dim3(blocks), dim3(kPackThreads), 0, s,
+                         static_cast<const __half*>(X), M, K, xs)) != GLMQ_OK)
+      return st;
   }
-  skinny_kernel<C><<<grid, kSkinnyThreads, C::SMEM_BYTES, s>>>(tw, a);
-  if ((st = launched()) != GLMQ_OK) return st;
+  if ((st = launch_pdl(skinny_kernel<C>, dim3(grid), dim3(kSkinnyThreads), C::SMEM_BYTES, s, tw, a)) != GLMQ_OK)
+    return st;
   if (a.parts > 1) {
     st = (e.bias || e.geglu) ? launch_finalize_epi(a.ws, a.scale, e, a.Y, M, N, s)
                              : launch_finalize(a.ws, a.scale, a.Y, M, N, s);

@@ -106,31 +106,52 @@ __device__ __forceinline__ void skinny_mma_block(uint32_t d, uint32_t a, uint32_
   umma_f16_tmem_a_lh<1>(d, a + 24, b_lo + 6, b_hi, C::IDESC, leader);
 }
 
+// Threads per block of the pre-pass: one such block fits on an SM beside a skinny CTA
+// (4 warps of at most 32 registers in the registers the skinny CTA leaves free).
+constexpr int kPackThreads = 128;
+
 // Pre-pass: X fp16 [M, K] -> the shared-memory image of every activation tile the
 // skinny kernel reads: for 64-wide K block b, BN rows (tokens) of 128 bytes with the
 // 128-byte swizzle (16-byte unit u of row r at (u ^ (r & 7)) * 16), rows >= M zero,
 // INT4 values of each 8-group in the order (0,4,1,5,2,6,3,7). Tiles of consecutive
 // K blocks are contiguous, so a stage's tiles are one contiguous range.
 template <class C>
-__global__ void __launch_bounds__(256) skinny_pack_x_kernel(const __half* __restrict__ X, int M, int K,
-                                                            uint8_t* __restrict__ xs) {
+__global__ void __launch_bounds__(kPackThreads) skinny_pack_x_kernel(const __half* __restrict__ X, int M, int K,
+                                                                     uint8_t* __restrict__ xs) {
+  // Launched with a grid dependency: let the skinny kernel launch now (its CTAs start
+  // streaming weights beside this pass), then wait for the kernel that produced X.
+  griddep_launch_dependents();
+  griddep_wait();
   const long long total = static_cast<long long>(K / 64) * C::kBN * 8;     // 16-byte units
-  for (long long i = blockIdx.x * 256LL + threadIdx.x; i < total; i += static_cast<long long>(gridDim.x) * 256) {
-    const int u = static_cast<int>(i & 7);
-    const long long rk = i >> 3;
-    const int r = static_cast<int>(rk % C::kBN);
-    const long long kb = rk / C::kBN;
-    uint4 o = make_uint4(0, 0, 0, 0);
-    if (r < M) {
-      const uint4 v = __ldg(reinterpret_cast<const uint4*>(X + static_cast<long long>(r) * K + kb * 64 + 8 * u));
-      if constexpr (C::kBits == 4) {
-        o = make_uint4(prmt(v.x, v.z, 0x5410u), prmt(v.x, v.z, 0x7632u), prmt(v.y, v.w, 0x5410u),
-                       prmt(v.y, v.w, 0x7632u));
-      } else {
-        o = v;
-      }
+  const long long stride = static_cast<long long>(gridDim.x) * kPackThreads;
+  constexpr int U = 4;   // units per thread and pass, their loads in flight together
+  for (long long i0 = static_cast<long long>(blockIdx.x) * kPackThreads + threadIdx.x; i0 < total;
+       i0 += U * stride) {
+    uint4 v[U];
+#pragma unroll
+    for (int q = 0; q < U; ++q) {
+      const long long i = i0 + q * stride;
+      const long long rk = i >> 3;
+      const int r = static_cast<int>(rk % C::kBN);
+      v[q] = make_uint4(0, 0, 0, 0);
+      if (i < total && r < M)
+        v[q] = __ldg(reinterpret_cast<const uint4*>(X + static_cast<long long>(r) * K + (rk / C::kBN) * 64 +
+                                                     8 * static_cast<int>(i & 7)));
     }
-    *reinterpret_cast<uint4*>(xs + kb * C::XT_BYTES + r * 128 + ((u ^ (r & 7)) << 4)) = o;
+#pragma unroll
+    for (int q = 0; q < U; ++q) {
+      const long long i = i0 + q * stride;
+      if (i >= total) break;
+      const int u = static_cast<int>(i & 7);
+      const long long rk = i >> 3;
+      const int r = static_cast<int>(rk % C::kBN);
+      const long long kb = rk / C::kBN;
+      uint4 o = v[q];
+      if constexpr (C::kBits == 4)
+        o = make_uint4(prmt(v[q].x, v[q].z, 0x5410u), prmt(v[q].x, v[q].z, 0x7632u), prmt(v[q].y, v[q].w, 0x5410u),
+                       prmt(v[q].y, v[q].w, 0x7632u));
+      *reinterpret_cast<uint4*>(xs + kb * C::XT_BYTES + r * 128 + ((u ^ (r & 7)) << 4)) = o;
+    }
   }
 }
 
@@ -230,6 +251,9 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
     }
   } else if (warp == kSkinnyXWarp) {
     // ------------------------------------------------------------ activation tiles (bulk copies)
+    // The activation image is written by the pre-pass, which may still be running: this
+    // is the one role that waits for the grid dependency before its first access.
+    griddep_wait();
     if (lane == 0) {
       uint32_t armed[SX] = {};
       int r = 0;
@@ -447,6 +471,7 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
     if ((!ok || !drained) && lane == 0) report_error(kErrPrefillWait);
   } else {
     // ------------------------------------------------------------ epilogue warps 12..15
+    griddep_wait();   // (its first output follows the activations anyway)
     const int quarter = warp & 3;
     const bool split = a.parts > 1;
     int it = 0;

@@ -588,12 +588,12 @@ glmq_status launch_skinny_cfg(const DeviceInfo& dev, const void* X, int M, const
   if ((st = allow_smem(skinny_kernel<C>, C::SMEM_BYTES)) != GLMQ_OK) return st;
   const int grid = a.units < dev.sms ? a.units : dev.sms;
   // Both launches carry a grid dependency. The pre-pass (one small block per SM at most,
-  // so a skinny CTA fits beside it) lets the skinny kernel launch at once; the
-  // skinny kernel's weight producer then streams weight boxes while the pre-pass runs,
-  // and only its activation producer (and epilogue) wait for the pre-pass. Reading the
-  // weights, scales and zero points early is safe: the pre-pass let the skinny kernel
-  // launch only after its own grid-dependency wait, i.e. after every earlier kernel
-  // had completed, and the pre-pass writes none of them.
+  // so a skinny CTA fits beside it) waits for the kernels before it and then lets the
+  // skinny kernel launch; the skinny kernel's weight producer streams weight boxes while
+  // the pre-pass runs, and only its activation producer (and epilogue) wait for the
+  // pre-pass. Reading the weights, scales and zero points early is safe: the skinny
+  // kernel launches only after the pre-pass has passed its grid-dependency wait, i.e.
+  // after every earlier kernel has completed, and the pre-pass writes none of them.
   {
     const long long units16 = static_cast<long long>(K / 64) * C::kBN * 8;
     const int blocks = static_cast<int>(std::min<long long>((units16 + kPackThreads - 1) / kPackThreads, dev.sms));

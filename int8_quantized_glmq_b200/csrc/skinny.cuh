@@ -118,10 +118,13 @@ constexpr int kPackThreads = 128;
 template <class C>
 __global__ void __launch_bounds__(kPackThreads) skinny_pack_x_kernel(const __half* __restrict__ X, int M, int K,
                                                                      uint8_t* __restrict__ xs) {
-  // Launched with a grid dependency: let the skinny kernel launch now (its CTAs start
-  // streaming weights beside this pass), then wait for the kernel that produced X.
-  griddep_launch_dependents();
+  // Launched with a grid dependency: wait for the kernels before this one (X, and the
+  // weights the skinny kernel reads without a wait of its own, are written by them),
+  // then let the skinny kernel launch, so that its CTAs start streaming weights beside
+  // this pass. The trigger must follow the wait: a dependent may launch as soon as
+  // every block of this grid has triggered.
   griddep_wait();
+  griddep_launch_dependents();
   const long long total = static_cast<long long>(K / 64) * C::kBN * 8;     // 16-byte units
   const long long stride = static_cast<long long>(gridDim.x) * kPackThreads;
   constexpr int U = 4;   // units per thread and pass, their loads in flight together

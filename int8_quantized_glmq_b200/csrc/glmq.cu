@@ -49,8 +49,10 @@ glmq_status launched() {
 
 // Launches kernel<<<grid, block, smem, s>>>(args...) with programmatic stream
 // serialization: it may begin (its shared-memory prologue) while the previous kernel
-// in the stream drains, and waits for that kernel (griddep_wait) before any
-// global-memory access. Counted like launched().
+// in the stream drains, and waits for that kernel (griddep_wait) before it touches
+// anything an earlier kernel may write. (The finalize pass and the skinny kernel read
+// per-layer constants earlier; finalize.cuh and launch_skinny_cfg state why that is
+// safe.) Counted like launched().
 template <typename... KArgs, typename... Args>
 glmq_status launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
                        Args... args) {
